@@ -1,0 +1,472 @@
+#!/usr/bin/env python3
+"""Benchmark of the Flash PD-SSM hot path on B200.
+
+One step = one pass of the forward path over one batch of synthetic input:
+hard selection (pdssm_select) then the chunked three-phase scan
+(pdssm_scan_fwd: dictionary plans, phase A, phase B, phase C).  Default
+workload: B=8, H=16, N=64, K=16, L=16384, D_in=128, chunk=128, bf16 inputs
+with fp32 state (the bf16-input forward workload).  ``--workload`` selects
+another of the five workloads (e.g. ``fwd_bwd`` adds the exact adjoint).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  ``value`` is whole-job state updates
+(B*H*L*N) per second with inputs resident in HBM; ``e2e`` is the same metric
+with inputs copied from pinned host memory and y / h_last copied back inside
+the timed region.  Multi-GPU runs (torchrun) give every rank its own batch
+(weak scaling, no data-path collective); time is the max over ranks.
+"""
+import argparse
+import hashlib
+import json
+import os
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import pdssm_inputs as gen  # noqa: E402
+
+WORKLOAD_ALIASES = {"tiny": 0, "fp32_mixed": 1, "bf16_select_fwd": 2, "stiff": 3,
+                    "fwd_bwd": 4}
+DEFAULT_WORKLOAD = 2
+METRIC = "PD-scan state-updates/s (B*H*L*N per s)"
+UNIT = "state-updates/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=str(DEFAULT_WORKLOAD))
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    return ap.parse_args()
+
+
+def workload_index(s):
+    return WORKLOAD_ALIASES[s] if s in WORKLOAD_ALIASES else int(s)
+
+
+def updates(cfg):
+    return cfg["B"] * cfg["H"] * cfg["L"] * cfg["N"]
+
+
+def algorithmic_bytes(cfg):
+    """Bytes the forward scan must move per launch: d, b, c read once, k read,
+    y written (h0 / h_last / dictionary are O(B*H*N))."""
+    es = 2 if cfg["dtype"] == "bf16" else 4
+    rows = cfg["B"] * cfg["H"] * cfg["L"]
+    fwd = rows * cfg["N"] * 3 * es + rows * 4 + rows * 4
+    bwd = 0
+    if cfg.get("grad"):
+        # reads d, b, c, k, g_y; writes g_b, g_d, g_c
+        bwd = rows * cfg["N"] * 3 * es + rows * 8 + rows * cfg["N"] * 3 * 4
+    sel = 0
+    if cfg["k_kind"] == "select":
+        sel = cfg["B"] * cfg["L"] * cfg["D_in"] * es + rows * 4
+    return fwd, bwd, sel
+
+
+def config_json(cfg, n_gpus):
+    return {"workload": cfg["name"], "B_per_gpu": cfg["B"], "H": cfg["H"], "N": cfg["N"],
+            "K": cfg["K"], "L": cfg["L"], "D_in": cfg["D_in"], "chunk": cfg["chunk"],
+            "input_dtype": cfg["dtype"], "state_dtype": "f32",
+            "path": "select+scan_fwd" + ("+scan_bwd" if cfg.get("grad") else "")
+            if cfg["k_kind"] == "select" else
+            "scan_fwd" + ("+scan_bwd" if cfg.get("grad") else ""),
+            "parallelism": f"dp{n_gpus} (independent batches)",
+            "l2": "inputs larger than L2, no flush needed"}
+
+
+# ---------------------------------------------------------------------------
+# oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def time_oracle(cfg, inp, budget_s):
+    """Run the plain CPU oracle on successive (b, h) sequences (selection for
+    that batch row's steps included) until the time budget is spent.
+    Returns (updates per second, description of the sample, threads)."""
+    import oracle
+    B, H, L, N = cfg["B"], cfg["H"], cfg["L"], cfg["N"]
+    # window of steps per piece keeps one piece to a few seconds
+    Lw = min(L, 4096)
+    done = 0
+    pieces = 0
+    t0 = time.perf_counter()
+    for bb in range(B):
+        for t_start in range(0, L, Lw):
+            sl = slice(t_start, t_start + Lw)
+            if cfg["k_kind"] == "select":
+                k = oracle.select(inp.u[bb:bb + 1, sl], inp.W)
+            else:
+                k = inp.k[bb:bb + 1, :, sl]
+            h0 = inp.h0[bb:bb + 1] if inp.h0 is not None else None
+            oracle.scan_fwd(inp.pi, k, inp.d[bb:bb + 1, :, sl], inp.b[bb:bb + 1, :, sl],
+                            inp.c[bb:bb + 1, :, sl], h0)
+            if cfg.get("grad"):
+                oracle.scan_bwd(inp.pi, k, inp.d[bb:bb + 1, :, sl], inp.b[bb:bb + 1, :, sl],
+                                inp.c[bb:bb + 1, :, sl], h0, inp.g_y[bb:bb + 1, :, sl])
+            n = H * min(Lw, L - t_start) * N
+            done += n
+            pieces += 1
+            if time.perf_counter() - t0 >= budget_s:
+                break
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    sample = (f"{pieces} piece(s) of batch rows x all {H} heads x <= {Lw} steps "
+              f"({done} state updates, {dt:.1f} s, single thread)")
+    return done / dt, sample, 1
+
+
+# ---------------------------------------------------------------------------
+# clock sampling (NVML, read only)
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    def __init__(self, device_index):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception as e:  # no NVML: report that instead of clocks
+            self.err = str(e)
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception:
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def report(self):
+        if not self.ok:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [f"nvml unavailable: {self.err}"]}
+        nv = self.nv
+        names = {nv.nvmlClocksEventReasonGpuIdle: "gpu_idle",
+                 nv.nvmlClocksEventReasonApplicationsClocksSetting: "applications_clocks_setting",
+                 nv.nvmlClocksEventReasonSwPowerCap: "sw_power_cap",
+                 nv.nvmlClocksEventReasonHwSlowdown: "hw_slowdown",
+                 nv.nvmlClocksEventReasonSyncBoost: "sync_boost",
+                 nv.nvmlClocksEventReasonSwThermalSlowdown: "sw_thermal_slowdown",
+                 nv.nvmlClocksEventReasonHwThermalSlowdown: "hw_thermal_slowdown",
+                 nv.nvmlClocksEventReasonHwPowerBrakeSlowdown: "hw_power_brake_slowdown"}
+        reasons = [v for k, v in names.items() if self.reasons & k]
+        med = float(np.median(self.samples)) if self.samples else None
+        return {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": reasons,
+                "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------
+# helpers
+# ---------------------------------------------------------------------------
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "structured_sparse_state_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, fn), "rb") as f:
+            h.update(fn.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload_name):
+    """Per-launch DRAM bytes of the scan from the committed ncu summary, if it
+    was taken on the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        tab = json.load(f)
+    ent = tab.get(workload_name)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("scan_fwd_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def run_ours(args, cfg):
+    import torch
+    import torch.distributed as dist
+    import structured_sparse_state_b200 as pd
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = gen.generate(cfg)
+    bf = cfg["dtype"] == "bf16"
+
+    def to_dev(x, dt=torch.float32, as_bf16=False):
+        if x is None:
+            return None
+        t = torch.from_numpy(np.ascontiguousarray(x))
+        t = t.to(torch.bfloat16) if as_bf16 else t.to(dt)
+        return t.to(dev)
+
+    pi = to_dev(inp.pi, torch.int32)
+    d, b, c = (to_dev(x, as_bf16=bf) for x in (inp.d, inp.b, inp.c))
+    h0 = to_dev(inp.h0)
+    W = to_dev(inp.W)
+    u = to_dev(inp.u, as_bf16=bf) if inp.u is not None else None
+    k_given = to_dev(inp.k, torch.int32) if inp.k is not None else None
+    g_y = to_dev(inp.g_y)
+    B, H, L, N, K = cfg["B"], cfg["H"], cfg["L"], cfg["N"], cfg["K"]
+    chunk = cfg["chunk"]
+    grad = bool(cfg.get("grad"))
+    select = cfg["k_kind"] == "select"
+    k_buf = torch.empty((B, H, L), dtype=torch.int32, device=dev)
+    y = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    h_last = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    ws = pd.make_workspace(B, H, L, N, K, chunk, dev, False, grad)
+    gouts = None
+    if grad:
+        gouts = (torch.empty_like(d, dtype=torch.float32), torch.empty_like(d, dtype=torch.float32),
+                 torch.empty_like(d, dtype=torch.float32),
+                 torch.empty((B, H, N), dtype=torch.float32, device=dev))
+    stream = torch.cuda.current_stream()
+    launches_per_step = (1 if select else 0) + 4 + (3 if grad else 0)
+
+    ev = None
+
+    def step(i=None):
+        k = pd.pdssm_select(u, W, k_out=k_buf, stream=stream) if select else k_given
+        if ev is not None:
+            ev[i][0].record(stream)
+        pd.pdssm_scan_fwd(pi, k, d, b, c, h0, chunk=chunk, ws=ws, y=y, h_last=h_last,
+                          for_bwd=grad, stream=stream)
+        if ev is not None:
+            ev[i][1].record(stream)
+        if grad:
+            pd.pdssm_scan_bwd(pi, k, d, b, c, h0, g_y, ws, chunk=chunk, out=gouts,
+                              stream=stream)
+
+    # warm-up and a status check of the path
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = pd.pdssm_ws_status(ws)
+    if st != 0:
+        raise RuntimeError(f"device status {st} after warm-up")
+
+    K_steps = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(K_steps)]
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev.index) as clk:
+        start.record(stream)
+        for i in range(K_steps):
+            step(i)
+        end.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms_total = start.elapsed_time(end)
+    scan_ms = sum(a.elapsed_time(bq) for a, bq in ev) / K_steps
+    t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_total = float(t.item())
+    ms_step = ms_total / K_steps
+    upd = updates(cfg)
+    value = upd * world / (ms_step * 1e-3)
+
+    # end to end: pinned host inputs -> device -> path -> y, h_last back to host
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, cfg, pd, torch, dev, stream, inp, bf, pi, W, world, dist)
+
+    if rank != 0:
+        if world > 1:
+            dist.destroy_process_group()
+        return None
+
+    peaks, peak_kind = measured_peaks()
+    fwd_bytes, bwd_bytes, sel_bytes = algorithmic_bytes(cfg)
+    achieved = fwd_bytes / (scan_ms * 1e-3) / 1e9
+    roofline = {"kernel": "pdssm_scan_fwd (plans + phase A + phase B + phase C)",
+                "bound": "hbm", "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": ncu_traffic(cfg["name"]),
+                "algorithmic_bytes_per_launch": fwd_bytes,
+                "launch_ms": round(scan_ms, 5),
+                "select_ms": round(ms_step - scan_ms, 5) if select and not grad else None}
+    out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+           "steps": K_steps, "warmup": args.warmup, "ms_per_step": ms_step,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+           "dtype": "bf16" if bf else "f32", "data": "synthetic (seeded PCG64)",
+           "config": config_json(cfg, world), "roofline": roofline,
+           "gpu_launches": launches_per_step * K_steps, "clocks": clk.report(),
+           "e2e": e2e}
+    if not args.no_cpu and world == 1:
+        v, sample, cores = time_oracle(cfg, inp, args.cpu_seconds)
+        out["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                               "sample": sample}
+    if world > 1:
+        dist.destroy_process_group()
+    return out
+
+
+def run_e2e(args, cfg, pd, torch, dev, stream, inp, bf, pi, W, world, dist):
+    B, H, L, N, K = cfg["B"], cfg["H"], cfg["L"], cfg["N"], cfg["K"]
+    chunk = cfg["chunk"]
+    grad = bool(cfg.get("grad"))
+    select = cfg["k_kind"] == "select"
+
+    def pinned(x, as_bf16=False, dt=torch.float32):
+        if x is None:
+            return None
+        t = torch.from_numpy(np.ascontiguousarray(x))
+        t = t.to(torch.bfloat16) if as_bf16 else t.to(dt)
+        return t.pin_memory()
+
+    hd = {name: pinned(getattr(inp, name), as_bf16=bf) for name in ("d", "b", "c")}
+    hd["u"] = pinned(inp.u, as_bf16=bf) if select else None
+    hd["k"] = pinned(inp.k, dt=torch.int32) if not select else None
+    hd["h0"] = pinned(inp.h0)
+    hd["g_y"] = pinned(inp.g_y)
+    dd = {kname: (torch.empty_like(v, device=dev) if v is not None else None)
+          for kname, v in hd.items()}
+    k_buf = torch.empty((B, H, L), dtype=torch.int32, device=dev)
+    y = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    h_last = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    y_host = torch.empty((B, H, L), dtype=torch.float32).pin_memory()
+    hl_host = torch.empty((B, H, N), dtype=torch.float32).pin_memory()
+    ws = pd.make_workspace(B, H, L, N, K, chunk, dev, False, grad)
+    gouts = None
+    gh = None
+    if grad:
+        gouts = tuple(torch.empty(s, dtype=torch.float32, device=dev)
+                      for s in ((B, H, L, N),) * 3 + ((B, H, N),))
+        gh = tuple(torch.empty(g.shape, dtype=torch.float32).pin_memory() for g in gouts)
+    h2d = sum(v.numel() * v.element_size() for v in hd.values() if v is not None)
+    d2h = y_host.numel() * 4 + hl_host.numel() * 4 + (
+        sum(g.numel() * 4 for g in gh) if grad else 0)
+
+    def step():
+        for kname, v in hd.items():
+            if v is not None:
+                dd[kname].copy_(v, non_blocking=True)
+        k = pd.pdssm_select(dd["u"], W, k_out=k_buf, stream=stream) if select else dd["k"]
+        pd.pdssm_scan_fwd(pi, k, dd["d"], dd["b"], dd["c"], dd["h0"], chunk=chunk, ws=ws, y=y,
+                          h_last=h_last, for_bwd=grad, stream=stream)
+        if grad:
+            pd.pdssm_scan_bwd(pi, k, dd["d"], dd["b"], dd["c"], dd["h0"], dd["g_y"], ws,
+                              chunk=chunk, out=gouts, stream=stream)
+            for g, hgt in zip(gouts, gh):
+                hgt.copy_(g, non_blocking=True)
+        y_host.copy_(y, non_blocking=True)
+        hl_host.copy_(h_last, non_blocking=True)
+
+    for _ in range(max(1, min(args.warmup, 3))):
+        step()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 20))
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize()
+    ms = start.elapsed_time(end) / steps
+    t = torch.tensor([ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms = float(t.item())
+    return {"value": updates(cfg) * world / (ms * 1e-3), "unit": UNIT,
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "ms_per_step": ms, "steps": steps}
+
+
+# ---------------------------------------------------------------------------
+# reference arm: the CPU oracle, as it stands, on a bounded sample
+# ---------------------------------------------------------------------------
+def run_reference(args, cfg):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return None
+    inp = gen.generate(cfg)
+    budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    vals = []
+    sample = None
+    for i in range(args.warmup + args.steps):
+        v, sample, cores = time_oracle(cfg, inp, budget)
+        if i >= args.warmup:
+            vals.append(v)
+    v = float(np.mean(vals)) if vals else 0.0
+    upd = updates(cfg)
+    return {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": upd / v * 1e3 if v else None, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64 (oracle arithmetic)", "data": "synthetic (seeded PCG64)",
+            "config": config_json(cfg, 1),
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"per step: {sample}"},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+
+
+def main():
+    args = parse()
+    cfg = gen.workload(workload_index(args.workload))
+    if args.impl == "reference":
+        out = run_reference(args, cfg)
+    else:
+        out = run_ours(args, cfg)
+    if out is not None:
+        print(json.dumps(out), flush=True)
+
+
+if __name__ == "__main__":
+    main()

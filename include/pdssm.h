@@ -1,0 +1,180 @@
+/*
+ * pdssm.h -- C ABI of the B200 (sm_100a) Flash PD-SSM scan library.
+ *
+ * The recurrence (Flash PD-SSM technical summary, Methodology §1 "hard
+ * selection", one-hot column selector; benchmark spec of the path):
+ *
+ *     k_t    = argmax_k (W_sel u_t)_k
+ *     h_t    = P_{k_t} diag(d_t) h_{t-1} + b_t,   P_k[pi_k(j), j] = 1
+ *     y_t    = <c_t, h_t>
+ *
+ * per (batch b, head h), evaluated as a chunked scan in three phases
+ * (Methodology §3: A chunk-local recurrence, B carry prefix scan, C carry
+ * correction), with its exact adjoint (Breaking the Memory Wall / PGF,
+ * abstract: exact analytical derivatives by chunked evolution, memory
+ * independent of L apart from per-chunk carries).
+ *
+ * Conventions for every call
+ * --------------------------
+ *  * All tensor pointers are DEVICE pointers to caller-owned, row-major,
+ *    contiguous memory.  The library allocates nothing and keeps no state
+ *    between calls; scratch lives in the caller's workspace `ws`.
+ *  * Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
+ *    default stream).  A returned PDSSM_OK means the kernels were launched;
+ *    device-side problems are recorded in the workspace status word and read
+ *    back with pdssm_ws_status().  pdssm_validate() and pdssm_ws_status()
+ *    synchronise the stream.
+ *  * Shapes:   u [B][L][D_in]        W_sel [H][K][D_in] (fp32)
+ *              pi_dict: entry (h,k,j) at pi_dict[h*pi_head_stride + k*N + j]
+ *                       (pi_head_stride = 0: one [K][N] dictionary for all heads,
+ *                        = K*N: one per head)
+ *              k [B][H][L] int32      d, b, c [B][H][L][N] (fp32 or bf16)
+ *              h0, h_last [B][H][N] fp32     y [B][H][L] fp32
+ *              g_y [B][H][L] fp32     g_b, g_d, g_c [B][H][L][N] fp32
+ *              g_hlast, g_h0 [B][H][N] fp32
+ *  * Limits: 1 <= N <= 64, 1 <= K <= 32, 1 <= D_in <= 256, chunk >= 1,
+ *    B, H >= 1, L >= 0.  L need not be a multiple of chunk.
+ *  * Errors: NULL required pointers, bad sizes or a too-small workspace give
+ *    PDSSM_ERR_INVALID_ARG / PDSSM_ERR_WORKSPACE before anything is launched;
+ *    sizes beyond the limits give PDSSM_ERR_UNSUPPORTED; a failed launch
+ *    gives PDSSM_ERR_CUDA.  Out-of-range k or pi values are clamped by the
+ *    kernels (memory-safe) and flagged PDSSM_ERR_BAD_INDEX in the status word;
+ *    pdssm_validate() checks them up front.
+ */
+#ifndef PDSSM_H
+#define PDSSM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct pdssm_dims {
+    int64_t B, H, L, N, K, D_in;   /* D_in is used by pdssm_select only */
+} pdssm_dims;
+
+typedef enum pdssm_dtype { PDSSM_F32 = 0, PDSSM_BF16 = 1 } pdssm_dtype;
+
+typedef enum pdssm_status {
+    PDSSM_OK = 0,
+    PDSSM_ERR_INVALID_ARG = 1,
+    PDSSM_ERR_UNSUPPORTED = 2,
+    PDSSM_ERR_BAD_INDEX = 3,
+    PDSSM_ERR_CUDA = 4,
+    PDSSM_ERR_TIMEOUT = 5,
+    PDSSM_ERR_WORKSPACE = 6
+} pdssm_status;
+
+/* Human-readable name of a status code.  Never NULL. */
+const char *pdssm_status_str(int status);
+
+/* Text of the last error seen by a call on this host thread ("" if none).
+ * Owned by the library; valid until the next call on the same thread. */
+const char *pdssm_last_error(void);
+
+/* Library ABI version (major * 100 + minor). */
+int pdssm_version(void);
+
+/*
+ * Workspace bytes needed by pdssm_scan_fwd (for_bwd = 0) or by the pair
+ * pdssm_scan_fwd + pdssm_scan_bwd (for_bwd = 1) at these sizes.  The
+ * workspace holds the gather plans of the dictionary (phase A0), the chunk
+ * transfers (Pi_c, Delta_c, v_c), the carries H_c and a status word:
+ * O(B*H*ceil(L/chunk)*N), i.e. 1/chunk of the size of d.  Returns 0 when the
+ * arguments are invalid.  Pure host function.
+ */
+size_t pdssm_workspace_bytes(const pdssm_dims *dims, int64_t pi_head_stride,
+                             int64_t chunk, int for_bwd);
+
+/*
+ * Hard selection (Flash PD-SSM technical summary, Methodology §1): for every
+ * (b, h, t),  k_out[b][h][t] = first index of the largest logit
+ *     l_k = sum_{q < D_in} W_sel[h][k][q] * u[b][t][q],
+ * each logit evaluated as the fp32 chain acc = fmaf(W, u, acc) in ascending q
+ * from acc = 0 (bf16 u is upcast exactly).  This fixed arithmetic makes k
+ * reproducible bit for bit on any IEEE machine.
+ * u: device [B][L][D_in] of u_dtype; W_sel: device fp32 [H][K][D_in];
+ * k_out: device int32 [B][H][L].  Needs no workspace.
+ */
+pdssm_status pdssm_select(const pdssm_dims *dims, const void *u,
+                          pdssm_dtype u_dtype, const float *W_sel,
+                          int32_t *k_out, void *stream);
+
+/*
+ * Chunked forward scan (Methodology §3).  Runs phase A0 (gather plans of the
+ * dictionary), A (per chunk: local readout of the state started from zero,
+ * closed PD transfer Pi_c, Delta_c, v_c), B (carry prefix scan H_c, h_last)
+ * and C (carry correction of the readout y).  Writes y [B][H][L] and, when
+ * non-NULL, h_last [B][H][N] = h_{L-1} (h0 when L = 0).  h0 may be NULL
+ * (zero initial state).  ws must hold pdssm_workspace_bytes(dims,
+ * pi_head_stride, chunk, 0) bytes, 256-byte aligned; its contents are
+ * overwritten.  d, b, c share in_dtype.
+ */
+pdssm_status pdssm_scan_fwd(const pdssm_dims *dims, const int32_t *pi_dict,
+                            int64_t pi_head_stride, const int32_t *k,
+                            const void *d, const void *b, const void *c,
+                            pdssm_dtype in_dtype, const float *h0, float *y,
+                            float *h_last, int64_t chunk, void *ws,
+                            size_t ws_bytes, void *stream);
+
+/*
+ * Exact adjoint of pdssm_scan_fwd (PGF: reverse evolution, per-chunk
+ * recompute) for the loss  sum_t g_y[t] y_t + <g_hlast, h_last>:
+ *     lambda_t = g_y[t] c_t + M_{t+1}^T lambda_{t+1},  (M^T x)[j] = d[j] x[pi(j)]
+ *     g_b_t = lambda_t,  g_c_t = g_y[t] h_t,
+ *     g_d_t[j] = h_{t-1}[j] lambda_t[pi_{k_t}(j)],  g_h0 = M_0^T lambda_0.
+ * Must follow pdssm_scan_fwd on the same stream with identical arguments and
+ * the SAME workspace, untouched in between, sized with for_bwd = 1: the
+ * forward's chunk transfers and carries are the backward's checkpoints; h is
+ * recomputed inside each chunk.  g_hlast may be NULL (zero).  g_h0 may be
+ * NULL (not written).  Writes g_b, g_d, g_c and g_h0 (fp32).
+ */
+pdssm_status pdssm_scan_bwd(const pdssm_dims *dims, const int32_t *pi_dict,
+                            int64_t pi_head_stride, const int32_t *k,
+                            const void *d, const void *b, const void *c,
+                            pdssm_dtype in_dtype, const float *h0,
+                            const float *g_y, const float *g_hlast,
+                            float *g_b, float *g_d, float *g_c, float *g_h0,
+                            int64_t chunk, void *ws, size_t ws_bytes,
+                            void *stream);
+
+/*
+ * Phase A alone, exposing each chunk's closed PD transfer (for tests of the
+ * composed index maps, which must match bit for bit):
+ *     h_e = P_{Pi_c} diag(Delta_c) h_{s-1} + v_c   for the chunk s..e.
+ * Pi_out int32, Delta_out and v_out fp32, each [B][H][ceil(L/chunk)][N],
+ * device.  ws as for pdssm_scan_fwd (for_bwd = 0).
+ */
+pdssm_status pdssm_chunk_transfers(const pdssm_dims *dims,
+                                   const int32_t *pi_dict,
+                                   int64_t pi_head_stride, const int32_t *k,
+                                   const void *d, const void *b,
+                                   pdssm_dtype in_dtype, int64_t chunk,
+                                   int32_t *Pi_out, float *Delta_out,
+                                   float *v_out, void *ws, size_t ws_bytes,
+                                   void *stream);
+
+/*
+ * Checks every dictionary entry lies in [0, N) and every k in [0, K) on the
+ * device, then synchronises the stream.  Returns PDSSM_ERR_BAD_INDEX if any
+ * does not.  Uses the first 256 bytes of ws (ws_bytes >= 256).
+ */
+pdssm_status pdssm_validate(const pdssm_dims *dims, const int32_t *pi_dict,
+                            int64_t pi_head_stride, const int32_t *k,
+                            void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Synchronises the stream, reads the workspace status word written by the
+ * kernels (PDSSM_ERR_BAD_INDEX for a clamped index, PDSSM_ERR_TIMEOUT for a
+ * staging wait that gave up) and clears it.  PDSSM_OK when nothing was
+ * recorded.
+ */
+pdssm_status pdssm_ws_status(void *ws, size_t ws_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* PDSSM_H */

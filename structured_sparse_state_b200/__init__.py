@@ -1,0 +1,290 @@
+"""Flash PD-SSM structured-sparse scan on B200 (sm_100a).
+
+Thin Python binding of ``libpdssm.so``: every function here only checks and
+marshals PyTorch tensors (device memory, the current stream) into the C ABI
+declared in ``include/pdssm.h``; all arithmetic runs in the CUDA kernels.
+There is no CPU path: importing this package without the built library, or
+calling it with CPU tensors, raises.
+
+    k = pdssm_select(u, W_sel)                          # hard selection
+    y, h_last, ws = pdssm_scan_fwd(pi, k, d, b, c, h0, chunk=128, for_bwd=True)
+    g_b, g_d, g_c, g_h0 = pdssm_scan_bwd(pi, k, d, b, c, h0, g_y, ws=ws, chunk=128)
+
+Page sources: Flash PD-SSM technical summary, Methodology §1 (hard
+selection, one-hot column selector) and §3 (three-phase chunked kernel);
+Breaking the Memory Wall (PGF), abstract (exact chunked adjoint).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libpdssm.so")
+
+PDSSM_F32, PDSSM_BF16 = 0, 1
+STATUS = {0: "PDSSM_OK", 1: "PDSSM_ERR_INVALID_ARG", 2: "PDSSM_ERR_UNSUPPORTED",
+          3: "PDSSM_ERR_BAD_INDEX", 4: "PDSSM_ERR_CUDA", 5: "PDSSM_ERR_TIMEOUT",
+          6: "PDSSM_ERR_WORKSPACE"}
+
+# every entry point declared in include/pdssm.h
+EXPORTS = ("pdssm_status_str", "pdssm_last_error", "pdssm_version",
+           "pdssm_workspace_bytes", "pdssm_select", "pdssm_scan_fwd",
+           "pdssm_scan_bwd", "pdssm_chunk_transfers", "pdssm_validate",
+           "pdssm_ws_status")
+
+
+class Dims(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("L", ctypes.c_int64),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("D_in", ctypes.c_int64)]
+
+
+class PdssmError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({last_error()})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with "
+            "`python -m structured_sparse_state_b200.build` (there is no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    D = ctypes.POINTER(Dims)
+    sig = {
+        "pdssm_status_str": (ctypes.c_char_p, [I32]),
+        "pdssm_last_error": (ctypes.c_char_p, []),
+        "pdssm_version": (I32, []),
+        "pdssm_workspace_bytes": (SZ, [D, I64, I64, I32]),
+        "pdssm_select": (I32, [D, P, I32, P, P, P]),
+        "pdssm_scan_fwd": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, I64, P, SZ, P]),
+        "pdssm_scan_bwd": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, P, P, P, P, I64, P,
+                                 SZ, P]),
+        "pdssm_chunk_transfers": (I32, [D, P, I64, P, P, P, I32, I64, P, P, P, P, SZ, P]),
+        "pdssm_validate": (I32, [D, P, I64, P, P, SZ, P]),
+        "pdssm_ws_status": (I32, [P, SZ, P]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    return lib
+
+
+class _Lazy:
+    """Loads libpdssm.so on first use, so the build step can import this
+    package before the library exists; any call without it raises."""
+    _cdll = None
+
+    def __getattr__(self, name):
+        if _Lazy._cdll is None:
+            _Lazy._cdll = _load()
+        return getattr(_Lazy._cdll, name)
+
+
+_lib = _Lazy()
+
+
+def lib():
+    """The loaded C library (for callers that want the raw ABI)."""
+    _lib.pdssm_version        # force the load
+    return _Lazy._cdll
+
+
+def last_error() -> str:
+    return (_lib.pdssm_last_error() or b"").decode()
+
+
+def version() -> int:
+    return int(_lib.pdssm_version())
+
+
+# ----------------------------------------------------------------------------
+# marshalling helpers
+# ----------------------------------------------------------------------------
+def _check(code: int, what: str):
+    if code != 0:
+        raise PdssmError(code, what)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _cuda(t: torch.Tensor, name: str, dtypes) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path)")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected one of {dtypes}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    return PDSSM_BF16 if t.dtype == torch.bfloat16 else PDSSM_F32
+
+
+def _dict_stride(pi: torch.Tensor, H: int, K: int, N: int) -> int:
+    if pi.dim() == 2:
+        if tuple(pi.shape) != (K, N):
+            raise ValueError(f"pi_dict shape {tuple(pi.shape)} != ({K}, {N})")
+        return 0
+    if tuple(pi.shape) != (H, K, N):
+        raise ValueError(f"pi_dict shape {tuple(pi.shape)} != ({H}, {K}, {N})")
+    return K * N
+
+
+def dims(B, H, L, N, K, D_in=0) -> Dims:
+    return Dims(int(B), int(H), int(L), int(N), int(K), int(D_in))
+
+
+# ----------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ----------------------------------------------------------------------------
+def pdssm_workspace_bytes(B, H, L, N, K, chunk, per_head_dict=False, for_bwd=False) -> int:
+    dm = dims(B, H, L, N, K)
+    n = _lib.pdssm_workspace_bytes(ctypes.byref(dm), K * N if per_head_dict else 0,
+                                   int(chunk), int(bool(for_bwd)))
+    if n == 0:
+        raise PdssmError(1, "pdssm_workspace_bytes")
+    return int(n)
+
+
+def pdssm_select(u: torch.Tensor, W_sel: torch.Tensor, k_out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """k[b, h, t] = first argmax_k of the fp32 fma chain sum_q W_sel[h,k,q] u[b,t,q]."""
+    _cuda(u, "u", (torch.float32, torch.bfloat16))
+    _cuda(W_sel, "W_sel", (torch.float32,))
+    B, L, D = u.shape
+    H, K, D2 = W_sel.shape
+    if D != D2:
+        raise ValueError("u and W_sel disagree on D_in")
+    if k_out is None:
+        k_out = torch.empty((B, H, L), dtype=torch.int32, device=u.device)
+    _cuda(k_out, "k_out", (torch.int32,))
+    dm = dims(B, H, L, 0, K, D)
+    _check(_lib.pdssm_select(ctypes.byref(dm), _ptr(u), _dtype_code(u), _ptr(W_sel),
+                             _ptr(k_out), _stream(stream)), "pdssm_select")
+    return k_out
+
+
+def _scan_shapes(pi, k, d, b, c):
+    _cuda(d, "d", (torch.float32, torch.bfloat16))
+    B, H, L, N = d.shape
+    for name, t in (("b", b), ("c", c)):
+        if t is None:
+            continue
+        _cuda(t, name, (d.dtype,))
+        if t.shape != d.shape:
+            raise ValueError(f"{name} shape {tuple(t.shape)} != d shape {tuple(d.shape)}")
+    _cuda(k, "k", (torch.int32,))
+    if tuple(k.shape) != (B, H, L):
+        raise ValueError("k must be [B, H, L]")
+    _cuda(pi, "pi_dict", (torch.int32,))
+    K = pi.shape[-2]
+    stride = _dict_stride(pi, H, K, N)
+    return B, H, L, N, K, stride
+
+
+def make_workspace(B, H, L, N, K, chunk, device, per_head_dict=False, for_bwd=False):
+    n = pdssm_workspace_bytes(B, H, L, N, K, chunk, per_head_dict, for_bwd)
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def pdssm_scan_fwd(pi_dict, k, d, b, c, h0=None, chunk=128, ws=None, y=None, h_last=None,
+                   for_bwd=False, stream=None):
+    """Chunked three-phase forward scan; returns (y, h_last, ws)."""
+    B, H, L, N, K, stride = _scan_shapes(pi_dict, k, d, b, c)
+    dev = d.device
+    if ws is None:
+        ws = make_workspace(B, H, L, N, K, chunk, dev, stride != 0, for_bwd)
+    _cuda(ws, "ws", (torch.uint8,))
+    if h0 is not None:
+        _cuda(h0, "h0", (torch.float32,))
+    if y is None:
+        y = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    if h_last is None:
+        h_last = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dm = dims(B, H, L, N, K)
+    _check(_lib.pdssm_scan_fwd(ctypes.byref(dm), _ptr(pi_dict), stride, _ptr(k), _ptr(d),
+                               _ptr(b), _ptr(c), _dtype_code(d), _ptr(h0), _ptr(y),
+                               _ptr(h_last), int(chunk), _ptr(ws), ws.numel(),
+                               _stream(stream)), "pdssm_scan_fwd")
+    return y, h_last, ws
+
+
+def pdssm_scan_bwd(pi_dict, k, d, b, c, h0, g_y, ws, chunk=128, g_hlast=None, out=None,
+                   stream=None):
+    """Exact adjoint; ws must be the forward's (sized with for_bwd=True).
+    Returns (g_b, g_d, g_c, g_h0)."""
+    B, H, L, N, K, stride = _scan_shapes(pi_dict, k, d, b, c)
+    dev = d.device
+    _cuda(ws, "ws", (torch.uint8,))
+    _cuda(g_y, "g_y", (torch.float32,))
+    if h0 is not None:
+        _cuda(h0, "h0", (torch.float32,))
+    if g_hlast is not None:
+        _cuda(g_hlast, "g_hlast", (torch.float32,))
+    if out is None:
+        out = (torch.empty((B, H, L, N), dtype=torch.float32, device=dev),
+               torch.empty((B, H, L, N), dtype=torch.float32, device=dev),
+               torch.empty((B, H, L, N), dtype=torch.float32, device=dev),
+               torch.empty((B, H, N), dtype=torch.float32, device=dev))
+    g_b, g_d, g_c, g_h0 = out
+    dm = dims(B, H, L, N, K)
+    _check(_lib.pdssm_scan_bwd(ctypes.byref(dm), _ptr(pi_dict), stride, _ptr(k), _ptr(d),
+                               _ptr(b), _ptr(c), _dtype_code(d), _ptr(h0), _ptr(g_y),
+                               _ptr(g_hlast), _ptr(g_b), _ptr(g_d), _ptr(g_c), _ptr(g_h0),
+                               int(chunk), _ptr(ws), ws.numel(), _stream(stream)),
+           "pdssm_scan_bwd")
+    return g_b, g_d, g_c, g_h0
+
+
+def pdssm_chunk_transfers(pi_dict, k, d, b, chunk, ws=None, stream=None):
+    """Phase A transfers (Pi int32, Delta fp32, v fp32), each [B, H, C, N]."""
+    B, H, L, N, K, stride = _scan_shapes(pi_dict, k, d, b, None)
+    dev = d.device
+    C = (L + chunk - 1) // chunk
+    if ws is None:
+        ws = make_workspace(B, H, L, N, K, chunk, dev, stride != 0)
+    Pi = torch.empty((B, H, C, N), dtype=torch.int32, device=dev)
+    Dl = torch.empty((B, H, C, N), dtype=torch.float32, device=dev)
+    v = torch.empty((B, H, C, N), dtype=torch.float32, device=dev)
+    dm = dims(B, H, L, N, K)
+    _check(_lib.pdssm_chunk_transfers(ctypes.byref(dm), _ptr(pi_dict), stride, _ptr(k),
+                                      _ptr(d), _ptr(b), _dtype_code(d), int(chunk), _ptr(Pi),
+                                      _ptr(Dl), _ptr(v), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "pdssm_chunk_transfers")
+    return Pi, Dl, v
+
+
+def pdssm_validate(pi_dict, k, N, ws=None, stream=None) -> int:
+    """Returns the status code (0 = all indices in range).  Synchronises."""
+    _cuda(pi_dict, "pi_dict", (torch.int32,))
+    _cuda(k, "k", (torch.int32,))
+    B, H, L = k.shape
+    K = pi_dict.shape[-2]
+    stride = _dict_stride(pi_dict, H, K, N)
+    if ws is None:
+        ws = torch.empty(256, dtype=torch.uint8, device=k.device)
+    dm = dims(B, H, L, N, K)
+    return int(_lib.pdssm_validate(ctypes.byref(dm), _ptr(pi_dict), stride, _ptr(k), _ptr(ws),
+                                   ws.numel(), _stream(stream)))
+
+
+def pdssm_ws_status(ws, stream=None) -> int:
+    """Reads and clears the workspace status word (synchronises)."""
+    _cuda(ws, "ws", (torch.uint8,))
+    return int(_lib.pdssm_ws_status(_ptr(ws), ws.numel(), _stream(stream)))

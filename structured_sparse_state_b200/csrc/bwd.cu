@@ -1,0 +1,590 @@
+// Exact adjoint of the chunked PD scan (Breaking the Memory Wall / PGF,
+// abstract and framework stages: chunk the sequence, evolve each chunk,
+// take derivatives from the transfers, combine the chunks).
+//
+// With M_t = P_{k_t} diag(d_t) and lambda_t = dl/dh_t:
+//   lambda_t = g_y[t] c_t + M_{t+1}^T lambda_{t+1},   (M^T x)[j] = d[j] x[pi(j)]
+// -- a gather, so the reverse recurrence needs no scatter plan.
+// Per chunk s..e the gradient leaving the chunk towards h_{s-1} is
+//   Lambda_{c-1} = w_c + diag(Delta_c) P_{Pi_c}^T Lambda_c,
+// i.e. Lambda_{c-1}[j] = w_c[j] + Delta_c[j] * Lambda_c[Pi_c[j]], with
+// w_c = M_s^T lambda^loc_s from the chunk's own readouts.  The forward's
+// (Pi_c, Delta_c) are reused; h inside a chunk is recomputed from H_{c-1}.
+//   bwd phase A  w_c per chunk (reverse sweep from a zero carry)
+//   bwd phase B  Lambda_c for every chunk and g_h0 = Lambda_{-1}
+//   bwd phase C  recompute h, sweep back, emit g_b, g_c, g_d.
+#include "common.cuh"
+
+namespace pdssm {
+
+__host__ __device__ inline int bwd_warp_smem_bytes(int ns, int nt, int rowb) {
+    // ring + pbuf (2 x 64) + lbuf (2 x 64) + checkpoints (16 x 64) + barriers
+    return ns * nt * kTS * rowb + 4 * kMaxN * 4 + (kBwdMaxChunk / kTS) * kMaxN * 4 +
+           kMaxStages * 8;
+}
+
+template <int NPL, bool EVEN>
+__device__ __forceinline__ void store_row(float *row, int lane, int N, const float (&v)[NPL]) {
+    if constexpr (NPL == 1) {
+        if (lane < N) row[lane] = v[0];
+    } else {
+        const int e0 = 2 * lane;
+        if constexpr (EVEN) {
+            if (e0 < N) *reinterpret_cast<float2 *>(row + e0) = make_float2(v[0], v[1]);
+        } else {
+            if (e0 < N) row[e0] = v[0];
+            if (e0 + 1 < N) row[e0 + 1] = v[1];
+        }
+    }
+}
+
+// Gather of one forward PD step (same plan format as the forward kernels).
+template <int NPL>
+__device__ __forceinline__ void fwd_step(float (&h)[NPL], const float (&dv)[NPL],
+                                         const float (&bv)[NPL], float *pb,
+                                         const int16_t *__restrict__ prow, int lane, int N) {
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        const int e = lane * NPL + r;
+        if (e < N) pb[e] = dv[r] * h[r];
+    }
+    __syncwarp();
+    float acc[NPL];
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) acc[r] = 0.f;
+    const uint4 q0 = __ldg(reinterpret_cast<const uint4 *>(prow));
+    const int G = (int)(int16_t)(q0.x & 0xffffu);
+    const int ent[7] = {(int)(int16_t)(q0.x >> 16), (int)(int16_t)(q0.y & 0xffffu),
+                        (int)(int16_t)(q0.y >> 16), (int)(int16_t)(q0.z & 0xffffu),
+                        (int)(int16_t)(q0.z >> 16), (int)(int16_t)(q0.w & 0xffffu),
+                        (int)(int16_t)(q0.w >> 16)};
+#pragma unroll
+    for (int g = 0; g < 7; ++g) {
+        if (g < G) {
+            const int e = ent[g];
+            if (e >= 0) {
+                const float val = pb[e & 127];
+                if (NPL == 1 || (e >> 7) == 0)
+                    acc[0] += val;
+                else
+                    acc[NPL - 1] += val;
+            }
+        }
+    }
+    for (int g0 = 8; g0 <= G; g0 += 8) {
+        const uint4 q = __ldg(reinterpret_cast<const uint4 *>(prow + g0));
+        const int en[8] = {(int)(int16_t)(q.x & 0xffffu), (int)(int16_t)(q.x >> 16),
+                           (int)(int16_t)(q.y & 0xffffu), (int)(int16_t)(q.y >> 16),
+                           (int)(int16_t)(q.z & 0xffffu), (int)(int16_t)(q.z >> 16),
+                           (int)(int16_t)(q.w & 0xffffu), (int)(int16_t)(q.w >> 16)};
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+            if (g0 + g <= G) {
+                const int e = en[g];
+                if (e >= 0) {
+                    const float val = pb[e & 127];
+                    if (NPL == 1 || (e >> 7) == 0)
+                        acc[0] += val;
+                    else
+                        acc[NPL - 1] += val;
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) h[r] = acc[r] + bv[r];
+}
+
+// ---------------------------------------------------------------------------
+// bwd phase A: w_c = M_s^T lambda^loc_s with lambda^loc from a zero carry
+// ---------------------------------------------------------------------------
+template <typename T, int NPL, bool EVEN>
+__global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
+    extern __shared__ __align__(128) unsigned char sm_ba[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
+    if (unit >= p.units) return;
+    const int N = (int)p.N, K = (int)p.K;
+    const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
+    const int64_t hh = bh % p.H;
+    const int64_t s = cidx * p.chunk;
+    const int len = (int)imin64(p.chunk, p.L - s);
+
+    unsigned char *wbase = sm_ba + (size_t)warp * p.smem_per_warp;
+    const int rowb = N * (int)sizeof(T);
+    Ring<2> ring;
+    ring.buf = wbase;
+    ring.rowb = rowb;
+    ring.esz = (int)sizeof(T);
+    ring.tens_bytes = kTS * rowb;
+    ring.stage_bytes = 2 * ring.tens_bytes;
+    ring.ns = p.ns;
+    ring.bulk = p.bulk != 0;
+    float *lbuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes);
+    ring.bar0 = smem_u32(lbuf + 2 * kMaxN);
+    const int64_t seq_row0 = bh * p.L;
+    ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * rowb;
+    ring.src[1] = reinterpret_cast<const unsigned char *>(p.c) + seq_row0 * rowb;
+    ring_init_bars(ring.bar0, p.ns, lane);
+
+    const int ntiles = (len + kTS - 1) / kTS;
+    auto tile_of = [&](int j) { return ntiles - 1 - j; };   // reverse order
+    for (int j = 0; j < p.ns && j < ntiles; ++j) {
+        const int ti = tile_of(j);
+        ring.issue(j, s + (int64_t)ti * kTS, min(kTS, len - ti * kTS), 2, lane);
+    }
+    const int32_t *dict = p.dict + hh * p.dict_hs;
+    const int64_t kbase = bh * p.L + s;
+    float mu[NPL];
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) mu[r] = 0.f;
+    int t0 = (ntiles - 1) * kTS;
+    int kreg = load_k(p.k, kbase + t0 + lane, lane < kTS && t0 + lane < len, K, p.status);
+    float gyreg = (lane < kTS && t0 + lane < len) ? p.g_y[kbase + t0 + lane] : 0.f;
+
+    for (int j = 0; j < ntiles; ++j) {
+        const int stage = j % p.ns;
+        if (!ring.wait(stage, (uint32_t)((j / p.ns) & 1))) {
+            ring_abort(ring, j, min(ntiles, j + p.ns), p.status, lane);
+            return;
+        }
+        const int ti = tile_of(j);
+        t0 = ti * kTS;
+        const int n = min(kTS, len - t0);
+        const int tp = t0 - kTS;   // previous tile (processed next)
+        const bool vp = lane < kTS && tp >= 0;
+        const int knext = load_k(p.k, kbase + tp + lane, vp, K, p.status);
+        const float gynext = vp ? p.g_y[kbase + tp + lane] : 0.f;
+        const T *td = reinterpret_cast<const T *>(ring.tile(stage, 0));
+        const T *tc = reinterpret_cast<const T *>(ring.tile(stage, 1));
+#pragma unroll
+        for (int q = kTS - 1; q >= 0; --q) {
+            if (q < n) {
+                const int kk = __shfl_sync(kFull, kreg, q);
+                const float gy = __shfl_sync(kFull, gyreg, q);
+                float dv[NPL], cv[NPL];
+                load_row<T, NPL, EVEN>(td + q * N, lane, N, dv);
+                load_row<T, NPL, EVEN>(tc + q * N, lane, N, cv);
+                float *lb = lbuf + (q & 1) * kMaxN;
+#pragma unroll
+                for (int r = 0; r < NPL; ++r) {
+                    const int e = lane * NPL + r;
+                    if (e < N) lb[e] = gy * cv[r] + mu[r];
+                }
+                __syncwarp();
+                const int32_t *pk = dict + (int64_t)kk * N;
+#pragma unroll
+                for (int r = 0; r < NPL; ++r) {
+                    const int e = lane * NPL + r;
+                    if (e < N) mu[r] = dv[r] * lb[__ldg(pk + e)];
+                }
+            }
+        }
+        __syncwarp();
+        if (j + p.ns < ntiles) {
+            const int tn = tile_of(j + p.ns);
+            ring.issue(stage, s + (int64_t)tn * kTS, min(kTS, len - tn * kTS), 2, lane);
+        }
+        kreg = knext;
+        gyreg = gynext;
+    }
+    const int64_t o = unit * p.N;
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        const int e = lane * NPL + r;
+        if (e < N) p.wc[o + e] = mu[r];
+    }
+}
+
+// ---------------------------------------------------------------------------
+// bwd phase B: reverse carry scan.  R_c(x)[j] = w_c[j] + Delta_c[j] x[Pi_c[j]]
+// maps Lambda_c to Lambda_{c-1}; compositions stay gathers:
+//   (R_a o R_b): w = w_a + Delta_a * w_b[Pi_a], Delta = Delta_a * Delta_b[Pi_a],
+//                Pi = Pi_b[Pi_a].
+// ---------------------------------------------------------------------------
+template <int NPL>
+__device__ __forceinline__ void load_rev(const ChunkParams &p, int64_t unit, int lane,
+                                         int (&P)[NPL], float (&D)[NPL], float (&W)[NPL]) {
+    const int64_t o = unit * p.N;
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        const int e = lane * NPL + r;
+        if (e < p.N) {
+            P[r] = p.Pi[o + e];
+            D[r] = p.Dl[o + e];
+            W[r] = p.wc[o + e];
+        } else {
+            P[r] = 0;
+            D[r] = 0.f;
+            W[r] = 0.f;
+        }
+    }
+}
+
+template <int NPL>
+__device__ __forceinline__ void apply_gather(const int (&P)[NPL], const float (&D)[NPL],
+                                             const float (&W)[NPL], float (&x)[NPL], float *sX,
+                                             int N, int lane) {
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        const int e = lane * NPL + r;
+        if (e < N) sX[e] = x[r];
+    }
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) x[r] = W[r] + D[r] * sX[P[r]];
+    __syncwarp();
+}
+
+template <int NPL>
+__global__ void k_bwdB(const ChunkParams p) {
+    extern __shared__ __align__(16) unsigned char sm_bb[];
+    const int nw = blockDim.x >> 5;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int N = (int)p.N;
+    const int64_t bh = blockIdx.x;
+    const int64_t C = p.C;
+    float *sXall = reinterpret_cast<float *>(sm_bb);             // [nw][64]
+    int *sPall = reinterpret_cast<int *>(sXall + nw * kMaxN);     // [nw][64]
+    float *sDall = reinterpret_cast<float *>(sPall + nw * kMaxN); // [nw][64]
+    int *aggP = reinterpret_cast<int *>(sDall + nw * kMaxN);
+    float *aggD = reinterpret_cast<float *>(aggP + nw * kMaxN);
+    float *aggW = aggD + nw * kMaxN;
+    float *carry = aggW + nw * kMaxN;
+    float *sX = sXall + warp * kMaxN;
+    int *sP = sPall + warp * kMaxN;
+    float *sD = sDall + warp * kMaxN;
+    const int64_t c0 = C * warp / nw, c1 = C * (warp + 1) / nw;
+    const int64_t u0 = bh * C;
+
+    if (c0 < c1) {
+        int aP[NPL];
+        float aD[NPL], aW[NPL];
+        load_rev<NPL>(p, u0 + c1 - 1, lane, aP, aD, aW);
+        for (int64_t c = c1 - 2; c >= c0; --c) {
+            int Pa[NPL];
+            float Da[NPL], Wa[NPL];
+            load_rev<NPL>(p, u0 + c, lane, Pa, Da, Wa);
+#pragma unroll
+            for (int r = 0; r < NPL; ++r) {
+                const int e = lane * NPL + r;
+                if (e < N) {
+                    sX[e] = aW[r];
+                    sP[e] = aP[r];
+                    sD[e] = aD[r];
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int r = 0; r < NPL; ++r) {
+                const int j = Pa[r];
+                aW[r] = Wa[r] + Da[r] * sX[j];
+                aD[r] = Da[r] * sD[j];
+                aP[r] = sP[j];
+            }
+            __syncwarp();
+        }
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) {
+            const int e = lane * NPL + r;
+            if (e < N) {
+                aggP[warp * kMaxN + e] = aP[r];
+                aggD[warp * kMaxN + e] = aD[r];
+                aggW[warp * kMaxN + e] = aW[r];
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {
+        float x[NPL];
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) {
+            const int e = lane * NPL + r;
+            x[r] = (e < N && p.g_hlast) ? p.g_hlast[bh * p.N + e] : 0.f;
+        }
+        for (int w = nw - 1; w >= 0; --w) {
+#pragma unroll
+            for (int r = 0; r < NPL; ++r) {
+                const int e = lane * NPL + r;
+                if (e < N) carry[w * kMaxN + e] = x[r];
+            }
+            if (C * w / nw < C * (w + 1) / nw) {
+                int P[NPL];
+                float D[NPL], W[NPL];
+#pragma unroll
+                for (int r = 0; r < NPL; ++r) {
+                    const int e = lane * NPL + r;
+                    P[r] = e < N ? aggP[w * kMaxN + e] : 0;
+                    D[r] = e < N ? aggD[w * kMaxN + e] : 0.f;
+                    W[r] = e < N ? aggW[w * kMaxN + e] : 0.f;
+                }
+                apply_gather<NPL>(P, D, W, x, sX, N, lane);
+            }
+        }
+        if (p.g_h0) {
+#pragma unroll
+            for (int r = 0; r < NPL; ++r) {
+                const int e = lane * NPL + r;
+                if (e < N) p.g_h0[bh * p.N + e] = x[r];
+            }
+        }
+    }
+    __syncthreads();
+    float x[NPL];
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        const int e = lane * NPL + r;
+        x[r] = e < N ? carry[warp * kMaxN + e] : 0.f;
+    }
+    for (int64_t c = c1 - 1; c >= c0; --c) {
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) {
+            const int e = lane * NPL + r;
+            if (e < N) p.lam[(u0 + c) * p.N + e] = x[r];
+        }
+        int P[NPL];
+        float D[NPL], W[NPL];
+        load_rev<NPL>(p, u0 + c, lane, P, D, W);
+        apply_gather<NPL>(P, D, W, x, sX, N, lane);
+    }
+}
+
+// ---------------------------------------------------------------------------
+// bwd phase C: per chunk, (1) forward recompute from H_{c-1} keeping the
+// state at every tile start in shared memory, (2) per tile in reverse:
+// recompute the tile's states into registers, then sweep back emitting
+// g_b = lambda, g_c = g_y h, g_d = h_{t-1} * lambda[pi(.)].
+// ---------------------------------------------------------------------------
+template <typename T, int NPL, bool EVEN>
+__global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
+    extern __shared__ __align__(128) unsigned char sm_bc[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
+    if (unit >= p.units) return;
+    const int N = (int)p.N, K = (int)p.K;
+    const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
+    const int64_t hh = bh % p.H;
+    const int64_t s = cidx * p.chunk;
+    const int len = (int)imin64(p.chunk, p.L - s);
+
+    unsigned char *wbase = sm_bc + (size_t)warp * p.smem_per_warp;
+    const int rowb = N * (int)sizeof(T);
+    Ring<3> ring;
+    ring.buf = wbase;
+    ring.rowb = rowb;
+    ring.esz = (int)sizeof(T);
+    ring.tens_bytes = kTS * rowb;
+    ring.stage_bytes = 3 * ring.tens_bytes;
+    ring.ns = p.ns;
+    ring.bulk = p.bulk != 0;
+    float *pbuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes);
+    float *lbuf = pbuf + 2 * kMaxN;
+    float *ck = lbuf + 2 * kMaxN;   // [kBwdMaxChunk / kTS][64]
+    ring.bar0 = smem_u32(ck + (kBwdMaxChunk / kTS) * kMaxN);
+    const int64_t seq_row0 = bh * p.L;
+    ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * rowb;
+    ring.src[1] = reinterpret_cast<const unsigned char *>(p.b) + seq_row0 * rowb;
+    ring.src[2] = reinterpret_cast<const unsigned char *>(p.c) + seq_row0 * rowb;
+    ring_init_bars(ring.bar0, p.ns, lane);
+
+    const int ntiles = (len + kTS - 1) / kTS;
+    const int total = 2 * ntiles;   // pass 1 tiles, then pass 2 tiles (reverse)
+    auto tile_of = [&](int m) { return m < ntiles ? m : 2 * ntiles - 1 - m; };
+    auto nt_of = [&](int m) { return m < ntiles ? 2 : 3; };
+    for (int m = 0; m < p.ns && m < total; ++m) {
+        const int ti = tile_of(m);
+        ring.issue(m, s + (int64_t)ti * kTS, min(kTS, len - ti * kTS), nt_of(m), lane);
+    }
+
+    const int32_t *dict = p.dict + hh * p.dict_hs;
+    const int16_t *plan = p.plan + (hh * p.dict_hs / p.N) * 32 * p.PW;
+    const int64_t kbase = bh * p.L + s;
+    float h[NPL], mu[NPL];
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        const int e = lane * NPL + r;
+        h[r] = 0.f;
+        mu[r] = 0.f;
+        if (e < N) {
+            h[r] = cidx == 0 ? (p.h0 ? p.h0[bh * p.N + e] : 0.f) : p.Hc[(unit - 1) * p.N + e];
+            mu[r] = p.lam[unit * p.N + e];
+        }
+    }
+    int kreg = load_k(p.k, kbase + lane, lane < kTS && lane < len, K, p.status);
+    float gyreg = 0.f;
+
+    for (int m = 0; m < total; ++m) {
+        const int stage = m % p.ns;
+        if (!ring.wait(stage, (uint32_t)((m / p.ns) & 1))) {
+            ring_abort(ring, m, min(total, m + p.ns), p.status, lane);
+            return;
+        }
+        const int ti = tile_of(m);
+        const int t0 = ti * kTS;
+        const int n = min(kTS, len - t0);
+        // next tile in processing order (for the k / g_y prefetch)
+        int knext = 0;
+        float gynext = 0.f;
+        if (m + 1 < total) {
+            const int tn0 = tile_of(m + 1) * kTS;
+            const bool v = lane < kTS && tn0 + lane < len;
+            knext = load_k(p.k, kbase + tn0 + lane, v, K, p.status);
+            if (m + 1 >= ntiles) gynext = v ? p.g_y[kbase + tn0 + lane] : 0.f;
+        }
+        const T *td = reinterpret_cast<const T *>(ring.tile(stage, 0));
+        const T *tb = reinterpret_cast<const T *>(ring.tile(stage, 1));
+        const T *tc = reinterpret_cast<const T *>(ring.tile(stage, 2));
+        if (m < ntiles) {
+            // pass 1: checkpoint at the tile start, then advance the state
+#pragma unroll
+            for (int r = 0; r < NPL; ++r) {
+                const int e = lane * NPL + r;
+                if (e < N) ck[ti * kMaxN + e] = h[r];
+            }
+#pragma unroll
+            for (int q = 0; q < kTS; ++q) {
+                if (q < n) {
+                    const int kk = __shfl_sync(kFull, kreg, q);
+                    float dv[NPL], bv[NPL];
+                    load_row<T, NPL, EVEN>(td + q * N, lane, N, dv);
+                    load_row<T, NPL, EVEN>(tb + q * N, lane, N, bv);
+                    fwd_step<NPL>(h, dv, bv, pbuf + (q & 1) * kMaxN,
+                                  plan + ((int64_t)kk * 32 + lane) * p.PW, lane, N);
+                }
+            }
+        } else {
+            // pass 2: states of this tile, hs[q] = h_{t0+q-1}
+            float hs[kTS + 1][NPL];
+#pragma unroll
+            for (int r = 0; r < NPL; ++r) {
+                const int e = lane * NPL + r;
+                hs[0][r] = e < N ? ck[ti * kMaxN + e] : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < kTS; ++q) {
+#pragma unroll
+                for (int r = 0; r < NPL; ++r) hs[q + 1][r] = hs[q][r];
+                if (q < n) {
+                    const int kk = __shfl_sync(kFull, kreg, q);
+                    float dv[NPL], bv[NPL];
+                    load_row<T, NPL, EVEN>(td + q * N, lane, N, dv);
+                    load_row<T, NPL, EVEN>(tb + q * N, lane, N, bv);
+                    fwd_step<NPL>(hs[q + 1], dv, bv, pbuf + (q & 1) * kMaxN,
+                                  plan + ((int64_t)kk * 32 + lane) * p.PW, lane, N);
+                }
+            }
+#pragma unroll
+            for (int q = kTS - 1; q >= 0; --q) {
+                if (q < n) {
+                    const int kk = __shfl_sync(kFull, kreg, q);
+                    const float gy = __shfl_sync(kFull, gyreg, q);
+                    const int64_t row = (kbase + t0 + q) * p.N;
+                    float dv[NPL], cv[NPL], lam[NPL], gc[NPL];
+                    load_row<T, NPL, EVEN>(td + q * N, lane, N, dv);
+                    load_row<T, NPL, EVEN>(tc + q * N, lane, N, cv);
+                    float *lb = lbuf + (q & 1) * kMaxN;
+#pragma unroll
+                    for (int r = 0; r < NPL; ++r) {
+                        const int e = lane * NPL + r;
+                        lam[r] = gy * cv[r] + mu[r];
+                        gc[r] = gy * hs[q + 1][r];
+                        if (e < N) lb[e] = lam[r];
+                    }
+                    store_row<NPL, EVEN>(p.g_b + row, lane, N, lam);
+                    store_row<NPL, EVEN>(p.g_c + row, lane, N, gc);
+                    __syncwarp();
+                    const int32_t *pk = dict + (int64_t)kk * N;
+                    float gd[NPL];
+#pragma unroll
+                    for (int r = 0; r < NPL; ++r) {
+                        const int e = lane * NPL + r;
+                        const float gl = e < N ? lb[__ldg(pk + e)] : 0.f;
+                        gd[r] = hs[q][r] * gl;
+                        mu[r] = dv[r] * gl;
+                    }
+                    store_row<NPL, EVEN>(p.g_d + row, lane, N, gd);
+                }
+            }
+        }
+        __syncwarp();
+        if (m + p.ns < total) {
+            const int mn = m + p.ns;
+            const int tn = tile_of(mn);
+            ring.issue(stage, s + (int64_t)tn * kTS, min(kTS, len - tn * kTS), nt_of(mn), lane);
+        }
+        kreg = knext;
+        gyreg = gynext;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// launchers
+// ---------------------------------------------------------------------------
+template <typename KernT>
+static cudaError_t launch_chunk_b(KernT kern, const ChunkParams &p, size_t smem,
+                                  cudaStream_t st) {
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = (p.units + kWPC - 1) / kWPC;
+    kern<<<(unsigned)grid, kWPC * 32, smem, st>>>(p);
+    return cudaGetLastError();
+}
+
+#define PDSSM_DISPATCH_B(KERNEL, p, st, smem)                                     \
+    do {                                                                         \
+        const bool even = ((p).N % 2) == 0;                                      \
+        if ((p).N > 32) {                                                        \
+            return even ? launch_chunk_b(KERNEL<T, 2, true>, p, smem, st)        \
+                        : launch_chunk_b(KERNEL<T, 2, false>, p, smem, st);      \
+        }                                                                        \
+        return launch_chunk_b(KERNEL<T, 1, true>, p, smem, st);                  \
+    } while (0)
+
+template <typename T>
+static cudaError_t bwdA_t(ChunkParams p, cudaStream_t st) {
+    const int rowb = (int)p.N * (int)sizeof(T);
+    p.smem_per_warp = (p.ns * 2 * kTS * rowb + 2 * kMaxN * 4 + kMaxStages * 8 + 127) / 128 * 128;
+    const size_t smem = (size_t)kWPC * p.smem_per_warp;
+    PDSSM_DISPATCH_B(k_bwdA, p, st, smem);
+}
+
+template <typename T>
+static cudaError_t bwdC_t(ChunkParams p, cudaStream_t st) {
+    const int rowb = (int)p.N * (int)sizeof(T);
+    p.smem_per_warp = (bwd_warp_smem_bytes(p.ns, 3, rowb) + 127) / 128 * 128;
+    const size_t smem = (size_t)kWPC * p.smem_per_warp;
+    PDSSM_DISPATCH_B(k_bwdC, p, st, smem);
+}
+
+cudaError_t launch_bwdA(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st) {
+    if (p.units == 0) return cudaSuccess;
+    return dt == PDSSM_BF16 ? bwdA_t<__nv_bfloat16>(p, st) : bwdA_t<float>(p, st);
+}
+
+cudaError_t launch_bwdC(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st) {
+    if (p.units == 0) return cudaSuccess;
+    return dt == PDSSM_BF16 ? bwdC_t<__nv_bfloat16>(p, st) : bwdC_t<float>(p, st);
+}
+
+cudaError_t launch_bwdB(const ChunkParams &p, cudaStream_t st) {
+    if (p.units == 0) return cudaSuccess;
+    const int nw = (int)imin64(32, p.C);
+    const size_t smem = (size_t)nw * kMaxN * 4 * 7;
+    const int64_t BH = p.B * p.H;
+    cudaError_t e;
+    if (p.N > 32) {
+        e = cudaFuncSetAttribute(k_bwdB<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return e;
+        k_bwdB<2><<<(unsigned)BH, nw * 32, smem, st>>>(p);
+    } else {
+        e = cudaFuncSetAttribute(k_bwdB<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e != cudaSuccess) return e;
+        k_bwdB<1><<<(unsigned)BH, nw * 32, smem, st>>>(p);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace pdssm

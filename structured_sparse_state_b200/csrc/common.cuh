@@ -1,0 +1,332 @@
+// Shared device helpers and launch plumbing for the PD-SSM kernels (sm_100a).
+//
+// Work decomposition used by every chunk kernel: one warp owns one
+// (batch, head, chunk) unit; lane l owns state elements e = l*NPL + r,
+// r < NPL, NPL = ceil(N / 32) in {1, 2}.  Chunk data (rows of d, b, c) are
+// contiguous in HBM, so each warp streams its chunk through shared memory in
+// tiles of kTS steps with 1-D bulk copies (cp.async.bulk, the TMA engine's
+// non-tensor path) completed on per-warp mbarriers, double- or
+// triple-buffered.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <type_traits>
+
+#include "../../include/pdssm.h"
+
+namespace pdssm {
+
+constexpr int kTS = 16;        // steps per staged tile = steps per readout group
+constexpr int kWPC = 4;        // warps (units) per CTA in the chunk kernels
+constexpr int kMaxN = 64;
+constexpr int kMaxStages = 4;
+constexpr int kBwdMaxChunk = 256;   // checkpoints of one chunk kept in shared memory
+constexpr unsigned kFull = 0xffffffffu;
+
+// status word bits (first int of the workspace)
+enum : int { kStBadIndex = 1, kStTimeout = 2 };
+
+// ---------------------------------------------------------------------------
+// workspace layout (all offsets 256-byte aligned)
+// ---------------------------------------------------------------------------
+struct WsLayout {
+    size_t status, dict, plan, Pi, Dl, v, Hc, wc, lam, total;
+    int64_t C, Hd, PW;
+};
+
+inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+__host__ __device__ __forceinline__ int64_t imin64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+inline WsLayout ws_layout(const pdssm_dims &dm, int64_t pi_hs, int64_t chunk,
+                          bool for_bwd) {
+    WsLayout w{};
+    w.C = dm.L > 0 ? (dm.L + chunk - 1) / chunk : 0;
+    w.Hd = pi_hs ? dm.H : 1;
+    w.PW = 8 * ((dm.N + 1 + 7) / 8);   // entries per plan row: count + sources
+    const size_t units = (size_t)(dm.B * dm.H * w.C);
+    const size_t vecs = units * (size_t)dm.N * 4;
+    size_t o = 0;
+    w.status = o; o += 256;
+    w.dict = o;   o = align256(o + (size_t)(w.Hd * dm.K * dm.N) * 4);
+    w.plan = o;   o = align256(o + (size_t)(w.Hd * dm.K * 32 * w.PW) * 2);
+    w.Pi = o;     o = align256(o + vecs);
+    w.Dl = o;     o = align256(o + vecs);
+    w.v = o;      o = align256(o + vecs);
+    w.Hc = o;     o = align256(o + vecs);
+    if (for_bwd) {
+        w.wc = o;  o = align256(o + vecs);
+        w.lam = o; o = align256(o + vecs);
+    }
+    w.total = o;
+    return w;
+}
+
+// ---------------------------------------------------------------------------
+// parameters of the chunk kernels
+// ---------------------------------------------------------------------------
+struct ChunkParams {
+    int64_t B, H, L, N, K, C, chunk, units;
+    int64_t dict_hs;          // head stride of the sanitised dictionary (0 or K*N)
+    const int32_t *dict;      // sanitised dictionary [Hd][K][N]
+    const int16_t *plan;      // gather plans [Hd][K][32][PW]
+    int PW;
+    const int32_t *k;
+    const void *d, *b, *c;
+    const float *h0;
+    float *y;
+    int32_t *Pi;
+    float *Dl, *v, *Hc, *wc, *lam;
+    const float *g_y, *g_hlast;
+    float *g_b, *g_d, *g_c, *g_h0;
+    float *h_last;
+    int *status;
+    int ns;                   // pipeline stages
+    int bulk;                 // 1: bulk-copy staging; 0: cooperative copies
+    int smem_per_warp;
+};
+
+// ---------------------------------------------------------------------------
+// small device helpers
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float to_f(T x);
+template <>
+__device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <>
+__device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void flag_status(int *status, int bit) {
+    atomicOr(status, bit);
+}
+
+__device__ __forceinline__ uint64_t global_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_mbar_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
+                 "r"(bytes)
+                 : "memory");
+}
+
+// 1-D bulk copy global -> shared, completion counted on an mbarrier.  Plain
+// per-CTA copy of this GPU's own memory (no multicast).
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
+                                         uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], "
+        "%2, [%3];" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar)
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait: gives up after ~2 s of wall time or 2^26 polls.
+static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = global_ns();
+    for (uint32_t it = 0; it < (1u << 26); ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 1023u) == 1023u && global_ns() - t0 > 2000000000ull) break;
+    }
+    return false;
+}
+
+// Reduce-scatter of 16 per-lane partials: lane l (and l + 16) returns
+// sum over all 32 lanes of v[l & 15].  16 shuffles for 16 values.
+__device__ __forceinline__ float reduce_scatter16(float (&v)[kTS]) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const bool up = lane & 8;
+        const float send = up ? v[i] : v[i + 8];
+        const float keep = up ? v[i + 8] : v[i];
+        v[i] = keep + __shfl_xor_sync(kFull, send, 8);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const bool up = lane & 4;
+        const float send = up ? v[i] : v[i + 4];
+        const float keep = up ? v[i + 4] : v[i];
+        v[i] = keep + __shfl_xor_sync(kFull, send, 4);
+    }
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+        const bool up = lane & 2;
+        const float send = up ? v[i] : v[i + 2];
+        const float keep = up ? v[i + 2] : v[i];
+        v[i] = keep + __shfl_xor_sync(kFull, send, 2);
+    }
+    {
+        const bool up = lane & 1;
+        const float send = up ? v[0] : v[1];
+        const float keep = up ? v[1] : v[0];
+        v[0] = keep + __shfl_xor_sync(kFull, send, 1);
+    }
+    return v[0] + __shfl_xor_sync(kFull, v[0], 16);
+}
+
+// Load the NPL elements a lane owns from one staged row (0 beyond N).
+template <typename T, int NPL, bool EVEN>
+__device__ __forceinline__ void load_row(const T *row, int lane, int N, float (&v)[NPL]) {
+    if constexpr (NPL == 1) {
+        v[0] = lane < N ? to_f<T>(row[lane]) : 0.f;
+    } else {
+        const int e0 = 2 * lane;
+        if constexpr (EVEN) {
+            if (e0 < N) {
+                if constexpr (std::is_same<T, float>::value) {
+                    const float2 q = *reinterpret_cast<const float2 *>(row + e0);
+                    v[0] = q.x;
+                    v[1] = q.y;
+                } else {
+                    const __nv_bfloat162 q = *reinterpret_cast<const __nv_bfloat162 *>(row + e0);
+                    v[0] = __low2float(q);
+                    v[1] = __high2float(q);
+                }
+            } else {
+                v[0] = 0.f;
+                v[1] = 0.f;
+            }
+        } else {
+            v[0] = e0 < N ? to_f<T>(row[e0]) : 0.f;
+            v[1] = e0 + 1 < N ? to_f<T>(row[e0 + 1]) : 0.f;
+        }
+    }
+}
+
+// Selection index of one step, clamped into [0, K) (flagged when it was not).
+__device__ __forceinline__ int load_k(const int32_t *kp, int64_t idx, bool valid, int K,
+                                      int *status) {
+    int kv = valid ? __ldg(kp + idx) : 0;
+    if (kv < 0 || kv >= K) {
+        flag_status(status, kStBadIndex);
+        kv = kv < 0 ? 0 : K - 1;
+    }
+    return kv;
+}
+
+// ---------------------------------------------------------------------------
+// per-warp staging ring: NT tensors, ns stages of kTS rows each
+// ---------------------------------------------------------------------------
+template <int NT>
+struct Ring {
+    unsigned char *buf;    // stage 0, tensor 0
+    uint32_t bar0;         // mbarrier of stage 0 (8 bytes each)
+    int stage_bytes;       // NT * tens_bytes
+    int tens_bytes;        // kTS * rowb
+    int rowb;              // N * element size
+    int esz;
+    int ns;
+    bool bulk;
+    const unsigned char *src[NT];   // row 0 of this (b, h) sequence, per tensor
+
+    __device__ unsigned char *tile(int stage, int q) const {
+        return buf + stage * stage_bytes + q * tens_bytes;
+    }
+
+    // Stage rows [t0, t0 + n) of the first nt tensors into `stage`.
+    __device__ void issue(int stage, int64_t t0, int n, int nt, int lane) const {
+        if (bulk) {
+            if (lane == 0) {
+                const uint32_t bar = bar0 + 8u * stage;
+                const uint32_t bytes = (uint32_t)(n * rowb);
+                mbar_expect_tx(bar, bytes * (uint32_t)nt);
+#pragma unroll
+                for (int q = 0; q < NT; ++q)
+                    if (q < nt) bulk_g2s(smem_u32(tile(stage, q)), src[q] + t0 * rowb, bytes, bar);
+            }
+        } else {
+            const int elems = n * (rowb / esz);
+#pragma unroll
+            for (int q = 0; q < NT; ++q) {
+                if (q >= nt) continue;
+                if (esz == 4) {
+                    const float *s = reinterpret_cast<const float *>(src[q] + t0 * rowb);
+                    float *dst = reinterpret_cast<float *>(tile(stage, q));
+                    for (int i = lane; i < elems; i += 32) dst[i] = s[i];
+                } else {
+                    const unsigned short *s =
+                        reinterpret_cast<const unsigned short *>(src[q] + t0 * rowb);
+                    unsigned short *dst = reinterpret_cast<unsigned short *>(tile(stage, q));
+                    for (int i = lane; i < elems; i += 32) dst[i] = s[i];
+                }
+            }
+            __syncwarp();
+        }
+    }
+
+    __device__ bool wait(int stage, uint32_t parity) const {
+        if (!bulk) return true;
+        return mbar_wait_bounded(bar0 + 8u * stage, parity);
+    }
+};
+
+// Initialise a warp's ns mbarriers (one arrival each: the expect_tx).
+__device__ __forceinline__ void ring_init_bars(uint32_t bar0, int ns, int lane) {
+    if (lane == 0) {
+        for (int s = 0; s < ns; ++s) mbar_init(bar0 + 8u * s, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+}
+
+// After a wait gave up: record it and wait (bounded) for the copies this warp
+// still has in flight into tiles [first, last) so none lands after exit.
+template <int NT>
+__device__ void ring_abort(const Ring<NT> &ring, int first, int last, int *status,
+                           int lane) {
+    if (lane == 0) flag_status(status, kStTimeout);
+    for (int i = first; i < last; ++i) ring.wait(i % ring.ns, (uint32_t)((i / ring.ns) & 1));
+    __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
+// host launchers (one per kernel family)
+// ---------------------------------------------------------------------------
+cudaError_t launch_select(const pdssm_dims &dm, const void *u, pdssm_dtype ut, const float *W,
+                          int32_t *k_out, cudaStream_t st);
+cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
+                        int16_t *plan, int PW, int64_t Hd, int *status, cudaStream_t st);
+cudaError_t launch_validate(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs,
+                            const int32_t *k, int *counts, cudaStream_t st);
+cudaError_t launch_phaseA(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st);
+cudaError_t launch_phaseB(const ChunkParams &p, cudaStream_t st);
+cudaError_t launch_phaseC(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st);
+cudaError_t launch_bwdA(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st);
+cudaError_t launch_bwdB(const ChunkParams &p, cudaStream_t st);
+cudaError_t launch_bwdC(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st);
+
+}  // namespace pdssm

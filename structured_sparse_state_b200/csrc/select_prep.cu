@@ -1,0 +1,200 @@
+// Hard selection (fused logits + first argmax), dictionary preparation
+// (phase A0: gather plans of each one-hot column selector) and index
+// validation.
+//
+// Flash PD-SSM technical summary, Methodology §1: at each step the input u_t
+// gives K scores through a linear map and the single highest-scoring
+// dictionary matrix is used; each matrix is a one-hot column selector, held
+// here as an index map pi_k : [N] -> [N] with P_k[pi_k(j), j] = 1.
+#include "common.cuh"
+
+namespace pdssm {
+
+// ---------------------------------------------------------------------------
+// k_select: one thread per (b, t) row, 128 rows per CTA.  The u tile is kept
+// transposed in shared memory ([D][129] fp32, conflict-free both ways); the
+// weights of one head are staged transposed ([D][KB]) and read as
+// broadcasts.  Each logit is the sequential fp32 chain acc = fma(W, u, acc)
+// over ascending d -- the selection contract -- so k is bit-reproducible.
+// ---------------------------------------------------------------------------
+constexpr int kSelRows = 128;
+
+__host__ __device__ inline size_t sel_u_floats(int D) {
+    return ((size_t)D * (kSelRows + 1) + 3) / 4 * 4;
+}
+
+template <typename TU, int KB>
+__global__ void __launch_bounds__(kSelRows) k_select(const TU *__restrict__ u,
+                                                     const float *__restrict__ W,
+                                                     int32_t *__restrict__ k_out, int64_t rows,
+                                                     int64_t L, int D, int H, int K) {
+    extern __shared__ __align__(16) float sm_sel[];
+    float *us = sm_sel;                          // [D][kSelRows + 1]
+    // weights start on a 16-byte boundary (float4 reads) whatever D is
+    float *wsm = us + sel_u_floats(D);           // [2][D][KB]
+    const int tid = threadIdx.x;
+    const int64_t row0 = (int64_t)blockIdx.x * kSelRows;
+    const int nrows = (int)imin64(kSelRows, rows - row0);
+
+    for (int idx = tid; idx < nrows * D; idx += kSelRows) {
+        const int r = idx / D, q = idx - r * D;
+        us[q * (kSelRows + 1) + r] = to_f<TU>(u[(row0 + r) * D + q]);
+    }
+    auto stage_w = [&](int h, float *dst) {
+        for (int idx = tid; idx < D * KB; idx += kSelRows) {
+            const int q = idx / KB, kk = idx - q * KB;
+            dst[idx] = kk < K ? W[((int64_t)h * K + kk) * D + q] : 0.f;
+        }
+    };
+    stage_w(0, wsm);
+    __syncthreads();
+
+    const int64_t row = row0 + tid;
+    const int64_t bb = row / L, t = row - bb * L;
+    for (int h = 0; h < H; ++h) {
+        float *wc = wsm + (size_t)(h & 1) * D * KB;
+        if (h + 1 < H) stage_w(h + 1, wsm + (size_t)((h + 1) & 1) * D * KB);
+        if (tid < nrows) {
+            float acc[KB];
+#pragma unroll
+            for (int kk = 0; kk < KB; ++kk) acc[kk] = 0.f;
+            for (int q = 0; q < D; ++q) {
+                const float uq = us[q * (kSelRows + 1) + tid];
+                const float4 *wr = reinterpret_cast<const float4 *>(wc + q * KB);
+#pragma unroll
+                for (int k4 = 0; k4 < KB / 4; ++k4) {
+                    const float4 w4 = wr[k4];
+                    acc[4 * k4 + 0] = __fmaf_rn(w4.x, uq, acc[4 * k4 + 0]);
+                    acc[4 * k4 + 1] = __fmaf_rn(w4.y, uq, acc[4 * k4 + 1]);
+                    acc[4 * k4 + 2] = __fmaf_rn(w4.z, uq, acc[4 * k4 + 2]);
+                    acc[4 * k4 + 3] = __fmaf_rn(w4.w, uq, acc[4 * k4 + 3]);
+                }
+            }
+            int best = 0;
+            float bv = acc[0];
+#pragma unroll
+            for (int kk = 1; kk < KB; ++kk)
+                if (kk < K && acc[kk] > bv) {
+                    bv = acc[kk];
+                    best = kk;
+                }
+            k_out[(bb * H + h) * L + t] = best;
+        }
+        __syncthreads();
+    }
+}
+
+template <typename TU, int KB>
+static cudaError_t select_t(const pdssm_dims &dm, const void *u, const float *W, int32_t *k_out,
+                            cudaStream_t st) {
+    const int64_t rows = dm.B * dm.L;
+    const int D = (int)dm.D_in;
+    const size_t smem = (sel_u_floats(D) + 2 * (size_t)D * KB) * sizeof(float);
+    auto kern = k_select<TU, KB>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = (rows + kSelRows - 1) / kSelRows;
+    kern<<<(unsigned)grid, kSelRows, smem, st>>>(reinterpret_cast<const TU *>(u), W, k_out,
+                                                 rows, dm.L, D, (int)dm.H, (int)dm.K);
+    return cudaGetLastError();
+}
+
+template <typename TU>
+static cudaError_t select_k(const pdssm_dims &dm, const void *u, const float *W, int32_t *k_out,
+                            cudaStream_t st) {
+    if (dm.K <= 4) return select_t<TU, 4>(dm, u, W, k_out, st);
+    if (dm.K <= 8) return select_t<TU, 8>(dm, u, W, k_out, st);
+    if (dm.K <= 16) return select_t<TU, 16>(dm, u, W, k_out, st);
+    return select_t<TU, 32>(dm, u, W, k_out, st);
+}
+
+cudaError_t launch_select(const pdssm_dims &dm, const void *u, pdssm_dtype ut, const float *W,
+                          int32_t *k_out, cudaStream_t st) {
+    if (dm.B * dm.L == 0) return cudaSuccess;
+    return ut == PDSSM_BF16 ? select_k<__nv_bfloat16>(dm, u, W, k_out, st)
+                            : select_k<float>(dm, u, W, k_out, st);
+}
+
+// ---------------------------------------------------------------------------
+// k_prep (phase A0): one warp per (dictionary, k).  Writes a sanitised copy
+// of the map (entries clamped into [0, N), flagged) and the gather plan:
+// for lane l, the sources j whose target pi(j) is an element lane l owns,
+// in ascending j, each encoded as j | (r << 7) with r = target - l*NPL.
+// Row layout [count G][e_1 .. e_G][-1 ...]; G is the maximum over lanes, so
+// every lane of a warp loops the same number of times.
+// ---------------------------------------------------------------------------
+__global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *__restrict__ dict,
+                       int16_t *__restrict__ plan, int PW, int64_t nmaps, int K, int N, int npl,
+                       int *status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t m = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (m >= nmaps) return;
+    const int64_t dk = m / K, kk = m - dk * K;
+    const int32_t *src = pi + dk * pi_hs + kk * N;
+    int32_t *dst = dict + m * N;
+    int16_t *row = plan + (m * 32 + lane) * PW;
+    int cnt = 0;
+    bool bad = false;
+    for (int j = 0; j < N; ++j) {
+        int tgt = __ldg(src + j);
+        if (tgt < 0 || tgt >= N) {
+            bad = true;
+            tgt = tgt < 0 ? 0 : N - 1;
+        }
+        if (lane == 0) dst[j] = tgt;
+        if (tgt / npl == lane) {
+            row[1 + cnt] = (int16_t)(j | ((tgt - lane * npl) << 7));
+            ++cnt;
+        }
+    }
+    if (bad && lane == 0) flag_status(status, kStBadIndex);
+    const int G = __reduce_max_sync(kFull, cnt);
+    row[0] = (int16_t)G;
+    for (int g = 1 + cnt; g < PW; ++g) row[g] = (int16_t)-1;
+}
+
+cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
+                        int16_t *plan, int PW, int64_t Hd, int *status, cudaStream_t st) {
+    const int64_t nmaps = Hd * dm.K;
+    const int npl = dm.N > 32 ? 2 : 1;
+    const int wpb = 4;
+    const int64_t grid = (nmaps + wpb - 1) / wpb;
+    k_prep<<<(unsigned)grid, 32 * wpb, 0, st>>>(pi, pi_hs, dict, plan, PW, nmaps, (int)dm.K,
+                                                (int)dm.N, npl, status);
+    return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// k_validate: counts dictionary entries outside [0, N) (counts[0]) and
+// selections outside [0, K) (counts[1]).
+// ---------------------------------------------------------------------------
+__global__ void k_validate(const int32_t *__restrict__ pi, int64_t pi_hs, int64_t Hd, int K,
+                           int N, const int32_t *__restrict__ k, int64_t nk, int *counts) {
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    const int64_t tid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t npi = Hd * K * N;
+    int bad_pi = 0, bad_k = 0;
+    for (int64_t i = tid; i < npi; i += stride) {
+        const int64_t dk = i / ((int64_t)K * N), rem = i - dk * K * N;
+        const int v = pi[dk * pi_hs + rem];
+        bad_pi += (v < 0 || v >= N);
+    }
+    if (k)
+        for (int64_t i = tid; i < nk; i += stride) {
+            const int v = k[i];
+            bad_k += (v < 0 || v >= K);
+        }
+    if (bad_pi) atomicAdd(counts, bad_pi);
+    if (bad_k) atomicAdd(counts + 1, bad_k);
+}
+
+cudaError_t launch_validate(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs,
+                            const int32_t *k, int *counts, cudaStream_t st) {
+    const int64_t Hd = pi_hs ? dm.H : 1;
+    k_validate<<<296, 256, 0, st>>>(pi, pi_hs, Hd, (int)dm.K, (int)dm.N, k, dm.B * dm.H * dm.L,
+                                    counts);
+    return cudaGetLastError();
+}
+
+}  // namespace pdssm

@@ -1,0 +1,248 @@
+"""GPU parity: the sm_100a kernels, called through the C ABI, against the CPU
+oracle on the same seeded inputs.  Indices (k, composed maps) must match bit
+for bit; floats within the floored relative error of 1e-5 (fp32 inputs) or
+2e-2 (bf16 inputs)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import pdssm_inputs as gen
+import structured_sparse_state_b200 as pd
+from parity_util import (TOL_F32, dev, floored_relerr, oracle_k, sample_rows, to_device,
+                         tol_for)
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def run_fwd(inp, chunk, k=None, for_bwd=False):
+    t = to_device(inp)
+    kk = k if k is not None else t["k"]
+    y, hl, ws = pd.pdssm_scan_fwd(t["pi"], kk, t["d"], t["b"], t["c"], t["h0"], chunk=chunk,
+                                  for_bwd=for_bwd)
+    assert pd.pdssm_ws_status(ws) == 0
+    return t, kk, y, hl, ws
+
+
+def check_fwd(inp, chunk, k_np=None):
+    t = to_device(inp)
+    if k_np is None:
+        k_np = oracle_k(inp)
+    kk = dev(k_np, torch.int32)
+    y, hl, ws = pd.pdssm_scan_fwd(t["pi"], kk, t["d"], t["b"], t["c"], t["h0"], chunk=chunk)
+    torch.cuda.synchronize()
+    assert pd.pdssm_ws_status(ws) == 0
+    y_ref, hl_ref = oracle.scan_fwd(inp.pi, k_np, inp.d, inp.b, inp.c, inp.h0)
+    tol = tol_for(inp)
+    ey = floored_relerr(y.cpu().numpy(), y_ref)
+    eh = floored_relerr(hl.cpu().numpy(), hl_ref)
+    assert ey <= tol, f"y error {ey}"
+    assert eh <= tol, f"h_last error {eh}"
+    return ey, eh
+
+
+# ----------------------------------------------------------------------------
+# selection
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("idx,over", [(0, {}), (1, dict(B=2, L=1500)),
+                                      (2, dict(B=1, L=777)), (2, dict(B=2, L=130, K=5))])
+def test_select_bit_exact(idx, over):
+    inp = gen.generate(gen.workload(idx, **over))
+    t = to_device(inp)
+    k = pd.pdssm_select(t["u"], t["W"]).cpu().numpy()
+    assert (k == oracle.select(inp.u, inp.W)).all()
+
+
+# ----------------------------------------------------------------------------
+# chunk transfers: composed maps bit-exact
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("idx,over,chunk", [
+    (0, {}, 32), (1, dict(B=1, L=1000), 64), (2, dict(B=1, H=2, L=600), 128),
+    (3, dict(H=2, L=1000), 256), (4, dict(B=1, H=2, L=700), 128), (4, dict(B=1, H=1, L=50), 7)])
+def test_chunk_transfers(idx, over, chunk):
+    inp = gen.generate(gen.workload(idx, **over))
+    k_np = oracle_k(inp)
+    t = to_device(inp)
+    Pi, Dl, v = pd.pdssm_chunk_transfers(t["pi"], dev(k_np, torch.int32), t["d"], t["b"], chunk)
+    Pi_r, Dl_r, v_r = oracle.chunk_transfers(inp.pi, k_np, inp.d, inp.b, chunk)
+    assert (Pi.cpu().numpy() == Pi_r).all()
+    tol = tol_for(inp)
+    assert floored_relerr(Dl.cpu().numpy(), Dl_r) <= tol
+    assert floored_relerr(v.cpu().numpy(), v_r) <= tol
+
+
+# ----------------------------------------------------------------------------
+# forward, reduced copies of the five workloads (several tiles, ragged tails)
+# ----------------------------------------------------------------------------
+@pytest.mark.parametrize("idx,over", [
+    (0, {}),
+    (1, {}),
+    (2, dict(B=2, H=3, L=1000)),
+    (3, dict(H=4, L=3000)),
+    (4, dict(B=1, H=3, L=2000)),
+])
+def test_forward_workloads_reduced(idx, over):
+    cfg = gen.workload(idx, **over)
+    check_fwd(gen.generate(cfg), cfg["chunk"])
+
+
+def test_stiff_impulse_elementwise():
+    """Impulse response with d down to 1e-4: elementwise relative error where
+    the oracle is >= 1e-30, tiny values elsewhere, no NaN/Inf."""
+    cfg = gen.workload(3, H=8, L=4096)
+    inp = gen.generate(cfg)
+    t = to_device(inp)
+    y, hl, ws = pd.pdssm_scan_fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], None, chunk=256)
+    y = y.cpu().numpy().astype(np.float64)
+    y_ref, _ = oracle.scan_fwd(inp.pi, inp.k, inp.d, inp.b, inp.c, None)
+    assert np.isfinite(y).all()
+    big = np.abs(y_ref) >= 1e-30
+    assert big.sum() > 8
+    assert np.max(np.abs(y[big] - y_ref[big]) / np.abs(y_ref[big])) <= 1e-5
+    assert np.max(np.abs(y[~big])) <= 1e-30
+
+
+# ----------------------------------------------------------------------------
+# edge cases
+# ----------------------------------------------------------------------------
+def small(seed, B, H, L, N, K, kind="maps", dtype="f32", per_head=False, h0=True):
+    rng = np.random.default_rng(seed)
+    nd = H if per_head else 1
+    if kind == "maps":
+        pi = rng.integers(0, N, size=(nd, K, N))
+    elif kind == "perm":
+        pi = np.stack([np.stack([rng.permutation(N) for _ in range(K)]) for _ in range(nd)])
+    elif kind == "identity":
+        pi = np.tile(np.arange(N), (nd, K, 1))
+    elif kind == "constant":
+        pi = np.stack([np.stack([np.full(N, rng.integers(0, N)) for _ in range(K)])
+                       for _ in range(nd)])
+    pi = pi.astype(np.int32)
+    if not per_head:
+        pi = pi[0]
+    shape = (B, H, L, N)
+    d = rng.uniform(0.5, 1.0, shape).astype(np.float32)
+    b = rng.standard_normal(shape).astype(np.float32)
+    c = rng.standard_normal(shape).astype(np.float32)
+    if dtype == "bf16":
+        d, b, c = (gen.round_bf16(x) for x in (d, b, c))
+    cfg = dict(dtype=dtype)
+    return gen.Inputs(cfg=cfg, pi=pi, d=d, b=b, c=c,
+                      k=rng.integers(0, K, size=(B, H, L)).astype(np.int32),
+                      h0=rng.standard_normal((B, H, N)).astype(np.float32) if h0 else None,
+                      g_y=rng.standard_normal((B, H, L)).astype(np.float32))
+
+
+@pytest.mark.parametrize("N", [1, 2, 3, 8, 31, 32, 33, 47, 63, 64])
+def test_forward_state_sizes(N):
+    check_fwd(small(N, 2, 2, 300, N, 5), chunk=37)
+
+
+@pytest.mark.parametrize("chunk", [1, 2, 7, 16, 17, 100, 999, 1000, 5000])
+def test_forward_chunk_sizes(chunk):
+    check_fwd(small(chunk, 1, 2, 1000, 24, 6), chunk=chunk)
+
+
+@pytest.mark.parametrize("kind", ["identity", "constant", "perm"])
+@pytest.mark.parametrize("N", [16, 64])
+def test_forward_map_kinds(kind, N):
+    check_fwd(small(7, 1, 2, 500, N, 3, kind=kind), chunk=64)
+
+
+@pytest.mark.parametrize("N", [8, 30, 64])
+def test_forward_bf16_aligned_and_unaligned_rows(N):
+    check_fwd(small(9, 1, 2, 400, N, 4, dtype="bf16"), chunk=48)
+
+
+def test_forward_per_head_dictionary_and_K1():
+    check_fwd(small(11, 2, 3, 333, 40, 6, per_head=True), chunk=50)
+    check_fwd(small(12, 1, 2, 200, 20, 1), chunk=32)
+
+
+def test_forward_zero_initial_state_and_tiny_lengths():
+    check_fwd(small(13, 1, 2, 1, 8, 3, h0=False), chunk=4)
+    check_fwd(small(14, 1, 2, 17, 64, 3, h0=False), chunk=4)
+
+
+def test_forward_empty_sequence():
+    inp = small(15, 1, 2, 0, 8, 3)
+    t = to_device(inp)
+    y, hl, ws = pd.pdssm_scan_fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=8)
+    torch.cuda.synchronize()
+    assert y.numel() == 0
+    assert torch.equal(hl, t["h0"])
+
+
+def test_forward_deterministic():
+    inp = gen.generate(gen.workload(4, B=1, H=4, L=4096))
+    t = to_device(inp)
+    y1, h1, _ = pd.pdssm_scan_fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=128)
+    y2, h2, _ = pd.pdssm_scan_fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=128)
+    assert torch.equal(y1, y2) and torch.equal(h1, h2)
+
+
+# ----------------------------------------------------------------------------
+# backward
+# ----------------------------------------------------------------------------
+def check_bwd(inp, chunk, g_hlast=None):
+    t = to_device(inp)
+    y, hl, ws = pd.pdssm_scan_fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"],
+                                  chunk=chunk, for_bwd=True)
+    ghl = dev(g_hlast) if g_hlast is not None else None
+    g = pd.pdssm_scan_bwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], t["g_y"], ws,
+                          chunk=chunk, g_hlast=ghl)
+    torch.cuda.synchronize()
+    assert pd.pdssm_ws_status(ws) == 0
+    ref = oracle.scan_bwd(inp.pi, inp.k, inp.d, inp.b, inp.c, inp.h0, inp.g_y, g_hlast)
+    tol = tol_for(inp)
+    for name, a, r in zip(("g_b", "g_d", "g_c", "g_h0"), g, ref):
+        e = floored_relerr(a.cpu().numpy(), r)
+        assert e <= tol, f"{name} error {e}"
+
+
+@pytest.mark.parametrize("N", [1, 5, 32, 33, 64])
+def test_backward_state_sizes(N):
+    check_bwd(small(20 + N, 1, 2, 300, N, 4), chunk=40)
+
+
+@pytest.mark.parametrize("chunk", [1, 3, 16, 100, 256])
+def test_backward_chunk_sizes(chunk):
+    inp = small(30 + chunk, 1, 2, 700, 24, 5)
+    rng = np.random.default_rng(chunk)
+    check_bwd(inp, chunk, g_hlast=rng.standard_normal((1, 2, 24)).astype(np.float32))
+
+
+def test_backward_workload_reduced():
+    cfg = gen.workload(4, B=1, H=2, L=3000)
+    check_bwd(gen.generate(cfg), cfg["chunk"])
+
+
+def test_backward_bf16_and_maps():
+    check_bwd(small(41, 1, 2, 400, 64, 4, dtype="bf16"), chunk=64)
+    check_bwd(small(42, 1, 2, 300, 16, 3, kind="constant"), chunk=32)
+
+
+# ----------------------------------------------------------------------------
+# index validation (host-side checks, clamped indices never fault)
+# ----------------------------------------------------------------------------
+def test_validate_and_clamped_indices_are_reported():
+    inp = small(50, 1, 2, 100, 8, 3)
+    t = to_device(inp)
+    assert pd.pdssm_validate(t["pi"], t["k"], 8) == 0
+    bad_k = t["k"].clone()
+    bad_k[0, 1, 17] = 3
+    assert pd.pdssm_validate(t["pi"], bad_k, 8) == 3
+    bad_pi = t["pi"].clone()
+    bad_pi[1, 2] = -1
+    assert pd.pdssm_validate(bad_pi, t["k"], 8) == 3
+    y, hl, ws = pd.pdssm_scan_fwd(t["pi"], bad_k, t["d"], t["b"], t["c"], t["h0"], chunk=16)
+    assert pd.pdssm_ws_status(ws) == 3
+    assert pd.pdssm_ws_status(ws) == 0
+    y, hl, ws = pd.pdssm_scan_fwd(bad_pi, t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=16)
+    assert pd.pdssm_ws_status(ws) == 3
