@@ -80,7 +80,7 @@ int pdssm_version(void);
 /*
  * Workspace bytes needed by pdssm_scan_fwd (for_bwd = 0) or by the pair
  * pdssm_scan_fwd + pdssm_scan_bwd (for_bwd = 1) at these sizes.  The
- * workspace holds the gather plans of the dictionary (phase A0), the chunk
+ * workspace holds a sanitised copy of the dictionary (phase A0), the chunk
  * transfers (Pi_c, Delta_c, v_c), the carries H_c and a status word:
  * O(B*H*ceil(L/chunk)*N), i.e. 1/chunk of the size of d.  Returns 0 when the
  * arguments are invalid.  Pure host function.
@@ -103,8 +103,8 @@ pdssm_status pdssm_select(const pdssm_dims *dims, const void *u,
                           int32_t *k_out, void *stream);
 
 /*
- * Chunked forward scan (Methodology §3).  Runs phase A0 (gather plans of the
- * dictionary), A (per chunk: local readout of the state started from zero,
+ * Chunked forward scan (Methodology §3).  Runs phase A0 (sanitised copy of
+ * the dictionary), A (per chunk: local readout of the state started from zero,
  * closed PD transfer Pi_c, Delta_c, v_c), B (carry prefix scan H_c, h_last)
  * and C (carry correction of the readout y).  Writes y [B][H][L] and, when
  * non-NULL, h_last [B][H][N] = h_{L-1} (h0 when L = 0).  h0 may be NULL

@@ -2,6 +2,7 @@
 // the launch sequence of each call.  Every call is asynchronous on the
 // caller's stream unless its declaration in pdssm.h says otherwise.
 #include <stdio.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include "common.cuh"
@@ -23,6 +24,15 @@ pdssm_status arg_fail(pdssm_status st, const char *why) {
 }
 
 bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+int stage_override() {
+    static const int v = [] {
+        const char *e = getenv("PDSSM_STAGES");
+        const int n = e ? atoi(e) : 0;
+        return (n >= 2 && n <= kMaxStages) ? n : 0;
+    }();
+    return v;
+}
 
 size_t dtype_size(pdssm_dtype t) { return t == PDSSM_BF16 ? 2 : 4; }
 
@@ -64,8 +74,8 @@ ChunkParams make_params(const pdssm_dims *dm, const WsLayout &w, void *ws, int64
     p.dict_hs = w.Hd > 1 ? dm->K * dm->N : 0;
     unsigned char *base = reinterpret_cast<unsigned char *>(ws);
     p.dict = reinterpret_cast<const int32_t *>(base + w.dict);
-    p.plan = reinterpret_cast<const int16_t *>(base + w.plan);
-    p.PW = (int)w.PW;
+    p.tab = reinterpret_cast<const uint8_t *>(base + w.tab);
+    p.fan = reinterpret_cast<const int32_t *>(base + w.fan);
     p.k = k;
     p.d = d;
     p.b = b;
@@ -82,8 +92,9 @@ ChunkParams make_params(const pdssm_dims *dm, const WsLayout &w, void *ws, int64
     const bool vec_ok = (rowb % 16) == 0;
     const bool ptr_ok = (!d || aligned(d, 16)) && (!b || aligned(b, 16)) && (!c || aligned(c, 16));
     p.bulk = (vec_ok && ptr_ok) ? 1 : 0;
-    // three stages while a stage of three tensors stays within 8 KB
-    p.ns = (3 * kTS * rowb <= 8192) ? 3 : 2;
+    // double-buffered tiles (plus L2 prefetch further ahead); PDSSM_STAGES
+    // overrides the depth (2..4) for tuning
+    p.ns = stage_override() > 0 ? stage_override() : 2;
     return p;
 }
 
@@ -154,7 +165,8 @@ static pdssm_status run_prep(const pdssm_dims *dims, const int32_t *pi_dict,
     cudaError_t e = cudaMemsetAsync(base + w.status, 0, 4, st);
     if (e != cudaSuccess) return cuda_fail(e, "status reset");
     e = launch_prep(*dims, pi_dict, pi_head_stride, reinterpret_cast<int32_t *>(base + w.dict),
-                    reinterpret_cast<int16_t *>(base + w.plan), (int)w.PW, w.Hd,
+                    reinterpret_cast<uint8_t *>(base + w.tab),
+                    reinterpret_cast<int32_t *>(base + w.fan), w.Hd,
                     reinterpret_cast<int *>(base + w.status), st);
     if (e != cudaSuccess) return cuda_fail(e, "prep");
     return PDSSM_OK;

@@ -17,10 +17,10 @@
 
 namespace pdssm {
 
+// bwd phase C warp: ring, exchange buffers (2 x kPbStride), lambda buffers
+// (2 x 64), checkpoints (16 x 64), barriers
 __host__ __device__ inline int bwd_warp_smem_bytes(int ns, int nt, int rowb) {
-    // ring + pbuf (2 x 64) + lbuf (2 x 64) + checkpoints (16 x 64) + barriers
-    return ns * nt * kTS * rowb + 4 * kMaxN * 4 + (kBwdMaxChunk / kTS) * kMaxN * 4 +
-           kMaxStages * 8;
+    return warp_smem_bytes(ns, nt, rowb, 2 * kMaxN * 4 + (kBwdMaxChunk / kTS) * kMaxN * 4);
 }
 
 template <int NPL, bool EVEN>
@@ -38,63 +38,6 @@ __device__ __forceinline__ void store_row(float *row, int lane, int N, const flo
     }
 }
 
-// Gather of one forward PD step (same plan format as the forward kernels).
-template <int NPL>
-__device__ __forceinline__ void fwd_step(float (&h)[NPL], const float (&dv)[NPL],
-                                         const float (&bv)[NPL], float *pb,
-                                         const int16_t *__restrict__ prow, int lane, int N) {
-#pragma unroll
-    for (int r = 0; r < NPL; ++r) {
-        const int e = lane * NPL + r;
-        if (e < N) pb[e] = dv[r] * h[r];
-    }
-    __syncwarp();
-    float acc[NPL];
-#pragma unroll
-    for (int r = 0; r < NPL; ++r) acc[r] = 0.f;
-    const uint4 q0 = __ldg(reinterpret_cast<const uint4 *>(prow));
-    const int G = (int)(int16_t)(q0.x & 0xffffu);
-    const int ent[7] = {(int)(int16_t)(q0.x >> 16), (int)(int16_t)(q0.y & 0xffffu),
-                        (int)(int16_t)(q0.y >> 16), (int)(int16_t)(q0.z & 0xffffu),
-                        (int)(int16_t)(q0.z >> 16), (int)(int16_t)(q0.w & 0xffffu),
-                        (int)(int16_t)(q0.w >> 16)};
-#pragma unroll
-    for (int g = 0; g < 7; ++g) {
-        if (g < G) {
-            const int e = ent[g];
-            if (e >= 0) {
-                const float val = pb[e & 127];
-                if (NPL == 1 || (e >> 7) == 0)
-                    acc[0] += val;
-                else
-                    acc[NPL - 1] += val;
-            }
-        }
-    }
-    for (int g0 = 8; g0 <= G; g0 += 8) {
-        const uint4 q = __ldg(reinterpret_cast<const uint4 *>(prow + g0));
-        const int en[8] = {(int)(int16_t)(q.x & 0xffffu), (int)(int16_t)(q.x >> 16),
-                           (int)(int16_t)(q.y & 0xffffu), (int)(int16_t)(q.y >> 16),
-                           (int)(int16_t)(q.z & 0xffffu), (int)(int16_t)(q.z >> 16),
-                           (int)(int16_t)(q.w & 0xffffu), (int)(int16_t)(q.w >> 16)};
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            if (g0 + g <= G) {
-                const int e = en[g];
-                if (e >= 0) {
-                    const float val = pb[e & 127];
-                    if (NPL == 1 || (e >> 7) == 0)
-                        acc[0] += val;
-                    else
-                        acc[NPL - 1] += val;
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < NPL; ++r) h[r] = acc[r] + bv[r];
-}
-
 // ---------------------------------------------------------------------------
 // bwd phase A: w_c = M_s^T lambda^loc_s with lambda^loc from a zero carry
 // ---------------------------------------------------------------------------
@@ -102,15 +45,15 @@ template <typename T, int NPL, bool EVEN>
 __global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_ba[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const SmemDict sd = stage_dict(p, sm_ba, warp, lane);
     const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
     if (unit >= p.units) return;
     const int N = (int)p.N, K = (int)p.K;
     const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
-    const int64_t hh = bh % p.H;
     const int64_t s = cidx * p.chunk;
     const int len = (int)imin64(p.chunk, p.L - s);
 
-    unsigned char *wbase = sm_ba + (size_t)warp * p.smem_per_warp;
+    unsigned char *wbase = sm_ba + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
     const int rowb = N * (int)sizeof(T);
     Ring<2> ring;
     ring.buf = wbase;
@@ -121,7 +64,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
     ring.ns = p.ns;
     ring.bulk = p.bulk != 0;
     float *lbuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes);
-    ring.bar0 = smem_u32(lbuf + 2 * kMaxN);
+    ring.bar0 = smem_u32(lbuf + 2 * kPbStride);
     const int64_t seq_row0 = bh * p.L;
     ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * rowb;
     ring.src[1] = reinterpret_cast<const unsigned char *>(p.c) + seq_row0 * rowb;
@@ -133,7 +76,10 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
         const int ti = tile_of(j);
         ring.issue(j, s + (int64_t)ti * kTS, min(kTS, len - ti * kTS), 2, lane);
     }
-    const int32_t *dict = p.dict + hh * p.dict_hs;
+    for (int j = p.ns; j < p.ns + kPrefetchTiles && j < ntiles; ++j) {
+        const int ti = tile_of(j);
+        ring.prefetch(s + (int64_t)ti * kTS, min(kTS, len - ti * kTS), 2, lane);
+    }
     const int64_t kbase = bh * p.L + s;
     float mu[NPL];
 #pragma unroll
@@ -165,18 +111,19 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
                 float dv[NPL], cv[NPL];
                 load_row<T, NPL, EVEN>(td + q * N, lane, N, dv);
                 load_row<T, NPL, EVEN>(tc + q * N, lane, N, cv);
-                float *lb = lbuf + (q & 1) * kMaxN;
+                float *lb = lbuf + (q & 1) * kPbStride;
 #pragma unroll
                 for (int r = 0; r < NPL; ++r) {
                     const int e = lane * NPL + r;
                     if (e < N) lb[e] = gy * cv[r] + mu[r];
                 }
                 __syncwarp();
-                const int32_t *pk = dict + (int64_t)kk * N;
+                int tgt[NPL];
+                own_targets<NPL, EVEN>(sd.map + kk * N, lane, N, tgt);
 #pragma unroll
                 for (int r = 0; r < NPL; ++r) {
                     const int e = lane * NPL + r;
-                    if (e < N) mu[r] = dv[r] * lb[__ldg(pk + e)];
+                    if (e < N) mu[r] = dv[r] * lb[tgt[r]];
                 }
             }
         }
@@ -184,6 +131,10 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
         if (j + p.ns < ntiles) {
             const int tn = tile_of(j + p.ns);
             ring.issue(stage, s + (int64_t)tn * kTS, min(kTS, len - tn * kTS), 2, lane);
+        }
+        if (j + p.ns + kPrefetchTiles < ntiles) {
+            const int tp2 = tile_of(j + p.ns + kPrefetchTiles);
+            ring.prefetch(s + (int64_t)tp2 * kTS, min(kTS, len - tp2 * kTS), 2, lane);
         }
         kreg = knext;
         gyreg = gynext;
@@ -359,15 +310,15 @@ template <typename T, int NPL, bool EVEN>
 __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_bc[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const SmemDict sd = stage_dict(p, sm_bc, warp, lane);
     const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
     if (unit >= p.units) return;
     const int N = (int)p.N, K = (int)p.K;
     const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
-    const int64_t hh = bh % p.H;
     const int64_t s = cidx * p.chunk;
     const int len = (int)imin64(p.chunk, p.L - s);
 
-    unsigned char *wbase = sm_bc + (size_t)warp * p.smem_per_warp;
+    unsigned char *wbase = sm_bc + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
     const int rowb = N * (int)sizeof(T);
     Ring<3> ring;
     ring.buf = wbase;
@@ -378,7 +329,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
     ring.ns = p.ns;
     ring.bulk = p.bulk != 0;
     float *pbuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes);
-    float *lbuf = pbuf + 2 * kMaxN;
+    float *lbuf = pbuf + 2 * kPbStride;
     float *ck = lbuf + 2 * kMaxN;   // [kBwdMaxChunk / kTS][64]
     ring.bar0 = smem_u32(ck + (kBwdMaxChunk / kTS) * kMaxN);
     const int64_t seq_row0 = bh * p.L;
@@ -395,9 +346,10 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
         const int ti = tile_of(m);
         ring.issue(m, s + (int64_t)ti * kTS, min(kTS, len - ti * kTS), nt_of(m), lane);
     }
+    for (int m = p.ns; m < p.ns + kPrefetchTiles && m < ntiles; ++m)
+        ring.prefetch(s + (int64_t)m * kTS, min(kTS, len - m * kTS), 3, lane);
 
-    const int32_t *dict = p.dict + hh * p.dict_hs;
-    const int16_t *plan = p.plan + (hh * p.dict_hs / p.N) * 32 * p.PW;
+    clear_pb(pbuf, lane);
     const int64_t kbase = bh * p.L + s;
     float h[NPL], mu[NPL];
 #pragma unroll
@@ -448,8 +400,9 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
                     float dv[NPL], bv[NPL];
                     load_row<T, NPL, EVEN>(td + q * N, lane, N, dv);
                     load_row<T, NPL, EVEN>(tb + q * N, lane, N, bv);
-                    fwd_step<NPL>(h, dv, bv, pbuf + (q & 1) * kMaxN,
-                                  plan + ((int64_t)kk * 32 + lane) * p.PW, lane, N);
+                    pd_gather_step<NPL>(h, dv, bv, pbuf + (q & 1) * kPbStride,
+                                        sd.tab + kk * (kDcap * 64), sd.fan[kk],
+                                        sd.map + kk * N, lane, N);
                 }
             }
         } else {
@@ -469,8 +422,9 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
                     float dv[NPL], bv[NPL];
                     load_row<T, NPL, EVEN>(td + q * N, lane, N, dv);
                     load_row<T, NPL, EVEN>(tb + q * N, lane, N, bv);
-                    fwd_step<NPL>(hs[q + 1], dv, bv, pbuf + (q & 1) * kMaxN,
-                                  plan + ((int64_t)kk * 32 + lane) * p.PW, lane, N);
+                    pd_gather_step<NPL>(hs[q + 1], dv, bv, pbuf + (q & 1) * kPbStride,
+                                        sd.tab + kk * (kDcap * 64), sd.fan[kk],
+                                        sd.map + kk * N, lane, N);
                 }
             }
 #pragma unroll
@@ -493,12 +447,13 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
                     store_row<NPL, EVEN>(p.g_b + row, lane, N, lam);
                     store_row<NPL, EVEN>(p.g_c + row, lane, N, gc);
                     __syncwarp();
-                    const int32_t *pk = dict + (int64_t)kk * N;
+                    int tgt[NPL];
+                    own_targets<NPL, EVEN>(sd.map + kk * N, lane, N, tgt);
                     float gd[NPL];
 #pragma unroll
                     for (int r = 0; r < NPL; ++r) {
                         const int e = lane * NPL + r;
-                        const float gl = e < N ? lb[__ldg(pk + e)] : 0.f;
+                        const float gl = e < N ? lb[tgt[r]] : 0.f;
                         gd[r] = hs[q][r] * gl;
                         mu[r] = dv[r] * gl;
                     }
@@ -511,6 +466,10 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
             const int mn = m + p.ns;
             const int tn = tile_of(mn);
             ring.issue(stage, s + (int64_t)tn * kTS, min(kTS, len - tn * kTS), nt_of(mn), lane);
+        }
+        if (m + p.ns + kPrefetchTiles < ntiles) {
+            const int tp2 = m + p.ns + kPrefetchTiles;
+            ring.prefetch(s + (int64_t)tp2 * kTS, min(kTS, len - tp2 * kTS), 3, lane);
         }
         kreg = knext;
         gyreg = gynext;
@@ -544,16 +503,16 @@ static cudaError_t launch_chunk_b(KernT kern, const ChunkParams &p, size_t smem,
 template <typename T>
 static cudaError_t bwdA_t(ChunkParams p, cudaStream_t st) {
     const int rowb = (int)p.N * (int)sizeof(T);
-    p.smem_per_warp = (p.ns * 2 * kTS * rowb + 2 * kMaxN * 4 + kMaxStages * 8 + 127) / 128 * 128;
-    const size_t smem = (size_t)kWPC * p.smem_per_warp;
+    p.smem_per_warp = warp_smem_bytes(p.ns, 2, rowb);
+    const size_t smem = (size_t)dict_region_bytes(p) + (size_t)kWPC * p.smem_per_warp;
     PDSSM_DISPATCH_B(k_bwdA, p, st, smem);
 }
 
 template <typename T>
 static cudaError_t bwdC_t(ChunkParams p, cudaStream_t st) {
     const int rowb = (int)p.N * (int)sizeof(T);
-    p.smem_per_warp = (bwd_warp_smem_bytes(p.ns, 3, rowb) + 127) / 128 * 128;
-    const size_t smem = (size_t)kWPC * p.smem_per_warp;
+    p.smem_per_warp = bwd_warp_smem_bytes(p.ns, 3, rowb);
+    const size_t smem = (size_t)dict_region_bytes(p) + (size_t)kWPC * p.smem_per_warp;
     PDSSM_DISPATCH_B(k_bwdC, p, st, smem);
 }
 

@@ -24,6 +24,10 @@ constexpr int kWPC = 4;        // warps (units) per CTA in the chunk kernels
 constexpr int kMaxN = 64;
 constexpr int kMaxStages = 4;
 constexpr int kBwdMaxChunk = 256;   // checkpoints of one chunk kept in shared memory
+constexpr int kDcap = 8;            // sources per target held in the slot table
+constexpr int kPrefetchTiles = 4;   // tiles prefetched into L2 ahead of the staged ones
+constexpr int kZeroSlot = 64;       // exchange-buffer entry that always holds 0
+constexpr int kPbStride = 80;       // floats per exchange buffer (64 + zero slot, padded)
 constexpr unsigned kFull = 0xffffffffu;
 
 // status word bits (first int of the workspace)
@@ -33,8 +37,8 @@ enum : int { kStBadIndex = 1, kStTimeout = 2 };
 // workspace layout (all offsets 256-byte aligned)
 // ---------------------------------------------------------------------------
 struct WsLayout {
-    size_t status, dict, plan, Pi, Dl, v, Hc, wc, lam, total;
-    int64_t C, Hd, PW;
+    size_t status, dict, tab, fan, Pi, Dl, v, Hc, wc, lam, total;
+    int64_t C, Hd;
 };
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
@@ -46,13 +50,13 @@ inline WsLayout ws_layout(const pdssm_dims &dm, int64_t pi_hs, int64_t chunk,
     WsLayout w{};
     w.C = dm.L > 0 ? (dm.L + chunk - 1) / chunk : 0;
     w.Hd = pi_hs ? dm.H : 1;
-    w.PW = 8 * ((dm.N + 1 + 7) / 8);   // entries per plan row: count + sources
     const size_t units = (size_t)(dm.B * dm.H * w.C);
     const size_t vecs = units * (size_t)dm.N * 4;
     size_t o = 0;
     w.status = o; o += 256;
     w.dict = o;   o = align256(o + (size_t)(w.Hd * dm.K * dm.N) * 4);
-    w.plan = o;   o = align256(o + (size_t)(w.Hd * dm.K * 32 * w.PW) * 2);
+    w.tab = o;    o = align256(o + (size_t)(w.Hd * dm.K * kDcap * 64));
+    w.fan = o;    o = align256(o + (size_t)(w.Hd * dm.K) * 4);
     w.Pi = o;     o = align256(o + vecs);
     w.Dl = o;     o = align256(o + vecs);
     w.v = o;      o = align256(o + vecs);
@@ -72,8 +76,8 @@ struct ChunkParams {
     int64_t B, H, L, N, K, C, chunk, units;
     int64_t dict_hs;          // head stride of the sanitised dictionary (0 or K*N)
     const int32_t *dict;      // sanitised dictionary [Hd][K][N]
-    const int16_t *plan;      // gather plans [Hd][K][32][PW]
-    int PW;
+    const uint8_t *tab;       // slot tables [Hd][K][kDcap][64]: s-th source of each target
+    const int32_t *fan;       // largest fan-in of each map [Hd][K]
     const int32_t *k;
     const void *d, *b, *c;
     const float *h0;
@@ -139,6 +143,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
         "%2, [%3];" ::"r"(dst),
         "l"(src), "r"(bytes), "r"(bar)
         : "memory");
+}
+
+// Bulk prefetch of global memory into L2 (no shared memory involved).
+__device__ __forceinline__ void bulk_prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
@@ -239,6 +248,89 @@ __device__ __forceinline__ int load_k(const int32_t *kp, int64_t idx, bool valid
 }
 
 // ---------------------------------------------------------------------------
+// dictionary in shared memory and the PD step as a shared-memory scatter
+// ---------------------------------------------------------------------------
+
+// Targets pi_k(e) of the elements a lane owns (e = lane*NPL + r).
+template <int NPL, bool EVEN>
+__device__ __forceinline__ void own_targets(const int *pk, int lane, int N, int (&tgt)[NPL]) {
+    if constexpr (NPL == 2 && EVEN) {
+        if (2 * lane < N) {
+            const int2 q = *reinterpret_cast<const int2 *>(pk + 2 * lane);
+            tgt[0] = q.x;
+            tgt[1] = q.y;
+        } else {
+            tgt[0] = 0;
+            tgt[1] = 0;
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) {
+            const int e = lane * NPL + r;
+            tgt[r] = e < N ? pk[e] : 0;
+        }
+    }
+}
+
+// One PD step h <- P_k diag(d) h + b on the lane-owned state, as a gather:
+// every lane stores d[j] h[j] of the sources it owns into `pb` (this step's
+// buffer of an alternating pair, entry kZeroSlot permanently 0), then sums,
+// for each element it owns, the sources listed by the map's slot table in
+// ascending j (padding entries point at the zero slot).  One warp barrier per
+// step; no atomics, so the result is deterministic.  Maps whose fan-in
+// exceeds kDcap scan all N sources instead.
+template <int NPL>
+__device__ __forceinline__ void pd_gather_step(float (&h)[NPL], const float (&dv)[NPL],
+                                               const float (&bv)[NPL], float *pb,
+                                               const uint8_t *tabk, int Dk, const int *pk,
+                                               int lane, int N) {
+    if constexpr (NPL == 2) {
+        if (2 * lane + 1 < N) {
+            *reinterpret_cast<float2 *>(pb + 2 * lane) = make_float2(dv[0] * h[0], dv[1] * h[1]);
+        } else if (2 * lane < N) {
+            pb[2 * lane] = dv[0] * h[0];
+        }
+    } else {
+        if (lane < N) pb[lane] = dv[0] * h[0];
+    }
+    __syncwarp();
+    float acc[NPL];
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) acc[r] = 0.f;
+    if (Dk <= kDcap) {
+        if constexpr (NPL == 2) {
+            const uint16_t *t16 = reinterpret_cast<const uint16_t *>(tabk) + lane;
+#pragma unroll 4
+            for (int sl = 0; sl < Dk; ++sl) {
+                const unsigned w = t16[sl * 32];
+                acc[0] += pb[w & 0xffu];
+                acc[1] += pb[w >> 8];
+            }
+        } else {
+            const uint8_t *t8 = tabk + lane;
+#pragma unroll 4
+            for (int sl = 0; sl < Dk; ++sl) acc[0] += pb[t8[sl * 64]];
+        }
+    } else {
+        for (int j = 0; j < N; ++j) {
+            const int t = pk[j];
+            const float v = pb[j];
+#pragma unroll
+            for (int r = 0; r < NPL; ++r)
+                if (t == lane * NPL + r) acc[r] += v;
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) h[r] = (lane * NPL + r < N) ? acc[r] + bv[r] : 0.f;
+}
+
+// Both exchange buffers of a warp: zero, including the zero slots.
+__device__ __forceinline__ void clear_pb(float *pb, int lane) {
+    for (int i = lane; i < 2 * kPbStride; i += 32) pb[i] = 0.f;
+    __syncwarp();
+}
+
+// ---------------------------------------------------------------------------
 // per-warp staging ring: NT tensors, ns stages of kTS rows each
 // ---------------------------------------------------------------------------
 template <int NT>
@@ -288,6 +380,17 @@ struct Ring {
         }
     }
 
+    // Pull rows [t0, t0 + n) of the first nt tensors towards L2 so that the
+    // later staging copy of them hits L2 instead of waiting on HBM.
+    __device__ void prefetch(int64_t t0, int n, int nt, int lane) const {
+        if (bulk && lane == 0 && n > 0) {
+            const uint32_t bytes = (uint32_t)(n * rowb);
+#pragma unroll
+            for (int q = 0; q < NT; ++q)
+                if (q < nt) bulk_prefetch_l2(src[q] + t0 * rowb, bytes);
+        }
+    }
+
     __device__ bool wait(int stage, uint32_t parity) const {
         if (!bulk) return true;
         return mbar_wait_bounded(bar0 + 8u * stage, parity);
@@ -313,13 +416,70 @@ __device__ void ring_abort(const Ring<NT> &ring, int first, int last, int *statu
     __syncwarp();
 }
 
+// Dynamic shared memory of the chunk kernels:
+//   [dictionary slots][warp 0][warp 1]...
+//   dictionary slot = [map K x N ints][slot tables K x kDcap x 64 bytes][fan-in K ints]
+//   warp = [staging ring][exchange buffers 2 x kPbStride floats][extra][barriers]
+__host__ __device__ inline int dict_slot_bytes(int K, int N) {
+    return (K * N * 4 + K * kDcap * 64 + K * 4 + 127) / 128 * 128;
+}
+__host__ __device__ inline int warp_smem_bytes(int ns, int nt, int rowb, int extra = 0) {
+    return (ns * nt * kTS * rowb + 2 * kPbStride * 4 + extra + kMaxStages * 8 + 127) / 128 * 128;
+}
+
+struct SmemDict {
+    const int *map;        // [K][N]
+    const uint8_t *tab;    // [K][kDcap][64]
+    const int *fan;        // [K]
+};
+
+__device__ __forceinline__ void copy_slot(unsigned char *dst, const ChunkParams &p, int64_t dk,
+                                          int tid, int nthr) {
+    const int K = (int)p.K, N = (int)p.N;
+    int *m = reinterpret_cast<int *>(dst);
+    uint32_t *t = reinterpret_cast<uint32_t *>(dst + K * N * 4);
+    int *f = reinterpret_cast<int *>(dst + K * N * 4 + K * kDcap * 64);
+    const int32_t *gm = p.dict + dk * K * N;
+    const uint32_t *gt = reinterpret_cast<const uint32_t *>(p.tab + dk * K * kDcap * 64);
+    const int32_t *gf = p.fan + dk * K;
+    for (int i = tid; i < K * N; i += nthr) m[i] = __ldg(gm + i);
+    for (int i = tid; i < K * kDcap * 16; i += nthr) t[i] = __ldg(gt + i);
+    for (int i = tid; i < K; i += nthr) f[i] = __ldg(gf + i);
+}
+
+// Loads the dictionary used by this CTA's warps into shared memory and
+// returns this warp's view.  Must be reached by every thread of the CTA.
+__device__ __forceinline__ SmemDict stage_dict(const ChunkParams &p, unsigned char *smem,
+                                               int warp, int lane) {
+    const int K = (int)p.K, N = (int)p.N;
+    const int slot = dict_slot_bytes(K, N);
+    unsigned char *mine = smem;
+    if (p.dict_hs == 0) {
+        copy_slot(smem, p, 0, threadIdx.x, blockDim.x);
+    } else {
+        mine = smem + warp * slot;
+        const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
+        if (unit < p.units) copy_slot(mine, p, (unit / p.C) % p.H, lane, 32);
+    }
+    __syncthreads();
+    SmemDict sd;
+    sd.map = reinterpret_cast<const int *>(mine);
+    sd.tab = mine + K * N * 4;
+    sd.fan = reinterpret_cast<const int *>(mine + K * N * 4 + K * kDcap * 64);
+    return sd;
+}
+
+__host__ __device__ inline int dict_region_bytes(const ChunkParams &p) {
+    return (p.dict_hs == 0 ? 1 : kWPC) * dict_slot_bytes((int)p.K, (int)p.N);
+}
+
 // ---------------------------------------------------------------------------
 // host launchers (one per kernel family)
 // ---------------------------------------------------------------------------
 cudaError_t launch_select(const pdssm_dims &dm, const void *u, pdssm_dtype ut, const float *W,
                           int32_t *k_out, cudaStream_t st);
 cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
-                        int16_t *plan, int PW, int64_t Hd, int *status, cudaStream_t st);
+                        uint8_t *tab, int32_t *fan, int64_t Hd, int *status, cudaStream_t st);
 cudaError_t launch_validate(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs,
                             const int32_t *k, int *counts, cudaStream_t st);
 cudaError_t launch_phaseA(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st);

@@ -4,7 +4,7 @@
 //   phase B  carry prefix scan over chunks: H_c = P_{Pi_c} diag(Delta_c) H_{c-1} + v_c;
 //   phase C  carry correction of the readout.
 //
-// Phase C here never rebuilds the state.  By linearity
+// Phase C never rebuilds the state.  By linearity
 //   h_t = v_t + P_{Pi_{s..t}} diag(Delta_{s..t}) H_{c-1},
 // so y_t = <c_t, v_t> + sum_j c_t[pos_t(j)] * w_t(j), where each carry
 // coordinate j travels one path pos_t(j) = pi_{k_t}(pos_{t-1}(j)) with weight
@@ -12,81 +12,13 @@
 // Phase A stores <c_t, v_t> in y; phase C adds the path sums.  Every
 // correction term is a product (no cancellation, no division), which keeps
 // the stiff regime (d down to 1e-4, products underflowing to 0) exact.
+//
+// The dictionary and its slot tables live in shared memory (one copy per CTA
+// when all heads share it, one per warp otherwise); the state update is the
+// deterministic slot gather pd_gather_step.
 #include "common.cuh"
 
 namespace pdssm {
-
-// Smem layout of one warp in the chunk kernels:
-//   [ns stages x NT tensors x kTS rows][pbuf 2 x 64 floats][ns mbarriers]
-__host__ __device__ inline int warp_smem_bytes(int ns, int nt, int rowb, int extra) {
-    return ns * nt * kTS * rowb + 2 * kMaxN * 4 + extra + kMaxStages * 8;
-}
-
-// Gather of one PD step: acc[r] = sum over sources j with pi(j) = own
-// element r of pb[j], listed in ascending j by the plan row.
-template <int NPL>
-__device__ __forceinline__ void plan_gather(const int16_t *__restrict__ prow, const float *pb,
-                                            float (&acc)[NPL]) {
-    const uint4 q0 = __ldg(reinterpret_cast<const uint4 *>(prow));
-    const int G = (int)(int16_t)(q0.x & 0xffffu);
-    const int ent[7] = {(int)(int16_t)(q0.x >> 16), (int)(int16_t)(q0.y & 0xffffu),
-                        (int)(int16_t)(q0.y >> 16), (int)(int16_t)(q0.z & 0xffffu),
-                        (int)(int16_t)(q0.z >> 16), (int)(int16_t)(q0.w & 0xffffu),
-                        (int)(int16_t)(q0.w >> 16)};
-#pragma unroll
-    for (int g = 0; g < 7; ++g) {
-        if (g < G) {
-            const int e = ent[g];
-            if (e >= 0) {
-                const float val = pb[e & 127];
-                if (NPL == 1 || (e >> 7) == 0)
-                    acc[0] += val;
-                else
-                    acc[NPL - 1] += val;
-            }
-        }
-    }
-    for (int g0 = 8; g0 <= G; g0 += 8) {
-        const uint4 q = __ldg(reinterpret_cast<const uint4 *>(prow + g0));
-        const int en[8] = {(int)(int16_t)(q.x & 0xffffu), (int)(int16_t)(q.x >> 16),
-                           (int)(int16_t)(q.y & 0xffffu), (int)(int16_t)(q.y >> 16),
-                           (int)(int16_t)(q.z & 0xffffu), (int)(int16_t)(q.z >> 16),
-                           (int)(int16_t)(q.w & 0xffffu), (int)(int16_t)(q.w >> 16)};
-#pragma unroll
-        for (int g = 0; g < 8; ++g) {
-            if (g0 + g <= G) {
-                const int e = en[g];
-                if (e >= 0) {
-                    const float val = pb[e & 127];
-                    if (NPL == 1 || (e >> 7) == 0)
-                        acc[0] += val;
-                    else
-                        acc[NPL - 1] += val;
-                }
-            }
-        }
-    }
-}
-
-// One PD step on the lane-owned state h: h <- P_k diag(d) h + b.
-// pb is this step's exchange buffer (N floats); the caller alternates two.
-template <int NPL>
-__device__ __forceinline__ void pd_step(float (&h)[NPL], const float (&dv)[NPL],
-                                        const float (&bv)[NPL], float *pb,
-                                        const int16_t *__restrict__ prow, int lane, int N) {
-#pragma unroll
-    for (int r = 0; r < NPL; ++r) {
-        const int e = lane * NPL + r;
-        if (e < N) pb[e] = dv[r] * h[r];
-    }
-    __syncwarp();
-    float acc[NPL];
-#pragma unroll
-    for (int r = 0; r < NPL; ++r) acc[r] = 0.f;
-    plan_gather<NPL>(prow, pb, acc);
-#pragma unroll
-    for (int r = 0; r < NPL; ++r) h[r] = acc[r] + bv[r];
-}
 
 // ---------------------------------------------------------------------------
 // phase A
@@ -95,18 +27,18 @@ template <typename T, int NPL, bool EVEN>
 __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_a[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const SmemDict sd = stage_dict(p, sm_a, warp, lane);
     const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
     if (unit >= p.units) return;
     const int N = (int)p.N, K = (int)p.K;
     const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
-    const int64_t hh = bh % p.H;
     const int64_t s = cidx * p.chunk;
     const int len = (int)imin64(p.chunk, p.L - s);
     const bool with_y = p.y != nullptr;
     const int nt = with_y ? 3 : 2;
 
-    unsigned char *wbase = sm_a + (size_t)warp * p.smem_per_warp;
     const int rowb = N * (int)sizeof(T);
+    unsigned char *wbase = sm_a + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
     Ring<3> ring;
     ring.buf = wbase;
     ring.rowb = rowb;
@@ -116,7 +48,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
     ring.ns = p.ns;
     ring.bulk = p.bulk != 0;
     float *pbuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes);
-    ring.bar0 = smem_u32(pbuf + 2 * kMaxN);
+    ring.bar0 = smem_u32(pbuf + 2 * kPbStride);
     const int64_t seq_row0 = bh * p.L;
     ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * rowb;
     ring.src[1] = reinterpret_cast<const unsigned char *>(p.b) + seq_row0 * rowb;
@@ -127,9 +59,11 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
     const int ntiles = (len + kTS - 1) / kTS;
     for (int i = 0; i < p.ns && i < ntiles; ++i)
         ring.issue(i, s + (int64_t)i * kTS, min(kTS, len - i * kTS), nt, lane);
+    for (int i = p.ns; i < p.ns + kPrefetchTiles && i < ntiles; ++i)
+        ring.prefetch(s + (int64_t)i * kTS, min(kTS, len - i * kTS), nt, lane);
 
-    const int32_t *dict = p.dict + hh * p.dict_hs;
-    const int16_t *plan = p.plan + (hh * p.dict_hs / p.N) * 32 * p.PW;
+    clear_pb(pbuf, lane);
+
     float h[NPL], Dl[NPL];
     int pos[NPL];
 #pragma unroll
@@ -160,22 +94,22 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
             yp[q] = 0.f;
             if (q < n) {
                 const int kk = __shfl_sync(kFull, kreg, q);
+                const int *pk = sd.map + kk * N;
                 const T *rd = td + q * N;
                 float dv[NPL], bv[NPL];
                 load_row<T, NPL, EVEN>(rd, lane, N, dv);
                 load_row<T, NPL, EVEN>(tb + q * N, lane, N, bv);
                 // transfer tracking: Delta picks up d at the column's current
                 // position, then the selected map moves the column
-                const int32_t *pk = dict + (int64_t)kk * N;
 #pragma unroll
                 for (int r = 0; r < NPL; ++r) {
                     if (lane * NPL + r < N) {
                         Dl[r] *= to_f<T>(rd[pos[r]]);
-                        pos[r] = __ldg(pk + pos[r]);
+                        pos[r] = pk[pos[r]];
                     }
                 }
-                const int16_t *prow = plan + ((int64_t)kk * 32 + lane) * p.PW;
-                pd_step<NPL>(h, dv, bv, pbuf + (q & 1) * kMaxN, prow, lane, N);
+                pd_gather_step<NPL>(h, dv, bv, pbuf + (q & 1) * kPbStride,
+                                    sd.tab + kk * (kDcap * 64), sd.fan[kk], pk, lane, N);
                 if (with_y) {
                     float cv[NPL];
                     load_row<T, NPL, EVEN>(tc + q * N, lane, N, cv);
@@ -194,6 +128,10 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
         if (i + p.ns < ntiles)
             ring.issue(stage, s + (int64_t)(i + p.ns) * kTS, min(kTS, len - (i + p.ns) * kTS), nt,
                        lane);
+        {
+            const int pf = i + p.ns + kPrefetchTiles;
+            if (pf < ntiles) ring.prefetch(s + (int64_t)pf * kTS, min(kTS, len - pf * kTS), nt, lane);
+        }
         kreg = knext;
     }
     const int64_t o = unit * p.N;
@@ -215,17 +153,17 @@ template <typename T, int NPL, bool EVEN>
 __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_c[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const SmemDict sd = stage_dict(p, sm_c, warp, lane);
     const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
     if (unit >= p.units) return;
     const int N = (int)p.N, K = (int)p.K;
     const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
     if (cidx == 0 && p.h0 == nullptr) return;   // zero initial state: nothing to correct
-    const int64_t hh = bh % p.H;
     const int64_t s = cidx * p.chunk;
     const int len = (int)imin64(p.chunk, p.L - s);
 
-    unsigned char *wbase = sm_c + (size_t)warp * p.smem_per_warp;
     const int rowb = N * (int)sizeof(T);
+    unsigned char *wbase = sm_c + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
     Ring<2> ring;
     ring.buf = wbase;
     ring.rowb = rowb;
@@ -234,7 +172,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
     ring.stage_bytes = 2 * ring.tens_bytes;
     ring.ns = p.ns;
     ring.bulk = p.bulk != 0;
-    ring.bar0 = smem_u32(wbase + p.ns * ring.stage_bytes + 2 * kMaxN * 4);
+    ring.bar0 = smem_u32(wbase + p.ns * ring.stage_bytes + 2 * kPbStride * 4);
     const int64_t seq_row0 = bh * p.L;
     ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * rowb;
     ring.src[1] = reinterpret_cast<const unsigned char *>(p.c) + seq_row0 * rowb;
@@ -243,8 +181,9 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
     const int ntiles = (len + kTS - 1) / kTS;
     for (int i = 0; i < p.ns && i < ntiles; ++i)
         ring.issue(i, s + (int64_t)i * kTS, min(kTS, len - i * kTS), 2, lane);
+    for (int i = p.ns; i < p.ns + kPrefetchTiles && i < ntiles; ++i)
+        ring.prefetch(s + (int64_t)i * kTS, min(kTS, len - i * kTS), 2, lane);
 
-    const int32_t *dict = p.dict + hh * p.dict_hs;
     float w[NPL];
     int pos[NPL];
 #pragma unroll
@@ -276,7 +215,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
             yp[q] = 0.f;
             if (q < n) {
                 const int kk = __shfl_sync(kFull, kreg, q);
-                const int32_t *pk = dict + (int64_t)kk * N;
+                const int *pk = sd.map + kk * N;
                 const T *rd = td + q * N;
                 const T *rc = tc + q * N;
                 float acc = 0.f;
@@ -284,7 +223,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
                 for (int r = 0; r < NPL; ++r) {
                     if (lane * NPL + r < N) {
                         w[r] *= to_f<T>(rd[pos[r]]);
-                        pos[r] = __ldg(pk + pos[r]);
+                        pos[r] = pk[pos[r]];
                         acc += to_f<T>(rc[pos[r]]) * w[r];
                     }
                 }
@@ -297,6 +236,10 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
         if (i + p.ns < ntiles)
             ring.issue(stage, s + (int64_t)(i + p.ns) * kTS, min(kTS, len - (i + p.ns) * kTS), 2,
                        lane);
+        {
+            const int pf = i + p.ns + kPrefetchTiles;
+            if (pf < ntiles) ring.prefetch(s + (int64_t)pf * kTS, min(kTS, len - pf * kTS), 2, lane);
+        }
         kreg = knext;
     }
 }
@@ -307,6 +250,11 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
 // (2) warp 0 chains the segment aggregates from h0, (3) each warp re-applies
 // its segment's transfers from its segment carry and stores every H_c.
 // ---------------------------------------------------------------------------
+
+// out = P_P diag(D) x + V for an arbitrary (composed) index map P: every
+// lane scans all N sources in ascending j (maps composed over a chunk often
+// collapse onto a few targets, so no bounded fan-in can be assumed).
+// sP, sZ are this warp's scratch rows.  x and out may alias.
 template <int NPL>
 __device__ __forceinline__ void apply_scatter(const int (&P)[NPL], const float (&D)[NPL],
                                               const float (&V)[NPL], const float (&x)[NPL],
@@ -324,6 +272,7 @@ __device__ __forceinline__ void apply_scatter(const int (&P)[NPL], const float (
     float acc[NPL];
 #pragma unroll
     for (int r = 0; r < NPL; ++r) acc[r] = 0.f;
+#pragma unroll 4
     for (int j = 0; j < N; ++j) {
         const int pj = sP[j];
         const float zj = sZ[j];
@@ -333,7 +282,7 @@ __device__ __forceinline__ void apply_scatter(const int (&P)[NPL], const float (
     }
     __syncwarp();
 #pragma unroll
-    for (int r = 0; r < NPL; ++r) out[r] = acc[r] + V[r];
+    for (int r = 0; r < NPL; ++r) out[r] = lane * NPL + r < N ? acc[r] + V[r] : 0.f;
 }
 
 template <int NPL>
@@ -363,13 +312,13 @@ __global__ void k_phaseB(const ChunkParams p) {
     const int N = (int)p.N;
     const int64_t bh = blockIdx.x;
     const int64_t C = p.C;
-    int *sPall = reinterpret_cast<int *>(sm_b);                 // [nw][64]
+    int *sPall = reinterpret_cast<int *>(sm_b);                    // [nw][64]
     float *sZall = reinterpret_cast<float *>(sPall + nw * kMaxN);  // [nw][64]
-    float *sDall = sZall + nw * kMaxN;                          // [nw][64]
-    int *aggP = reinterpret_cast<int *>(sDall + nw * kMaxN);    // [nw][64]
+    float *sDall = sZall + nw * kMaxN;                             // [nw][64]
+    int *aggP = reinterpret_cast<int *>(sDall + nw * kMaxN);       // [nw][64]
     float *aggD = reinterpret_cast<float *>(aggP + nw * kMaxN);
     float *aggV = aggD + nw * kMaxN;
-    float *carry = aggV + nw * kMaxN;                           // [nw][64]
+    float *carry = aggV + nw * kMaxN;                              // [nw][64]
     int *sP = sPall + warp * kMaxN;
     float *sZ = sZall + warp * kMaxN;
     float *sD = sDall + warp * kMaxN;
@@ -378,14 +327,17 @@ __global__ void k_phaseB(const ChunkParams p) {
     const int64_t u0 = bh * C;
 
     // (1) segment aggregate: T_{c1-1} o ... o T_{c0}
-    int aP[NPL];
-    float aD[NPL], aV[NPL];
     if (c0 < c1) {
+        int aP[NPL];
+        float aD[NPL], aV[NPL];
         load_transfer<NPL>(p, u0 + c0, lane, aP, aD, aV);
+        int P2[NPL];
+        float D2[NPL], V2[NPL];
+        if (c0 + 1 < c1) load_transfer<NPL>(p, u0 + c0 + 1, lane, P2, D2, V2);
         for (int64_t c = c0 + 1; c < c1; ++c) {
-            int P2[NPL];
-            float D2[NPL], V2[NPL];
-            load_transfer<NPL>(p, u0 + c, lane, P2, D2, V2);
+            int Pn[NPL];
+            float Dn[NPL], Vn[NPL];
+            if (c + 1 < c1) load_transfer<NPL>(p, u0 + c + 1, lane, Pn, Dn, Vn);
 #pragma unroll
             for (int r = 0; r < NPL; ++r) {
                 const int e = lane * NPL + r;
@@ -403,13 +355,16 @@ __global__ void k_phaseB(const ChunkParams p) {
                 nD[r] = aD[r] * sD[aP[r]];
             }
             __syncwarp();
-            float nV[NPL];
-            apply_scatter<NPL>(P2, D2, V2, aV, nV, sP, sZ, N, lane);
+            apply_scatter<NPL>(P2, D2, V2, aV, aV, sP, sZ, N, lane);
 #pragma unroll
             for (int r = 0; r < NPL; ++r) {
                 aP[r] = nP[r];
                 aD[r] = nD[r];
-                aV[r] = nV[r];
+                if (c + 1 < c1) {
+                    P2[r] = Pn[r];
+                    D2[r] = Dn[r];
+                    V2[r] = Vn[r];
+                }
             }
         }
 #pragma unroll
@@ -466,15 +421,29 @@ __global__ void k_phaseB(const ChunkParams p) {
         const int e = lane * NPL + r;
         x[r] = e < N ? carry[warp * kMaxN + e] : 0.f;
     }
-    for (int64_t c = c0; c < c1; ++c) {
+    if (c0 < c1) {
         int P[NPL];
         float D[NPL], V[NPL];
-        load_transfer<NPL>(p, u0 + c, lane, P, D, V);
-        apply_scatter<NPL>(P, D, V, x, x, sP, sZ, N, lane);
+        load_transfer<NPL>(p, u0 + c0, lane, P, D, V);
+        for (int64_t c = c0; c < c1; ++c) {
+            int Pn[NPL];
+            float Dn[NPL], Vn[NPL];
 #pragma unroll
-        for (int r = 0; r < NPL; ++r) {
-            const int e = lane * NPL + r;
-            if (e < N) p.Hc[(u0 + c) * p.N + e] = x[r];
+            for (int r = 0; r < NPL; ++r) {
+                Pn[r] = 0;
+                Dn[r] = 0.f;
+                Vn[r] = 0.f;
+            }
+            if (c + 1 < c1) load_transfer<NPL>(p, u0 + c + 1, lane, Pn, Dn, Vn);
+            apply_scatter<NPL>(P, D, V, x, x, sP, sZ, N, lane);
+#pragma unroll
+            for (int r = 0; r < NPL; ++r) {
+                const int e = lane * NPL + r;
+                if (e < N) p.Hc[(u0 + c) * p.N + e] = x[r];
+                P[r] = Pn[r];
+                D[r] = Dn[r];
+                V[r] = Vn[r];
+            }
         }
     }
 }
@@ -505,16 +474,16 @@ static cudaError_t launch_chunk(KernT kern, const ChunkParams &p, size_t smem, c
 template <typename T>
 static cudaError_t phaseA_t(ChunkParams p, cudaStream_t st) {
     const int rowb = (int)p.N * (int)sizeof(T);
-    p.smem_per_warp = (warp_smem_bytes(p.ns, 3, rowb, 0) + 127) / 128 * 128;
-    const size_t smem = (size_t)kWPC * p.smem_per_warp;
+    p.smem_per_warp = warp_smem_bytes(p.ns, 3, rowb);
+    const size_t smem = (size_t)dict_region_bytes(p) + (size_t)kWPC * p.smem_per_warp;
     PDSSM_DISPATCH(k_phaseA, p, st, smem);
 }
 
 template <typename T>
 static cudaError_t phaseC_t(ChunkParams p, cudaStream_t st) {
     const int rowb = (int)p.N * (int)sizeof(T);
-    p.smem_per_warp = (warp_smem_bytes(p.ns, 2, rowb, 0) + 127) / 128 * 128;
-    const size_t smem = (size_t)kWPC * p.smem_per_warp;
+    p.smem_per_warp = warp_smem_bytes(p.ns, 2, rowb);
+    const size_t smem = (size_t)dict_region_bytes(p) + (size_t)kWPC * p.smem_per_warp;
     PDSSM_DISPATCH(k_phaseC, p, st, smem);
 }
 

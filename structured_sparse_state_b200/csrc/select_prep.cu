@@ -1,6 +1,5 @@
 // Hard selection (fused logits + first argmax), dictionary preparation
-// (phase A0: gather plans of each one-hot column selector) and index
-// validation.
+// (phase A0) and index validation.
 //
 // Flash PD-SSM technical summary, Methodology §1: at each step the input u_t
 // gives K scores through a linear map and the single highest-scoring
@@ -117,24 +116,25 @@ cudaError_t launch_select(const pdssm_dims &dm, const void *u, pdssm_dtype ut, c
 }
 
 // ---------------------------------------------------------------------------
-// k_prep (phase A0): one warp per (dictionary, k).  Writes a sanitised copy
-// of the map (entries clamped into [0, N), flagged) and the gather plan:
-// for lane l, the sources j whose target pi(j) is an element lane l owns,
-// in ascending j, each encoded as j | (r << 7) with r = target - l*NPL.
-// Row layout [count G][e_1 .. e_G][-1 ...]; G is the maximum over lanes, so
-// every lane of a warp loops the same number of times.
+// k_prep (phase A0): one warp per dictionary map.  Writes
+//   * a sanitised copy of the map (entries clamped into [0, N), flagged);
+//   * its slot table: tab[s][i] = the s-th source j (ascending) with
+//     pi(j) = i, for s < kDcap, or kZeroSlot when i has fewer sources;
+//   * its largest fan-in (the number of slots a step must visit; above kDcap
+//     the kernels scan all sources instead).
 // ---------------------------------------------------------------------------
 __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *__restrict__ dict,
-                       int16_t *__restrict__ plan, int PW, int64_t nmaps, int K, int N, int npl,
-                       int *status) {
+                       uint8_t *__restrict__ tab, int32_t *__restrict__ fan, int64_t nmaps,
+                       int K, int N, int *status) {
     const int lane = threadIdx.x & 31;
     const int64_t m = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     if (m >= nmaps) return;
     const int64_t dk = m / K, kk = m - dk * K;
     const int32_t *src = pi + dk * pi_hs + kk * N;
-    int32_t *dst = dict + m * N;
-    int16_t *row = plan + (m * 32 + lane) * PW;
-    int cnt = 0;
+    uint8_t *t = tab + m * (kDcap * 64);
+    for (int i = lane; i < kDcap * 64; i += 32) t[i] = (uint8_t)kZeroSlot;
+    __syncwarp();
+    int cnt0 = 0, cnt1 = 0;   // sources of targets lane and lane + 32
     bool bad = false;
     for (int j = 0; j < N; ++j) {
         int tgt = __ldg(src + j);
@@ -142,26 +142,27 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
             bad = true;
             tgt = tgt < 0 ? 0 : N - 1;
         }
-        if (lane == 0) dst[j] = tgt;
-        if (tgt / npl == lane) {
-            row[1 + cnt] = (int16_t)(j | ((tgt - lane * npl) << 7));
-            ++cnt;
+        if (lane == 0) dict[m * N + j] = tgt;
+        if (tgt == lane) {
+            if (cnt0 < kDcap) t[cnt0 * 64 + lane] = (uint8_t)j;
+            ++cnt0;
+        } else if (tgt == lane + 32) {
+            if (cnt1 < kDcap) t[cnt1 * 64 + lane + 32] = (uint8_t)j;
+            ++cnt1;
         }
     }
     if (bad && lane == 0) flag_status(status, kStBadIndex);
-    const int G = __reduce_max_sync(kFull, cnt);
-    row[0] = (int16_t)G;
-    for (int g = 1 + cnt; g < PW; ++g) row[g] = (int16_t)-1;
+    const int D = __reduce_max_sync(kFull, max(cnt0, cnt1));
+    if (lane == 0) fan[m] = D;
 }
 
 cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
-                        int16_t *plan, int PW, int64_t Hd, int *status, cudaStream_t st) {
+                        uint8_t *tab, int32_t *fan, int64_t Hd, int *status, cudaStream_t st) {
     const int64_t nmaps = Hd * dm.K;
-    const int npl = dm.N > 32 ? 2 : 1;
     const int wpb = 4;
     const int64_t grid = (nmaps + wpb - 1) / wpb;
-    k_prep<<<(unsigned)grid, 32 * wpb, 0, st>>>(pi, pi_hs, dict, plan, PW, nmaps, (int)dm.K,
-                                                (int)dm.N, npl, status);
+    k_prep<<<(unsigned)grid, 32 * wpb, 0, st>>>(pi, pi_hs, dict, tab, fan, nmaps, (int)dm.K,
+                                                (int)dm.N, status);
     return cudaGetLastError();
 }
 

@@ -155,6 +155,23 @@ def test_forward_map_kinds(kind, N):
     check_fwd(small(7, 1, 2, 500, N, 3, kind=kind), chunk=64)
 
 
+@pytest.mark.parametrize("fan", [7, 8, 9, 20])
+@pytest.mark.parametrize("N", [24, 64])
+def test_forward_fan_in_around_slot_capacity(fan, N):
+    """One target of each map receives exactly `fan` sources; the slot table
+    holds up to 8 per target and larger fan-ins take the full scan."""
+    inp = small(60 + fan, 1, 2, 300, N, 4)
+    rng = np.random.default_rng(fan)
+    pi = inp.pi.copy()
+    for kk in range(pi.shape[0]):
+        row = rng.permutation(N).astype(np.int32)
+        row[rng.choice(N, size=fan, replace=False)] = rng.integers(0, N)
+        pi[kk] = row
+    inp.pi = pi
+    check_fwd(inp, chunk=50)
+    check_bwd(inp, chunk=50)
+
+
 @pytest.mark.parametrize("N", [8, 30, 64])
 def test_forward_bf16_aligned_and_unaligned_rows(N):
     check_fwd(small(9, 1, 2, 400, N, 4, dtype="bf16"), chunk=48)
