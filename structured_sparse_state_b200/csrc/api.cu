@@ -100,6 +100,16 @@ ChunkParams make_params(const pdssm_dims *dm, const WsLayout &w, void *ws, int64
 
 }  // namespace
 
+// The tensor-core selection path is the default where it applies;
+// PDSSM_SELECT_FMA=1 forces the plain fma-chain kernel (for comparisons).
+bool pdssm::select_tc_enabled() {
+    static const bool on = [] {
+        const char *e = getenv("PDSSM_SELECT_FMA");
+        return !(e && atoi(e) != 0);
+    }();
+    return on;
+}
+
 extern "C" {
 
 const char *pdssm_status_str(int status) {

@@ -17,23 +17,37 @@
 
 namespace pdssm {
 
-// bwd phase C warp: ring, exchange buffers (2 x kPbStride), lambda buffers
-// (2 x 64), checkpoints (16 x 64), barriers
+// bwd phase C warp: ring, exchange buffers (2 x kPbStride), readout buffer,
+// lambda buffers (2 x kPbStride), checkpoints (16 x 64), tile states (17 x 64)
+constexpr int kBwdExtraFloats = 2 * kPbStride + (kBwdMaxChunk / kTS) * kMaxN + (kTS + 1) * kMaxN;
 __host__ __device__ inline int bwd_warp_smem_bytes(int ns, int nt, int rowb) {
-    return warp_smem_bytes(ns, nt, rowb, 2 * kMaxN * 4 + (kBwdMaxChunk / kTS) * kMaxN * 4);
+    return warp_smem_bytes(ns, nt, rowb, kBwdExtraFloats * 4);
 }
 
-template <int NPL, bool EVEN>
-__device__ __forceinline__ void store_row(float *row, int lane, int N, const float (&v)[NPL]) {
-    if constexpr (NPL == 1) {
-        if (lane < N) row[lane] = v[0];
+template <int NPL, bool FULL>
+__device__ __forceinline__ void st_own(float *row, int lane, int N, const float (&v)[NPL]) {
+    if constexpr (FULL && NPL == 2) {
+        *reinterpret_cast<float2 *>(row + 2 * lane) = make_float2(v[0], v[1]);
     } else {
-        const int e0 = 2 * lane;
-        if constexpr (EVEN) {
-            if (e0 < N) *reinterpret_cast<float2 *>(row + e0) = make_float2(v[0], v[1]);
-        } else {
-            if (e0 < N) row[e0] = v[0];
-            if (e0 + 1 < N) row[e0 + 1] = v[1];
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) {
+            const int e = lane * NPL + r;
+            if (FULL || e < N) row[e] = v[r];
+        }
+    }
+}
+
+template <int NPL, bool FULL>
+__device__ __forceinline__ void own_targets2(const int *pk, int lane, int N, int (&tgt)[NPL]) {
+    if constexpr (FULL && NPL == 2) {
+        const int2 q = *reinterpret_cast<const int2 *>(pk + 2 * lane);
+        tgt[0] = q.x;
+        tgt[1] = q.y;
+    } else {
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) {
+            const int e = lane * NPL + r;
+            tgt[r] = (FULL || e < N) ? pk[e] : 0;
         }
     }
 }
@@ -41,7 +55,7 @@ __device__ __forceinline__ void store_row(float *row, int lane, int N, const flo
 // ---------------------------------------------------------------------------
 // bwd phase A: w_c = M_s^T lambda^loc_s with lambda^loc from a zero carry
 // ---------------------------------------------------------------------------
-template <typename T, int NPL, bool EVEN>
+template <typename T, int NPL, bool FULL>
 __global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_ba[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -64,7 +78,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
     ring.ns = p.ns;
     ring.bulk = p.bulk != 0;
     float *lbuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes);
-    ring.bar0 = smem_u32(lbuf + 2 * kPbStride);
+    ring.bar0 = smem_u32(lbuf + 2 * kPbStride + kYbufFloats);
     const int64_t seq_row0 = bh * p.L;
     ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * rowb;
     ring.src[1] = reinterpret_cast<const unsigned char *>(p.c) + seq_row0 * rowb;
@@ -80,13 +94,14 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
         const int ti = tile_of(j);
         ring.prefetch(s + (int64_t)ti * kTS, min(kTS, len - ti * kTS), 2, lane);
     }
-    const int64_t kbase = bh * p.L + s;
+    const int32_t *kp = p.k + bh * p.L + s;
+    const float *gyp = p.g_y + bh * p.L + s;
     float mu[NPL];
 #pragma unroll
     for (int r = 0; r < NPL; ++r) mu[r] = 0.f;
     int t0 = (ntiles - 1) * kTS;
-    int kreg = load_k(p.k, kbase + t0 + lane, lane < kTS && t0 + lane < len, K, p.status);
-    float gyreg = (lane < kTS && t0 + lane < len) ? p.g_y[kbase + t0 + lane] : 0.f;
+    int kreg = load_k(kp, t0 + lane, lane < kTS && t0 + lane < len, K, p.status);
+    float gyreg = (lane < kTS && t0 + lane < len) ? gyp[t0 + lane] : 0.f;
 
     for (int j = 0; j < ntiles; ++j) {
         const int stage = j % p.ns;
@@ -94,38 +109,30 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
             ring_abort(ring, j, min(ntiles, j + p.ns), p.status, lane);
             return;
         }
-        const int ti = tile_of(j);
-        t0 = ti * kTS;
+        t0 = tile_of(j) * kTS;
         const int n = min(kTS, len - t0);
-        const int tp = t0 - kTS;   // previous tile (processed next)
+        const int tp = t0 - kTS;   // the tile processed next
         const bool vp = lane < kTS && tp >= 0;
-        const int knext = load_k(p.k, kbase + tp + lane, vp, K, p.status);
-        const float gynext = vp ? p.g_y[kbase + tp + lane] : 0.f;
+        const int knext = load_k(kp, tp + lane, vp, K, p.status);
+        const float gynext = vp ? gyp[tp + lane] : 0.f;
         const T *td = reinterpret_cast<const T *>(ring.tile(stage, 0));
         const T *tc = reinterpret_cast<const T *>(ring.tile(stage, 1));
+#pragma unroll 2
+        for (int q = n - 1; q >= 0; --q) {
+            const int kk = __shfl_sync(kFull, kreg, q);
+            const float gy = __shfl_sync(kFull, gyreg, q);
+            float dv[NPL], cv[NPL], lam[NPL];
+            ld_own<T, NPL, FULL>(td + q * N, lane, N, dv);
+            ld_own<T, NPL, FULL>(tc + q * N, lane, N, cv);
 #pragma unroll
-        for (int q = kTS - 1; q >= 0; --q) {
-            if (q < n) {
-                const int kk = __shfl_sync(kFull, kreg, q);
-                const float gy = __shfl_sync(kFull, gyreg, q);
-                float dv[NPL], cv[NPL];
-                load_row<T, NPL, EVEN>(td + q * N, lane, N, dv);
-                load_row<T, NPL, EVEN>(tc + q * N, lane, N, cv);
-                float *lb = lbuf + (q & 1) * kPbStride;
+            for (int r = 0; r < NPL; ++r) lam[r] = gy * cv[r] + mu[r];
+            float *lb = lbuf + (q & 1) * kPbStride;
+            st_own<NPL, FULL>(lb, lane, N, lam);
+            __syncwarp();
+            int tgt[NPL];
+            own_targets2<NPL, FULL>(sd.map + kk * N, lane, N, tgt);
 #pragma unroll
-                for (int r = 0; r < NPL; ++r) {
-                    const int e = lane * NPL + r;
-                    if (e < N) lb[e] = gy * cv[r] + mu[r];
-                }
-                __syncwarp();
-                int tgt[NPL];
-                own_targets<NPL, EVEN>(sd.map + kk * N, lane, N, tgt);
-#pragma unroll
-                for (int r = 0; r < NPL; ++r) {
-                    const int e = lane * NPL + r;
-                    if (e < N) mu[r] = dv[r] * lb[tgt[r]];
-                }
-            }
+            for (int r = 0; r < NPL; ++r) mu[r] = dv[r] * lb[tgt[r]];
         }
         __syncwarp();
         if (j + p.ns < ntiles) {
@@ -303,10 +310,10 @@ __global__ void k_bwdB(const ChunkParams p) {
 // ---------------------------------------------------------------------------
 // bwd phase C: per chunk, (1) forward recompute from H_{c-1} keeping the
 // state at every tile start in shared memory, (2) per tile in reverse:
-// recompute the tile's states into registers, then sweep back emitting
+// recompute the tile's states into shared memory, then sweep back emitting
 // g_b = lambda, g_c = g_y h, g_d = h_{t-1} * lambda[pi(.)].
 // ---------------------------------------------------------------------------
-template <typename T, int NPL, bool EVEN>
+template <typename T, int NPL, bool FULL>
 __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_bc[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -329,9 +336,10 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
     ring.ns = p.ns;
     ring.bulk = p.bulk != 0;
     float *pbuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes);
-    float *lbuf = pbuf + 2 * kPbStride;
-    float *ck = lbuf + 2 * kMaxN;   // [kBwdMaxChunk / kTS][64]
-    ring.bar0 = smem_u32(ck + (kBwdMaxChunk / kTS) * kMaxN);
+    float *lbuf = pbuf + 2 * kPbStride + kYbufFloats;
+    float *ck = lbuf + 2 * kPbStride;                 // [kBwdMaxChunk / kTS][64]
+    float *hsm = ck + (kBwdMaxChunk / kTS) * kMaxN;   // [kTS + 1][64]
+    ring.bar0 = smem_u32(hsm + (kTS + 1) * kMaxN);
     const int64_t seq_row0 = bh * p.L;
     ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * rowb;
     ring.src[1] = reinterpret_cast<const unsigned char *>(p.b) + seq_row0 * rowb;
@@ -348,9 +356,10 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
     }
     for (int m = p.ns; m < p.ns + kPrefetchTiles && m < ntiles; ++m)
         ring.prefetch(s + (int64_t)m * kTS, min(kTS, len - m * kTS), 3, lane);
-
     clear_pb(pbuf, lane);
-    const int64_t kbase = bh * p.L + s;
+
+    const int32_t *kp = p.k + bh * p.L + s;
+    const float *gyp = p.g_y + bh * p.L + s;
     float h[NPL], mu[NPL];
 #pragma unroll
     for (int r = 0; r < NPL; ++r) {
@@ -362,7 +371,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
             mu[r] = p.lam[unit * p.N + e];
         }
     }
-    int kreg = load_k(p.k, kbase + lane, lane < kTS && lane < len, K, p.status);
+    int kreg = load_k(kp, lane, lane < kTS && lane < len, K, p.status);
     float gyreg = 0.f;
 
     for (int m = 0; m < total; ++m) {
@@ -374,91 +383,75 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
         const int ti = tile_of(m);
         const int t0 = ti * kTS;
         const int n = min(kTS, len - t0);
-        // next tile in processing order (for the k / g_y prefetch)
         int knext = 0;
         float gynext = 0.f;
         if (m + 1 < total) {
             const int tn0 = tile_of(m + 1) * kTS;
             const bool v = lane < kTS && tn0 + lane < len;
-            knext = load_k(p.k, kbase + tn0 + lane, v, K, p.status);
-            if (m + 1 >= ntiles) gynext = v ? p.g_y[kbase + tn0 + lane] : 0.f;
+            knext = load_k(kp, tn0 + lane, v, K, p.status);
+            if (m + 1 >= ntiles) gynext = v ? gyp[tn0 + lane] : 0.f;
         }
         const T *td = reinterpret_cast<const T *>(ring.tile(stage, 0));
         const T *tb = reinterpret_cast<const T *>(ring.tile(stage, 1));
         const T *tc = reinterpret_cast<const T *>(ring.tile(stage, 2));
         if (m < ntiles) {
             // pass 1: checkpoint at the tile start, then advance the state
-#pragma unroll
-            for (int r = 0; r < NPL; ++r) {
-                const int e = lane * NPL + r;
-                if (e < N) ck[ti * kMaxN + e] = h[r];
-            }
-#pragma unroll
-            for (int q = 0; q < kTS; ++q) {
-                if (q < n) {
-                    const int kk = __shfl_sync(kFull, kreg, q);
-                    float dv[NPL], bv[NPL];
-                    load_row<T, NPL, EVEN>(td + q * N, lane, N, dv);
-                    load_row<T, NPL, EVEN>(tb + q * N, lane, N, bv);
-                    pd_gather_step<NPL>(h, dv, bv, pbuf + (q & 1) * kPbStride,
-                                        sd.tab + kk * (kDcap * 64), sd.fan[kk],
-                                        sd.map + kk * N, lane, N);
-                }
+            st_own<NPL, FULL>(ck + ti * kMaxN, lane, N, h);
+#pragma unroll 2
+            for (int q = 0; q < n; ++q) {
+                const int kk = __shfl_sync(kFull, kreg, q);
+                float dv[NPL], bv[NPL];
+                ld_own<T, NPL, FULL>(td + q * N, lane, N, dv);
+                ld_own<T, NPL, FULL>(tb + q * N, lane, N, bv);
+                pd_gather_step<NPL, FULL>(h, dv, bv, pbuf + (q & 1) * kPbStride,
+                                          sd.tab + kk * (kDcap * 64) + lane * NPL, sd.fan[kk],
+                                          sd.map + kk * N, lane, N);
             }
         } else {
-            // pass 2: states of this tile, hs[q] = h_{t0+q-1}
-            float hs[kTS + 1][NPL];
-#pragma unroll
-            for (int r = 0; r < NPL; ++r) {
-                const int e = lane * NPL + r;
-                hs[0][r] = e < N ? ck[ti * kMaxN + e] : 0.f;
+            // pass 2: states of this tile, hsm[q] = h_{t0+q-1}
+            float x[NPL];
+            ld_own<float, NPL, FULL>(ck + ti * kMaxN, lane, N, x);
+            st_own<NPL, FULL>(hsm, lane, N, x);
+#pragma unroll 2
+            for (int q = 0; q < n; ++q) {
+                const int kk = __shfl_sync(kFull, kreg, q);
+                float dv[NPL], bv[NPL];
+                ld_own<T, NPL, FULL>(td + q * N, lane, N, dv);
+                ld_own<T, NPL, FULL>(tb + q * N, lane, N, bv);
+                pd_gather_step<NPL, FULL>(x, dv, bv, pbuf + (q & 1) * kPbStride,
+                                          sd.tab + kk * (kDcap * 64) + lane * NPL, sd.fan[kk],
+                                          sd.map + kk * N, lane, N);
+                st_own<NPL, FULL>(hsm + (q + 1) * kMaxN, lane, N, x);
             }
+#pragma unroll 2
+            for (int q = n - 1; q >= 0; --q) {
+                const int kk = __shfl_sync(kFull, kreg, q);
+                const float gy = __shfl_sync(kFull, gyreg, q);
+                const int64_t row = (int64_t)(t0 + q) * p.N;
+                float dv[NPL], cv[NPL], hq[NPL], hp[NPL], lam[NPL], gc[NPL], gd[NPL];
+                ld_own<T, NPL, FULL>(td + q * N, lane, N, dv);
+                ld_own<T, NPL, FULL>(tc + q * N, lane, N, cv);
+                ld_own<float, NPL, FULL>(hsm + (q + 1) * kMaxN, lane, N, hq);
+                ld_own<float, NPL, FULL>(hsm + q * kMaxN, lane, N, hp);
 #pragma unroll
-            for (int q = 0; q < kTS; ++q) {
-#pragma unroll
-                for (int r = 0; r < NPL; ++r) hs[q + 1][r] = hs[q][r];
-                if (q < n) {
-                    const int kk = __shfl_sync(kFull, kreg, q);
-                    float dv[NPL], bv[NPL];
-                    load_row<T, NPL, EVEN>(td + q * N, lane, N, dv);
-                    load_row<T, NPL, EVEN>(tb + q * N, lane, N, bv);
-                    pd_gather_step<NPL>(hs[q + 1], dv, bv, pbuf + (q & 1) * kPbStride,
-                                        sd.tab + kk * (kDcap * 64), sd.fan[kk],
-                                        sd.map + kk * N, lane, N);
+                for (int r = 0; r < NPL; ++r) {
+                    lam[r] = gy * cv[r] + mu[r];
+                    gc[r] = gy * hq[r];
                 }
-            }
+                float *lb = lbuf + (q & 1) * kPbStride;
+                st_own<NPL, FULL>(lb, lane, N, lam);
+                st_own<NPL, FULL>(p.g_b + seq_row0 * p.N + s * p.N + row, lane, N, lam);
+                st_own<NPL, FULL>(p.g_c + seq_row0 * p.N + s * p.N + row, lane, N, gc);
+                __syncwarp();
+                int tgt[NPL];
+                own_targets2<NPL, FULL>(sd.map + kk * N, lane, N, tgt);
 #pragma unroll
-            for (int q = kTS - 1; q >= 0; --q) {
-                if (q < n) {
-                    const int kk = __shfl_sync(kFull, kreg, q);
-                    const float gy = __shfl_sync(kFull, gyreg, q);
-                    const int64_t row = (kbase + t0 + q) * p.N;
-                    float dv[NPL], cv[NPL], lam[NPL], gc[NPL];
-                    load_row<T, NPL, EVEN>(td + q * N, lane, N, dv);
-                    load_row<T, NPL, EVEN>(tc + q * N, lane, N, cv);
-                    float *lb = lbuf + (q & 1) * kMaxN;
-#pragma unroll
-                    for (int r = 0; r < NPL; ++r) {
-                        const int e = lane * NPL + r;
-                        lam[r] = gy * cv[r] + mu[r];
-                        gc[r] = gy * hs[q + 1][r];
-                        if (e < N) lb[e] = lam[r];
-                    }
-                    store_row<NPL, EVEN>(p.g_b + row, lane, N, lam);
-                    store_row<NPL, EVEN>(p.g_c + row, lane, N, gc);
-                    __syncwarp();
-                    int tgt[NPL];
-                    own_targets<NPL, EVEN>(sd.map + kk * N, lane, N, tgt);
-                    float gd[NPL];
-#pragma unroll
-                    for (int r = 0; r < NPL; ++r) {
-                        const int e = lane * NPL + r;
-                        const float gl = e < N ? lb[tgt[r]] : 0.f;
-                        gd[r] = hs[q][r] * gl;
-                        mu[r] = dv[r] * gl;
-                    }
-                    store_row<NPL, EVEN>(p.g_d + row, lane, N, gd);
+                for (int r = 0; r < NPL; ++r) {
+                    const float gl = lb[tgt[r]];
+                    gd[r] = hp[r] * gl;
+                    mu[r] = dv[r] * gl;
                 }
+                st_own<NPL, FULL>(p.g_d + seq_row0 * p.N + s * p.N + row, lane, N, gd);
             }
         }
         __syncwarp();
@@ -492,12 +485,10 @@ static cudaError_t launch_chunk_b(KernT kern, const ChunkParams &p, size_t smem,
 
 #define PDSSM_DISPATCH_B(KERNEL, p, st, smem)                                     \
     do {                                                                         \
-        const bool even = ((p).N % 2) == 0;                                      \
-        if ((p).N > 32) {                                                        \
-            return even ? launch_chunk_b(KERNEL<T, 2, true>, p, smem, st)        \
-                        : launch_chunk_b(KERNEL<T, 2, false>, p, smem, st);      \
-        }                                                                        \
-        return launch_chunk_b(KERNEL<T, 1, true>, p, smem, st);                  \
+        if ((p).N == 64) return launch_chunk_b(KERNEL<T, 2, true>, p, smem, st); \
+        if ((p).N > 32) return launch_chunk_b(KERNEL<T, 2, false>, p, smem, st); \
+        if ((p).N == 32) return launch_chunk_b(KERNEL<T, 1, true>, p, smem, st); \
+        return launch_chunk_b(KERNEL<T, 1, false>, p, smem, st);                 \
     } while (0)
 
 template <typename T>

@@ -272,46 +272,72 @@ __device__ __forceinline__ void own_targets(const int *pk, int lane, int N, int 
     }
 }
 
+// Loads the NPL elements a lane owns from one staged row.  FULL means the
+// state fills the warp (N == 32 * NPL): no guards, vector loads.
+template <typename T, int NPL, bool FULL>
+__device__ __forceinline__ void ld_own(const T *row, int lane, int N, float (&v)[NPL]) {
+    if constexpr (FULL) {
+        if constexpr (NPL == 1) {
+            v[0] = to_f<T>(row[lane]);
+        } else if constexpr (std::is_same<T, float>::value) {
+            const float2 q = *reinterpret_cast<const float2 *>(row + 2 * lane);
+            v[0] = q.x;
+            v[1] = q.y;
+        } else {
+            const __nv_bfloat162 q = *reinterpret_cast<const __nv_bfloat162 *>(row + 2 * lane);
+            v[0] = __low2float(q);
+            v[1] = __high2float(q);
+        }
+    } else {
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) {
+            const int e = lane * NPL + r;
+            v[r] = e < N ? to_f<T>(row[e]) : 0.f;
+        }
+    }
+}
+
 // One PD step h <- P_k diag(d) h + b on the lane-owned state, as a gather:
 // every lane stores d[j] h[j] of the sources it owns into `pb` (this step's
 // buffer of an alternating pair, entry kZeroSlot permanently 0), then sums,
 // for each element it owns, the sources listed by the map's slot table in
 // ascending j (padding entries point at the zero slot).  One warp barrier per
-// step; no atomics, so the result is deterministic.  Maps whose fan-in
-// exceeds kDcap scan all N sources instead.
-template <int NPL>
+// step; no atomics, so the result is deterministic.  `tabl` is the map's
+// table advanced to this lane's first element; Dk the map's largest fan-in
+// (maps above kDcap scan all N sources instead).
+template <int NPL, bool FULL>
 __device__ __forceinline__ void pd_gather_step(float (&h)[NPL], const float (&dv)[NPL],
                                                const float (&bv)[NPL], float *pb,
-                                               const uint8_t *tabk, int Dk, const int *pk,
+                                               const uint8_t *tabl, int Dk, const int *pk,
                                                int lane, int N) {
     if constexpr (NPL == 2) {
-        if (2 * lane + 1 < N) {
+        if (FULL || 2 * lane + 1 < N) {
             *reinterpret_cast<float2 *>(pb + 2 * lane) = make_float2(dv[0] * h[0], dv[1] * h[1]);
         } else if (2 * lane < N) {
             pb[2 * lane] = dv[0] * h[0];
         }
     } else {
-        if (lane < N) pb[lane] = dv[0] * h[0];
+        if (FULL || lane < N) pb[lane] = dv[0] * h[0];
     }
     __syncwarp();
     float acc[NPL];
-#pragma unroll
-    for (int r = 0; r < NPL; ++r) acc[r] = 0.f;
     if (Dk <= kDcap) {
         if constexpr (NPL == 2) {
-            const uint16_t *t16 = reinterpret_cast<const uint16_t *>(tabk) + lane;
-#pragma unroll 4
-            for (int sl = 0; sl < Dk; ++sl) {
-                const unsigned w = t16[sl * 32];
+            unsigned w = *reinterpret_cast<const uint16_t *>(tabl);
+            acc[0] = pb[w & 0xffu];
+            acc[1] = pb[w >> 8];
+            for (int sl = 1; sl < Dk; ++sl) {
+                w = *reinterpret_cast<const uint16_t *>(tabl + sl * 64);
                 acc[0] += pb[w & 0xffu];
                 acc[1] += pb[w >> 8];
             }
         } else {
-            const uint8_t *t8 = tabk + lane;
-#pragma unroll 4
-            for (int sl = 0; sl < Dk; ++sl) acc[0] += pb[t8[sl * 64]];
+            acc[0] = pb[tabl[0]];
+            for (int sl = 1; sl < Dk; ++sl) acc[0] += pb[tabl[sl * 64]];
         }
     } else {
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) acc[r] = 0.f;
         for (int j = 0; j < N; ++j) {
             const int t = pk[j];
             const float v = pb[j];
@@ -321,7 +347,19 @@ __device__ __forceinline__ void pd_gather_step(float (&h)[NPL], const float (&dv
         }
     }
 #pragma unroll
-    for (int r = 0; r < NPL; ++r) h[r] = (lane * NPL + r < N) ? acc[r] + bv[r] : 0.f;
+    for (int r = 0; r < NPL; ++r) h[r] = (FULL || lane * NPL + r < N) ? acc[r] + bv[r] : 0.f;
+}
+
+// Sum over the warp of per-step partials staged in ybuf[q][33] (rows
+// q < n): lane q < n returns the total of row q.  Caller synchronises.
+__device__ __forceinline__ float ybuf_row_sum(const float *ybuf, int lane, int n) {
+    float s = 0.f;
+    if (lane < n) {
+        const float *row = ybuf + lane * 33;
+#pragma unroll 8
+        for (int j = 0; j < 32; ++j) s += row[j];
+    }
+    return s;
 }
 
 // Both exchange buffers of a warp: zero, including the zero slots.
@@ -419,12 +457,15 @@ __device__ void ring_abort(const Ring<NT> &ring, int first, int last, int *statu
 // Dynamic shared memory of the chunk kernels:
 //   [dictionary slots][warp 0][warp 1]...
 //   dictionary slot = [map K x N ints][slot tables K x kDcap x 64 bytes][fan-in K ints]
-//   warp = [staging ring][exchange buffers 2 x kPbStride floats][extra][barriers]
+//   warp = [staging ring][exchange buffers 2 x kPbStride floats]
+//          [readout buffer kTS x 33 floats][extra][barriers]
+constexpr int kYbufFloats = kTS * 33;
 __host__ __device__ inline int dict_slot_bytes(int K, int N) {
     return (K * N * 4 + K * kDcap * 64 + K * 4 + 127) / 128 * 128;
 }
 __host__ __device__ inline int warp_smem_bytes(int ns, int nt, int rowb, int extra = 0) {
-    return (ns * nt * kTS * rowb + 2 * kPbStride * 4 + extra + kMaxStages * 8 + 127) / 128 * 128;
+    return (ns * nt * kTS * rowb + 2 * kPbStride * 4 + kYbufFloats * 4 + extra + kMaxStages * 8 +
+            127) / 128 * 128;
 }
 
 struct SmemDict {
@@ -478,6 +519,10 @@ __host__ __device__ inline int dict_region_bytes(const ChunkParams &p) {
 // ---------------------------------------------------------------------------
 cudaError_t launch_select(const pdssm_dims &dm, const void *u, pdssm_dtype ut, const float *W,
                           int32_t *k_out, cudaStream_t st);
+bool select_tc_supported(const pdssm_dims &dm, pdssm_dtype ut, const void *u);
+bool select_tc_enabled();
+cudaError_t launch_select_tc(const pdssm_dims &dm, const void *u, const float *W, int32_t *k_out,
+                             cudaStream_t st);
 cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
                         uint8_t *tab, int32_t *fan, int64_t Hd, int *status, cudaStream_t st);
 cudaError_t launch_validate(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs,

@@ -23,7 +23,7 @@ namespace pdssm {
 // ---------------------------------------------------------------------------
 // phase A
 // ---------------------------------------------------------------------------
-template <typename T, int NPL, bool EVEN>
+template <typename T, int NPL, bool FULL>
 __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_a[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -48,7 +48,8 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
     ring.ns = p.ns;
     ring.bulk = p.bulk != 0;
     float *pbuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes);
-    ring.bar0 = smem_u32(pbuf + 2 * kPbStride);
+    float *ybuf = pbuf + 2 * kPbStride;
+    ring.bar0 = smem_u32(ybuf + kYbufFloats);
     const int64_t seq_row0 = bh * p.L;
     ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * rowb;
     ring.src[1] = reinterpret_cast<const unsigned char *>(p.b) + seq_row0 * rowb;
@@ -61,7 +62,6 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
         ring.issue(i, s + (int64_t)i * kTS, min(kTS, len - i * kTS), nt, lane);
     for (int i = p.ns; i < p.ns + kPrefetchTiles && i < ntiles; ++i)
         ring.prefetch(s + (int64_t)i * kTS, min(kTS, len - i * kTS), nt, lane);
-
     clear_pb(pbuf, lane);
 
     float h[NPL], Dl[NPL];
@@ -72,8 +72,8 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
         Dl[r] = 1.f;
         pos[r] = min(lane * NPL + r, N - 1);
     }
-    const int64_t kbase = bh * p.L + s;
-    int kreg = load_k(p.k, kbase + lane, lane < kTS && lane < len, K, p.status);
+    const int32_t *kp = p.k + bh * p.L + s;
+    int kreg = load_k(kp, lane, lane < kTS && lane < len, K, p.status);
 
     for (int i = 0; i < ntiles; ++i) {
         const int stage = i % p.ns;
@@ -83,46 +83,43 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
-        const int knext = load_k(p.k, kbase + t0 + kTS + lane,
-                                 lane < kTS && t0 + kTS + lane < len, K, p.status);
-        const T *td = reinterpret_cast<const T *>(ring.tile(stage, 0));
-        const T *tb = reinterpret_cast<const T *>(ring.tile(stage, 1));
-        const T *tc = reinterpret_cast<const T *>(ring.tile(stage, 2));
-        float yp[kTS];
+        const int knext = load_k(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len, K,
+                                 p.status);
+        const T *rd = reinterpret_cast<const T *>(ring.tile(stage, 0));
+        const T *rb = reinterpret_cast<const T *>(ring.tile(stage, 1));
+        const T *rc = reinterpret_cast<const T *>(ring.tile(stage, 2));
+#pragma unroll 2
+        for (int q = 0; q < n; ++q, rd += N, rb += N, rc += N) {
+            const int kk = __shfl_sync(kFull, kreg, q);
+            const int *pk = sd.map + kk * N;
+            float dv[NPL], bv[NPL];
+            ld_own<T, NPL, FULL>(rd, lane, N, dv);
+            ld_own<T, NPL, FULL>(rb, lane, N, bv);
+            // transfer tracking: Delta picks up d at the column's current
+            // position, then the selected map moves the column
 #pragma unroll
-        for (int q = 0; q < kTS; ++q) {
-            yp[q] = 0.f;
-            if (q < n) {
-                const int kk = __shfl_sync(kFull, kreg, q);
-                const int *pk = sd.map + kk * N;
-                const T *rd = td + q * N;
-                float dv[NPL], bv[NPL];
-                load_row<T, NPL, EVEN>(rd, lane, N, dv);
-                load_row<T, NPL, EVEN>(tb + q * N, lane, N, bv);
-                // transfer tracking: Delta picks up d at the column's current
-                // position, then the selected map moves the column
-#pragma unroll
-                for (int r = 0; r < NPL; ++r) {
-                    if (lane * NPL + r < N) {
-                        Dl[r] *= to_f<T>(rd[pos[r]]);
-                        pos[r] = pk[pos[r]];
-                    }
-                }
-                pd_gather_step<NPL>(h, dv, bv, pbuf + (q & 1) * kPbStride,
-                                    sd.tab + kk * (kDcap * 64), sd.fan[kk], pk, lane, N);
-                if (with_y) {
-                    float cv[NPL];
-                    load_row<T, NPL, EVEN>(tc + q * N, lane, N, cv);
-                    float acc = 0.f;
-#pragma unroll
-                    for (int r = 0; r < NPL; ++r) acc += cv[r] * h[r];
-                    yp[q] = acc;
+            for (int r = 0; r < NPL; ++r) {
+                if (FULL || lane * NPL + r < N) {
+                    Dl[r] *= to_f<T>(rd[pos[r]]);
+                    pos[r] = pk[pos[r]];
                 }
             }
+            pd_gather_step<NPL, FULL>(h, dv, bv, pbuf + (q & 1) * kPbStride,
+                                      sd.tab + kk * (kDcap * 64) + lane * NPL, sd.fan[kk], pk,
+                                      lane, N);
+            if (with_y) {
+                float cv[NPL];
+                ld_own<T, NPL, FULL>(rc, lane, N, cv);
+                float acc = cv[0] * h[0];
+#pragma unroll
+                for (int r = 1; r < NPL; ++r) acc = fmaf(cv[r], h[r], acc);
+                ybuf[q * 33 + lane] = acc;
+            }
         }
+        __syncwarp();
         if (with_y) {
-            const float ys = reduce_scatter16(yp);
-            if (lane < n) p.y[kbase + t0 + lane] = ys;
+            const float ys = ybuf_row_sum(ybuf, lane, n);
+            if (lane < n) p.y[bh * p.L + s + t0 + lane] = ys;
         }
         __syncwarp();
         if (i + p.ns < ntiles)
@@ -149,7 +146,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
 // ---------------------------------------------------------------------------
 // phase C (carry correction in path form)
 // ---------------------------------------------------------------------------
-template <typename T, int NPL, bool EVEN>
+template <typename T, int NPL, bool FULL>
 __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_c[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -172,7 +169,8 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
     ring.stage_bytes = 2 * ring.tens_bytes;
     ring.ns = p.ns;
     ring.bulk = p.bulk != 0;
-    ring.bar0 = smem_u32(wbase + p.ns * ring.stage_bytes + 2 * kPbStride * 4);
+    float *ybuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes) + 2 * kPbStride;
+    ring.bar0 = smem_u32(ybuf + kYbufFloats);
     const int64_t seq_row0 = bh * p.L;
     ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * rowb;
     ring.src[1] = reinterpret_cast<const unsigned char *>(p.c) + seq_row0 * rowb;
@@ -193,8 +191,9 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
         w[r] = 0.f;
         if (e < N) w[r] = cidx == 0 ? p.h0[bh * p.N + e] : p.Hc[(unit - 1) * p.N + e];
     }
-    const int64_t kbase = bh * p.L + s;
-    int kreg = load_k(p.k, kbase + lane, lane < kTS && lane < len, K, p.status);
+    const int32_t *kp = p.k + bh * p.L + s;
+    float *yp = p.y + bh * p.L + s;
+    int kreg = load_k(kp, lane, lane < kTS && lane < len, K, p.status);
 
     for (int i = 0; i < ntiles; ++i) {
         const int stage = i % p.ns;
@@ -204,34 +203,29 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
-        const int knext = load_k(p.k, kbase + t0 + kTS + lane,
-                                 lane < kTS && t0 + kTS + lane < len, K, p.status);
-        const float yold = lane < n ? p.y[kbase + t0 + lane] : 0.f;
-        const T *td = reinterpret_cast<const T *>(ring.tile(stage, 0));
-        const T *tc = reinterpret_cast<const T *>(ring.tile(stage, 1));
-        float yp[kTS];
+        const int knext = load_k(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len, K,
+                                 p.status);
+        const float yold = lane < n ? yp[t0 + lane] : 0.f;
+        const T *rd = reinterpret_cast<const T *>(ring.tile(stage, 0));
+        const T *rc = reinterpret_cast<const T *>(ring.tile(stage, 1));
+#pragma unroll 2
+        for (int q = 0; q < n; ++q, rd += N, rc += N) {
+            const int kk = __shfl_sync(kFull, kreg, q);
+            const int *pk = sd.map + kk * N;
+            float acc = 0.f;
 #pragma unroll
-        for (int q = 0; q < kTS; ++q) {
-            yp[q] = 0.f;
-            if (q < n) {
-                const int kk = __shfl_sync(kFull, kreg, q);
-                const int *pk = sd.map + kk * N;
-                const T *rd = td + q * N;
-                const T *rc = tc + q * N;
-                float acc = 0.f;
-#pragma unroll
-                for (int r = 0; r < NPL; ++r) {
-                    if (lane * NPL + r < N) {
-                        w[r] *= to_f<T>(rd[pos[r]]);
-                        pos[r] = pk[pos[r]];
-                        acc += to_f<T>(rc[pos[r]]) * w[r];
-                    }
+            for (int r = 0; r < NPL; ++r) {
+                if (FULL || lane * NPL + r < N) {
+                    w[r] *= to_f<T>(rd[pos[r]]);
+                    pos[r] = pk[pos[r]];
+                    acc = fmaf(to_f<T>(rc[pos[r]]), w[r], acc);
                 }
-                yp[q] = acc;
             }
+            ybuf[q * 33 + lane] = acc;
         }
-        const float ys = reduce_scatter16(yp);
-        if (lane < n) p.y[kbase + t0 + lane] = yold + ys;
+        __syncwarp();
+        const float ys = ybuf_row_sum(ybuf, lane, n);
+        if (lane < n) yp[t0 + lane] = yold + ys;
         __syncwarp();
         if (i + p.ns < ntiles)
             ring.issue(stage, s + (int64_t)(i + p.ns) * kTS, min(kTS, len - (i + p.ns) * kTS), 2,
@@ -461,14 +455,13 @@ static cudaError_t launch_chunk(KernT kern, const ChunkParams &p, size_t smem, c
     return cudaGetLastError();
 }
 
+// Template choice: NPL = elements per lane, FULL = the state fills the warp.
 #define PDSSM_DISPATCH(KERNEL, p, st, smem)                                       \
     do {                                                                         \
-        const bool even = ((p).N % 2) == 0;                                      \
-        if ((p).N > 32) {                                                        \
-            return even ? launch_chunk(KERNEL<T, 2, true>, p, smem, st)          \
-                        : launch_chunk(KERNEL<T, 2, false>, p, smem, st);        \
-        }                                                                        \
-        return launch_chunk(KERNEL<T, 1, true>, p, smem, st);                    \
+        if ((p).N == 64) return launch_chunk(KERNEL<T, 2, true>, p, smem, st);   \
+        if ((p).N > 32) return launch_chunk(KERNEL<T, 2, false>, p, smem, st);   \
+        if ((p).N == 32) return launch_chunk(KERNEL<T, 1, true>, p, smem, st);   \
+        return launch_chunk(KERNEL<T, 1, false>, p, smem, st);                   \
     } while (0)
 
 template <typename T>

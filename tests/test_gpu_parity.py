@@ -59,6 +59,64 @@ def test_select_bit_exact(idx, over):
     assert (k == oracle.select(inp.u, inp.W)).all()
 
 
+@pytest.mark.parametrize("H,K,D", [(16, 16, 128), (2, 8, 64), (1, 4, 16), (4, 32, 32),
+                                   (3, 2, 48)])
+def test_select_tensor_core_shapes_bit_exact(H, K, D):
+    """bf16 u with K a power of two takes the tcgen05 path (certified
+    argmax, exact fma-chain recompute near ties)."""
+    rng = np.random.default_rng(H * 1000 + K * 10 + D)
+    B, L = 2, 333
+    u = gen.round_bf16(rng.standard_normal((B, L, D)).astype(np.float32))
+    W = (rng.standard_normal((H, K, D)) / np.sqrt(D)).astype(np.float32)
+    k = pd.pdssm_select(dev(u, bf16=True), dev(W)).cpu().numpy()
+    assert (k == oracle.select(u, W)).all()
+
+
+def test_select_near_ties_take_the_exact_path():
+    """Rows of W that differ by ~1e-6 make most top-2 gaps smaller than the
+    certification bound, so the exact fma chains decide."""
+    rng = np.random.default_rng(77)
+    H, K, D, B, L = 4, 16, 128, 1, 512
+    base = (rng.standard_normal((H, 1, D)) / np.sqrt(D)).astype(np.float32)
+    W = (base + 1e-6 * rng.standard_normal((H, K, D))).astype(np.float32)
+    W[:, 5] = W[:, 3]                        # exact duplicates: first index wins
+    u = gen.round_bf16(rng.standard_normal((B, L, D)).astype(np.float32))
+    k = pd.pdssm_select(dev(u, bf16=True), dev(W)).cpu().numpy()
+    kr = oracle.select(u, W)
+    assert (k == kr).all()
+    assert not (kr == 5).any() or (kr == 3).any()
+
+
+def test_select_full_size_tensor_core_equals_fma_kernel(tmp_path):
+    """The full bf16 selection workload: the tensor-core kernel and the plain
+    fma-chain kernel (forced in a child process) agree on every index, and a
+    sample of rows matches the oracle."""
+    import subprocess
+    import sys
+    inp = gen.generate(gen.workload(2))
+    u = dev(inp.u, bf16=True)
+    W = dev(inp.W)
+    k_tc = pd.pdssm_select(u, W).cpu().numpy()
+    np.save(tmp_path / "u.npy", inp.u)
+    np.save(tmp_path / "W.npy", inp.W)
+    code = (
+        "import sys, numpy as np, torch; sys.path.insert(0, %r);"
+        "import structured_sparse_state_b200 as pd;"
+        "u = torch.from_numpy(np.load(%r)).to(torch.bfloat16).cuda();"
+        "W = torch.from_numpy(np.load(%r)).cuda();"
+        "np.save(%r, pd.pdssm_select(u, W).cpu().numpy())"
+    ) % (str(__import__('pathlib').Path(__file__).resolve().parents[1]), str(tmp_path / "u.npy"),
+         str(tmp_path / "W.npy"), str(tmp_path / "k.npy"))
+    env = dict(__import__('os').environ, PDSSM_SELECT_FMA="1")
+    subprocess.run([sys.executable, "-c", code], check=True, env=env, timeout=600)
+    k_fma = np.load(tmp_path / "k.npy")
+    assert (k_tc == k_fma).all()
+    rows = [0, 1, 7, 4095, 9999, 16383]
+    for b in (0, 5):
+        kr = oracle.select(inp.u[b:b + 1, rows], inp.W)
+        assert (k_tc[b][:, rows] == kr[0]).all()
+
+
 # ----------------------------------------------------------------------------
 # chunk transfers: composed maps bit-exact
 # ----------------------------------------------------------------------------
