@@ -56,11 +56,11 @@ __device__ __forceinline__ void own_targets2(const int *pk, int lane, int N, int
 // bwd phase A: w_c = M_s^T lambda^loc_s with lambda^loc from a zero carry
 // ---------------------------------------------------------------------------
 template <typename T, int NPL, bool FULL>
-__global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
+__global__ void __launch_bounds__(kMaxWPC * 32) k_bwdA(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_ba[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const SmemDict sd = stage_dict(p, sm_ba, warp, lane);
-    const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
+    const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
     if (unit >= p.units) return;
     const int N = (int)p.N, K = (int)p.K;
     const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
@@ -113,7 +113,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
         const int n = min(kTS, len - t0);
         const int tp = t0 - kTS;   // the tile processed next
         const bool vp = lane < kTS && tp >= 0;
-        const int knext = load_k(kp, tp + lane, vp, K, p.status);
+        const int knext = load_k_raw(kp, tp + lane, vp);
         const float gynext = vp ? gyp[tp + lane] : 0.f;
         const T *td = reinterpret_cast<const T *>(ring.tile(stage, 0));
         const T *tc = reinterpret_cast<const T *>(ring.tile(stage, 1));
@@ -143,7 +143,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdA(const ChunkParams p) {
             const int tp2 = tile_of(j + p.ns + kPrefetchTiles);
             ring.prefetch(s + (int64_t)tp2 * kTS, min(kTS, len - tp2 * kTS), 2, lane);
         }
-        kreg = knext;
+        kreg = clamp_k(knext, K, p.status);
         gyreg = gynext;
     }
     const int64_t o = unit * p.N;
@@ -314,11 +314,11 @@ __global__ void k_bwdB(const ChunkParams p) {
 // g_b = lambda, g_c = g_y h, g_d = h_{t-1} * lambda[pi(.)].
 // ---------------------------------------------------------------------------
 template <typename T, int NPL, bool FULL>
-__global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
+__global__ void __launch_bounds__(kMaxWPC * 32) k_bwdC(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_bc[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const SmemDict sd = stage_dict(p, sm_bc, warp, lane);
-    const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
+    const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
     if (unit >= p.units) return;
     const int N = (int)p.N, K = (int)p.K;
     const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
@@ -388,7 +388,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
         if (m + 1 < total) {
             const int tn0 = tile_of(m + 1) * kTS;
             const bool v = lane < kTS && tn0 + lane < len;
-            knext = load_k(kp, tn0 + lane, v, K, p.status);
+            knext = load_k_raw(kp, tn0 + lane, v);
             if (m + 1 >= ntiles) gynext = v ? gyp[tn0 + lane] : 0.f;
         }
         const T *td = reinterpret_cast<const T *>(ring.tile(stage, 0));
@@ -464,7 +464,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
             const int tp2 = m + p.ns + kPrefetchTiles;
             ring.prefetch(s + (int64_t)tp2 * kTS, min(kTS, len - tp2 * kTS), 3, lane);
         }
-        kreg = knext;
+        kreg = clamp_k(knext, K, p.status);
         gyreg = gynext;
     }
 }
@@ -473,14 +473,8 @@ __global__ void __launch_bounds__(kWPC * 32) k_bwdC(const ChunkParams p) {
 // launchers
 // ---------------------------------------------------------------------------
 template <typename KernT>
-static cudaError_t launch_chunk_b(KernT kern, const ChunkParams &p, size_t smem,
-                                  cudaStream_t st) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int64_t grid = (p.units + kWPC - 1) / kWPC;
-    kern<<<(unsigned)grid, kWPC * 32, smem, st>>>(p);
-    return cudaGetLastError();
+static cudaError_t launch_chunk_b(KernT kern, const ChunkParams &p, size_t, cudaStream_t st) {
+    return launch_units(kern, p, p.smem_per_warp, st);
 }
 
 #define PDSSM_DISPATCH_B(KERNEL, p, st, smem)                                     \
@@ -495,7 +489,7 @@ template <typename T>
 static cudaError_t bwdA_t(ChunkParams p, cudaStream_t st) {
     const int rowb = (int)p.N * (int)sizeof(T);
     p.smem_per_warp = warp_smem_bytes(p.ns, 2, rowb);
-    const size_t smem = (size_t)dict_region_bytes(p) + (size_t)kWPC * p.smem_per_warp;
+    const size_t smem = 0;
     PDSSM_DISPATCH_B(k_bwdA, p, st, smem);
 }
 
@@ -503,17 +497,19 @@ template <typename T>
 static cudaError_t bwdC_t(ChunkParams p, cudaStream_t st) {
     const int rowb = (int)p.N * (int)sizeof(T);
     p.smem_per_warp = bwd_warp_smem_bytes(p.ns, 3, rowb);
-    const size_t smem = (size_t)dict_region_bytes(p) + (size_t)kWPC * p.smem_per_warp;
+    const size_t smem = 0;
     PDSSM_DISPATCH_B(k_bwdC, p, st, smem);
 }
 
 cudaError_t launch_bwdA(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st) {
     if (p.units == 0) return cudaSuccess;
+    if (fast_path(p)) return launch_bwdA_fast(p, dt, st);
     return dt == PDSSM_BF16 ? bwdA_t<__nv_bfloat16>(p, st) : bwdA_t<float>(p, st);
 }
 
 cudaError_t launch_bwdC(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st) {
     if (p.units == 0) return cudaSuccess;
+    if (fast_path(p)) return launch_bwdC_fast(p, dt, st);
     return dt == PDSSM_BF16 ? bwdC_t<__nv_bfloat16>(p, st) : bwdC_t<float>(p, st);
 }
 

@@ -19,8 +19,8 @@
 
 namespace pdssm {
 
-constexpr int kTS = 16;        // steps per staged tile = steps per readout group
-constexpr int kWPC = 4;        // warps (units) per CTA in the chunk kernels
+constexpr int kTS = 8;         // steps per staged tile = steps per readout group
+constexpr int kMaxWPC = 8;     // most warps (units) per CTA in the chunk kernels
 constexpr int kMaxN = 64;
 constexpr int kMaxStages = 4;
 constexpr int kBwdMaxChunk = 256;   // checkpoints of one chunk kept in shared memory
@@ -89,6 +89,7 @@ struct ChunkParams {
     float *h_last;
     int *status;
     int ns;                   // pipeline stages
+    int wpc;                  // warps (units) per CTA
     int bulk;                 // 1: bulk-copy staging; 0: cooperative copies
     int smem_per_warp;
 };
@@ -173,6 +174,73 @@ static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t par
     return false;
 }
 
+// ---------------------------------------------------------------------------
+// explicit 32-bit shared-memory accesses for the hot loops
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float lds_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float2 lds_f32x2(uint32_t a) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ int lds_s32(uint32_t a) {
+    int v;
+    asm volatile("ld.shared.s32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ int2 lds_s32x2(uint32_t a) {
+    int2 v;
+    asm volatile("ld.shared.v2.s32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ unsigned lds_u8(uint32_t a) {
+    unsigned v;
+    asm volatile("ld.shared.u8 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ unsigned lds_u16(uint32_t a) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ unsigned lds_u32(uint32_t a) {
+    unsigned v;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts_f32(uint32_t a, float v) {
+    asm volatile("st.shared.f32 [%0], %1;" ::"r"(a), "f"(v) : "memory");
+}
+__device__ __forceinline__ void sts_f32x2(uint32_t a, float x, float y) {
+    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(a), "f"(x), "f"(y) : "memory");
+}
+__device__ __forceinline__ void warp_barrier() {
+    asm volatile("bar.warp.sync -1;" ::: "memory");
+}
+// One element of type T at a shared address, as float.
+template <typename T>
+__device__ __forceinline__ float lds_elem(uint32_t a);
+template <>
+__device__ __forceinline__ float lds_elem<float>(uint32_t a) { return lds_f32(a); }
+template <>
+__device__ __forceinline__ float lds_elem<__nv_bfloat16>(uint32_t a) {
+    return __uint_as_float(lds_u16(a) << 16);
+}
+// Two consecutive elements of type T at a shared address (8- or 4-aligned).
+template <typename T>
+__device__ __forceinline__ float2 lds_pair(uint32_t a);
+template <>
+__device__ __forceinline__ float2 lds_pair<float>(uint32_t a) { return lds_f32x2(a); }
+template <>
+__device__ __forceinline__ float2 lds_pair<__nv_bfloat16>(uint32_t a) {
+    const unsigned w = lds_u32(a);
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
 // Reduce-scatter of 16 per-lane partials: lane l (and l + 16) returns
 // sum over all 32 lanes of v[l & 15].  16 shuffles for 16 values.
 __device__ __forceinline__ float reduce_scatter16(float (&v)[kTS]) {
@@ -237,14 +305,21 @@ __device__ __forceinline__ void load_row(const T *row, int lane, int N, float (&
 }
 
 // Selection index of one step, clamped into [0, K) (flagged when it was not).
-__device__ __forceinline__ int load_k(const int32_t *kp, int64_t idx, bool valid, int K,
-                                      int *status) {
-    int kv = valid ? __ldg(kp + idx) : 0;
+__device__ __forceinline__ int clamp_k(int kv, int K, int *status) {
     if (kv < 0 || kv >= K) {
         flag_status(status, kStBadIndex);
         kv = kv < 0 ? 0 : K - 1;
     }
     return kv;
+}
+__device__ __forceinline__ int load_k(const int32_t *kp, int64_t idx, bool valid, int K,
+                                      int *status) {
+    return clamp_k(valid ? __ldg(kp + idx) : 0, K, status);
+}
+// Raw load of the next tile's indices; clamp_k them only when they are used,
+// so the load's latency is hidden behind the current tile.
+__device__ __forceinline__ int load_k_raw(const int32_t *kp, int64_t idx, bool valid) {
+    return valid ? __ldg(kp + idx) : 0;
 }
 
 // ---------------------------------------------------------------------------
@@ -475,7 +550,7 @@ struct SmemDict {
 };
 
 __device__ __forceinline__ void copy_slot(unsigned char *dst, const ChunkParams &p, int64_t dk,
-                                          int tid, int nthr) {
+                                          int tid, int nthr, int scale) {
     const int K = (int)p.K, N = (int)p.N;
     int *m = reinterpret_cast<int *>(dst);
     uint32_t *t = reinterpret_cast<uint32_t *>(dst + K * N * 4);
@@ -483,24 +558,25 @@ __device__ __forceinline__ void copy_slot(unsigned char *dst, const ChunkParams 
     const int32_t *gm = p.dict + dk * K * N;
     const uint32_t *gt = reinterpret_cast<const uint32_t *>(p.tab + dk * K * kDcap * 64);
     const int32_t *gf = p.fan + dk * K;
-    for (int i = tid; i < K * N; i += nthr) m[i] = __ldg(gm + i);
+    for (int i = tid; i < K * N; i += nthr) m[i] = __ldg(gm + i) * scale;
     for (int i = tid; i < K * kDcap * 16; i += nthr) t[i] = __ldg(gt + i);
     for (int i = tid; i < K; i += nthr) f[i] = __ldg(gf + i);
 }
 
 // Loads the dictionary used by this CTA's warps into shared memory and
 // returns this warp's view.  Must be reached by every thread of the CTA.
+// scale = 4 stores map entries as byte offsets into int32 rows.
 __device__ __forceinline__ SmemDict stage_dict(const ChunkParams &p, unsigned char *smem,
-                                               int warp, int lane) {
+                                               int warp, int lane, int scale = 1) {
     const int K = (int)p.K, N = (int)p.N;
     const int slot = dict_slot_bytes(K, N);
     unsigned char *mine = smem;
     if (p.dict_hs == 0) {
-        copy_slot(smem, p, 0, threadIdx.x, blockDim.x);
+        copy_slot(smem, p, 0, threadIdx.x, blockDim.x, scale);
     } else {
         mine = smem + warp * slot;
-        const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
-        if (unit < p.units) copy_slot(mine, p, (unit / p.C) % p.H, lane, 32);
+        const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
+        if (unit < p.units) copy_slot(mine, p, (unit / p.C) % p.H, lane, 32, scale);
     }
     __syncthreads();
     SmemDict sd;
@@ -511,7 +587,132 @@ __device__ __forceinline__ SmemDict stage_dict(const ChunkParams &p, unsigned ch
 }
 
 __host__ __device__ inline int dict_region_bytes(const ChunkParams &p) {
-    return (p.dict_hs == 0 ? 1 : kWPC) * dict_slot_bytes((int)p.K, (int)p.N);
+    return (p.dict_hs == 0 ? 1 : p.wpc) * dict_slot_bytes((int)p.K, (int)p.N);
+}
+
+// ---------------------------------------------------------------------------
+// fast-path helpers (state filling the warp: N = 32 * NPL)
+// ---------------------------------------------------------------------------
+template <typename T, int NPL>
+__device__ __forceinline__ void lds_own(uint32_t a, float (&v)[NPL]) {
+    if constexpr (NPL == 1) {
+        v[0] = lds_elem<T>(a);
+    } else {
+        const float2 q = lds_pair<T>(a);
+        v[0] = q.x;
+        v[1] = q.y;
+    }
+}
+
+// byte offset of element `pos4 / 4` in a row of T
+template <typename T>
+__device__ __forceinline__ uint32_t elem_off(int pos4) {
+    return sizeof(T) == 4 ? (uint32_t)pos4 : (uint32_t)pos4 >> 1;
+}
+
+// The PD step with the slot gather fully unrolled to S slots (S >= the
+// map's fan-in; padding slots point at the zero entry).  Table entries are
+// read-only, so they are fetched before the warp barrier; the S value loads
+// after it issue back to back, and the sums keep the slot (ascending source)
+// order.
+template <int NPL, int S>
+__device__ __forceinline__ void step_slots(float (&h)[NPL], const float (&dv)[NPL],
+                                           const float (&bv)[NPL], uint32_t pb, uint32_t tl,
+                                           int lane) {
+    unsigned w[S];
+#pragma unroll
+    for (int sl = 0; sl < S; ++sl) w[sl] = NPL == 1 ? lds_u8(tl + sl * 64) : lds_u16(tl + sl * 64);
+    if constexpr (NPL == 1)
+        sts_f32(pb + lane * 4, dv[0] * h[0]);
+    else
+        sts_f32x2(pb + lane * 8, dv[0] * h[0], dv[1] * h[1]);
+    warp_barrier();
+    float v[NPL][S];
+#pragma unroll
+    for (int sl = 0; sl < S; ++sl) {
+        if constexpr (NPL == 1) {
+            v[0][sl] = lds_f32(pb + w[sl] * 4);
+        } else {
+            v[0][sl] = lds_f32(pb + (w[sl] & 0xffu) * 4);
+            v[1][sl] = lds_f32(pb + (w[sl] >> 8) * 4);
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        float acc = v[r][0];
+#pragma unroll
+        for (int sl = 1; sl < S; ++sl) acc += v[r][sl];
+        h[r] = acc + bv[r];
+    }
+}
+
+// Dispatch on the map's fan-in class; above kDcap, scan all sources.
+template <int NPL>
+__device__ __forceinline__ void step_any(float (&h)[NPL], const float (&dv)[NPL],
+                                         const float (&bv)[NPL], uint32_t pb, uint32_t tl,
+                                         int Dk, uint32_t pk, int lane) {
+    if (Dk <= 1) {
+        step_slots<NPL, 1>(h, dv, bv, pb, tl, lane);
+    } else if (Dk <= 2) {
+        step_slots<NPL, 2>(h, dv, bv, pb, tl, lane);
+    } else if (Dk <= 4) {
+        step_slots<NPL, 4>(h, dv, bv, pb, tl, lane);
+    } else if (Dk <= kDcap) {
+        step_slots<NPL, kDcap>(h, dv, bv, pb, tl, lane);
+    } else {
+        constexpr int N = 32 * NPL;
+        if constexpr (NPL == 1)
+            sts_f32(pb + lane * 4, dv[0] * h[0]);
+        else
+            sts_f32x2(pb + lane * 8, dv[0] * h[0], dv[1] * h[1]);
+        warp_barrier();
+        float acc[NPL];
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) acc[r] = 0.f;
+        for (int j = 0; j < N; ++j) {
+            const int t4 = lds_s32(pk + j * 4);
+            const float vj = lds_f32(pb + j * 4);
+#pragma unroll
+            for (int r = 0; r < NPL; ++r)
+                if (t4 == (lane * NPL + r) * 4) acc[r] += vj;
+        }
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) h[r] = acc[r] + bv[r];
+    }
+}
+
+// Warps per CTA for a chunk kernel with `per_warp` bytes of shared memory
+// per warp: 4 or 8, whichever keeps more warps resident per SM (the
+// dictionary region is paid once per CTA); assumes <= 64 registers/thread.
+inline int choose_wpc(const ChunkParams &p, int per_warp) {
+    const int budget = 227 * 1024;
+    int best = 4, best_warps = -1;
+    for (int wpc = 4; wpc <= kMaxWPC; wpc *= 2) {
+        ChunkParams q = p;
+        q.wpc = wpc;
+        const int cta = dict_region_bytes(q) + wpc * per_warp + 1024;
+        if (cta > budget) continue;
+        int warps = (228 * 1024 / cta) * wpc;
+        warps = warps > 32 ? 32 : warps;
+        if (warps >= best_warps) {
+            best_warps = warps;
+            best = wpc;
+        }
+    }
+    return best;
+}
+
+template <typename KernT>
+inline cudaError_t launch_units(KernT kern, ChunkParams p, int per_warp, cudaStream_t st) {
+    p.smem_per_warp = per_warp;
+    p.wpc = choose_wpc(p, per_warp);
+    const size_t smem = (size_t)dict_region_bytes(p) + (size_t)p.wpc * per_warp;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    const int64_t grid = (p.units + p.wpc - 1) / p.wpc;
+    kern<<<(unsigned)grid, p.wpc * 32, smem, st>>>(p);
+    return cudaGetLastError();
 }
 
 // ---------------------------------------------------------------------------
@@ -528,6 +729,11 @@ cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, 
 cudaError_t launch_validate(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs,
                             const int32_t *k, int *counts, cudaStream_t st);
 cudaError_t launch_phaseA(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st);
+bool fast_path(const ChunkParams &p);
+cudaError_t launch_phaseA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
+cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
+cudaError_t launch_bwdA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
+cudaError_t launch_bwdC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
 cudaError_t launch_phaseB(const ChunkParams &p, cudaStream_t st);
 cudaError_t launch_phaseC(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st);
 cudaError_t launch_bwdA(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st);

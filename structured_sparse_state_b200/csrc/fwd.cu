@@ -24,11 +24,11 @@ namespace pdssm {
 // phase A
 // ---------------------------------------------------------------------------
 template <typename T, int NPL, bool FULL>
-__global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
+__global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_a[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const SmemDict sd = stage_dict(p, sm_a, warp, lane);
-    const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
+    const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
     if (unit >= p.units) return;
     const int N = (int)p.N, K = (int)p.K;
     const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
@@ -83,8 +83,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
-        const int knext = load_k(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len, K,
-                                 p.status);
+        const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
         const T *rd = reinterpret_cast<const T *>(ring.tile(stage, 0));
         const T *rb = reinterpret_cast<const T *>(ring.tile(stage, 1));
         const T *rc = reinterpret_cast<const T *>(ring.tile(stage, 2));
@@ -129,7 +128,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
             const int pf = i + p.ns + kPrefetchTiles;
             if (pf < ntiles) ring.prefetch(s + (int64_t)pf * kTS, min(kTS, len - pf * kTS), nt, lane);
         }
-        kreg = knext;
+        kreg = clamp_k(knext, K, p.status);
     }
     const int64_t o = unit * p.N;
 #pragma unroll
@@ -147,11 +146,11 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseA(const ChunkParams p) {
 // phase C (carry correction in path form)
 // ---------------------------------------------------------------------------
 template <typename T, int NPL, bool FULL>
-__global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
+__global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_c[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const SmemDict sd = stage_dict(p, sm_c, warp, lane);
-    const int64_t unit = (int64_t)blockIdx.x * kWPC + warp;
+    const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
     if (unit >= p.units) return;
     const int N = (int)p.N, K = (int)p.K;
     const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
@@ -203,8 +202,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
-        const int knext = load_k(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len, K,
-                                 p.status);
+        const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
         const float yold = lane < n ? yp[t0 + lane] : 0.f;
         const T *rd = reinterpret_cast<const T *>(ring.tile(stage, 0));
         const T *rc = reinterpret_cast<const T *>(ring.tile(stage, 1));
@@ -234,7 +232,7 @@ __global__ void __launch_bounds__(kWPC * 32) k_phaseC(const ChunkParams p) {
             const int pf = i + p.ns + kPrefetchTiles;
             if (pf < ntiles) ring.prefetch(s + (int64_t)pf * kTS, min(kTS, len - pf * kTS), 2, lane);
         }
-        kreg = knext;
+        kreg = clamp_k(knext, K, p.status);
     }
 }
 
@@ -446,13 +444,8 @@ __global__ void k_phaseB(const ChunkParams p) {
 // launchers
 // ---------------------------------------------------------------------------
 template <typename KernT>
-static cudaError_t launch_chunk(KernT kern, const ChunkParams &p, size_t smem, cudaStream_t st) {
-    cudaError_t e =
-        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    const int64_t grid = (p.units + kWPC - 1) / kWPC;
-    kern<<<(unsigned)grid, kWPC * 32, smem, st>>>(p);
-    return cudaGetLastError();
+static cudaError_t launch_chunk(KernT kern, const ChunkParams &p, size_t, cudaStream_t st) {
+    return launch_units(kern, p, p.smem_per_warp, st);
 }
 
 // Template choice: NPL = elements per lane, FULL = the state fills the warp.
@@ -468,7 +461,7 @@ template <typename T>
 static cudaError_t phaseA_t(ChunkParams p, cudaStream_t st) {
     const int rowb = (int)p.N * (int)sizeof(T);
     p.smem_per_warp = warp_smem_bytes(p.ns, 3, rowb);
-    const size_t smem = (size_t)dict_region_bytes(p) + (size_t)kWPC * p.smem_per_warp;
+    const size_t smem = 0;
     PDSSM_DISPATCH(k_phaseA, p, st, smem);
 }
 
@@ -476,17 +469,19 @@ template <typename T>
 static cudaError_t phaseC_t(ChunkParams p, cudaStream_t st) {
     const int rowb = (int)p.N * (int)sizeof(T);
     p.smem_per_warp = warp_smem_bytes(p.ns, 2, rowb);
-    const size_t smem = (size_t)dict_region_bytes(p) + (size_t)kWPC * p.smem_per_warp;
+    const size_t smem = 0;
     PDSSM_DISPATCH(k_phaseC, p, st, smem);
 }
 
 cudaError_t launch_phaseA(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st) {
     if (p.units == 0) return cudaSuccess;
+    if (fast_path(p)) return launch_phaseA_fast(p, dt, st);
     return dt == PDSSM_BF16 ? phaseA_t<__nv_bfloat16>(p, st) : phaseA_t<float>(p, st);
 }
 
 cudaError_t launch_phaseC(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st) {
     if (p.units == 0) return cudaSuccess;
+    if (fast_path(p)) return launch_phaseC_fast(p, dt, st);
     return dt == PDSSM_BF16 ? phaseC_t<__nv_bfloat16>(p, st) : phaseC_t<float>(p, st);
 }
 

@@ -1,0 +1,276 @@
+// Forward phases A and C for a state that fills the warp (N = 32 or 64):
+// the same arithmetic as fwd.cu, written against explicit 32-bit shared
+// addresses so that a step costs few integer instructions:
+//   * the dictionary is staged as byte offsets (entry * 4), so following a
+//     column is one shared load per step;
+//   * the three tensors of a staged row sit at fixed distances, read with
+//     immediate offsets;
+//   * readout partials go to the per-warp transpose buffer.
+// The general kernels in fwd.cu serve every other N.
+#include "common.cuh"
+
+namespace pdssm {
+
+template <typename T, int NPL>
+__global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA_fast(const ChunkParams p) {
+    extern __shared__ __align__(128) unsigned char sm_a[];
+    constexpr int N = 32 * NPL;
+    constexpr int ROWB = N * (int)sizeof(T);
+    constexpr int TENS = kTS * ROWB;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const SmemDict sd = stage_dict(p, sm_a, warp, lane, 4);
+    const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
+    if (unit >= p.units) return;
+    const int K = (int)p.K;
+    const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
+    const int64_t s = cidx * p.chunk;
+    const int len = (int)imin64(p.chunk, p.L - s);
+    const bool with_y = p.y != nullptr;
+    const int nt = with_y ? 3 : 2;
+
+    unsigned char *wbase = sm_a + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
+    Ring<3> ring;
+    ring.buf = wbase;
+    ring.rowb = ROWB;
+    ring.esz = (int)sizeof(T);
+    ring.tens_bytes = TENS;
+    ring.stage_bytes = 3 * TENS;
+    ring.ns = p.ns;
+    ring.bulk = p.bulk != 0;
+    float *pbuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes);
+    float *ybuf = pbuf + 2 * kPbStride;
+    ring.bar0 = smem_u32(ybuf + kYbufFloats);
+    const int64_t seq_row0 = bh * p.L;
+    ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * ROWB;
+    ring.src[1] = reinterpret_cast<const unsigned char *>(p.b) + seq_row0 * ROWB;
+    ring.src[2] = with_y ? reinterpret_cast<const unsigned char *>(p.c) + seq_row0 * ROWB
+                         : ring.src[1];
+    ring_init_bars(ring.bar0, p.ns, lane);
+
+    const int ntiles = (len + kTS - 1) / kTS;
+    for (int i = 0; i < p.ns && i < ntiles; ++i)
+        ring.issue(i, s + (int64_t)i * kTS, min(kTS, len - i * kTS), nt, lane);
+    for (int i = p.ns; i < p.ns + kPrefetchTiles && i < ntiles; ++i)
+        ring.prefetch(s + (int64_t)i * kTS, min(kTS, len - i * kTS), nt, lane);
+    clear_pb(pbuf, lane);
+
+    const uint32_t map_s = smem_u32(sd.map), fan_s = smem_u32(sd.fan);
+    const uint32_t tab_lane = smem_u32(sd.tab) + lane * NPL;
+    const uint32_t pb_s = smem_u32(pbuf), yb_lane = smem_u32(ybuf) + lane * 4;
+    const uint32_t own_off = lane * NPL * (uint32_t)sizeof(T);
+
+    float h[NPL], Dl[NPL];
+    int pos4[NPL];
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        h[r] = 0.f;
+        Dl[r] = 1.f;
+        pos4[r] = (lane * NPL + r) * 4;
+    }
+    const int32_t *kp = p.k + seq_row0 + s;
+    int kreg = load_k(kp, lane, lane < kTS && lane < len, K, p.status);
+
+    for (int i = 0; i < ntiles; ++i) {
+        const int stage = i % p.ns;
+        if (!ring.wait(stage, (uint32_t)((i / p.ns) & 1))) {
+            ring_abort(ring, i, min(ntiles, i + p.ns), p.status, lane);
+            return;
+        }
+        const int t0 = i * kTS;
+        const int n = min(kTS, len - t0);
+        const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
+        uint32_t row = smem_u32(ring.tile(stage, 0));
+        uint32_t yb = yb_lane;
+        // values of step q that do not depend on the state, loaded one step
+        // ahead so their latency overlaps the previous step's gather
+        int kk = __shfl_sync(kFull, kreg, 0);
+        uint32_t pk = map_s + kk * (N * 4);
+        float dv[NPL], bv[NPL], cv[NPL];
+        lds_own<T, NPL>(row + own_off, dv);
+        lds_own<T, NPL>(row + own_off + TENS, bv);
+        if (with_y) lds_own<T, NPL>(row + own_off + 2 * TENS, cv);
+        int Dk = lds_s32(fan_s + kk * 4);
+        uint32_t tl = tab_lane + kk * (kDcap * 64);
+        for (int q = 0; q < n; ++q, row += ROWB, yb += 33 * 4) {
+            // transfer tracking: Delta picks up d at the column's current
+            // position, then the selected map moves the column
+#pragma unroll
+            for (int r = 0; r < NPL; ++r) {
+                Dl[r] *= lds_elem<T>(row + elem_off<T>(pos4[r]));
+                pos4[r] = lds_s32(pk + pos4[r]);
+            }
+            step_any<NPL>(h, dv, bv, pb_s + (q & 1) * (kPbStride * 4), tl, Dk, pk, lane);
+            // next step's state-independent values
+            const int q1 = q + 1 < n ? q + 1 : q;
+            const int kk_n = __shfl_sync(kFull, kreg, q1);
+            const uint32_t pk_n = map_s + kk_n * (N * 4);
+            const uint32_t row_n = row + (q + 1 < n ? ROWB : 0);
+            float dv_n[NPL], bv_n[NPL], cv_n[NPL];
+            lds_own<T, NPL>(row_n + own_off, dv_n);
+            lds_own<T, NPL>(row_n + own_off + TENS, bv_n);
+            if (with_y) lds_own<T, NPL>(row_n + own_off + 2 * TENS, cv_n);
+            const int Dk_n = lds_s32(fan_s + kk_n * 4);
+            const uint32_t tl_n = tab_lane + kk_n * (kDcap * 64);
+            if (with_y) {
+                float ya = cv[0] * h[0];
+#pragma unroll
+                for (int r = 1; r < NPL; ++r) ya = fmaf(cv[r], h[r], ya);
+                sts_f32(yb, ya);
+            }
+            kk = kk_n;
+            pk = pk_n;
+            Dk = Dk_n;
+            tl = tl_n;
+#pragma unroll
+            for (int r = 0; r < NPL; ++r) {
+                dv[r] = dv_n[r];
+                bv[r] = bv_n[r];
+                cv[r] = cv_n[r];
+            }
+        }
+        warp_barrier();
+        if (with_y) {
+            const float ys = ybuf_row_sum(ybuf, lane, n);
+            if (lane < n) p.y[seq_row0 + s + t0 + lane] = ys;
+        }
+        warp_barrier();
+        if (i + p.ns < ntiles)
+            ring.issue(stage, s + (int64_t)(i + p.ns) * kTS, min(kTS, len - (i + p.ns) * kTS), nt,
+                       lane);
+        {
+            const int pf = i + p.ns + kPrefetchTiles;
+            if (pf < ntiles) ring.prefetch(s + (int64_t)pf * kTS, min(kTS, len - pf * kTS), nt, lane);
+        }
+        kreg = clamp_k(knext, K, p.status);
+    }
+    const int64_t o = unit * p.N;
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        const int e = lane * NPL + r;
+        p.Pi[o + e] = pos4[r] >> 2;
+        p.Dl[o + e] = Dl[r];
+        p.v[o + e] = h[r];
+    }
+}
+
+template <typename T, int NPL>
+__global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams p) {
+    extern __shared__ __align__(128) unsigned char sm_c[];
+    constexpr int N = 32 * NPL;
+    constexpr int ROWB = N * (int)sizeof(T);
+    constexpr int TENS = kTS * ROWB;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const SmemDict sd = stage_dict(p, sm_c, warp, lane, 4);
+    const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
+    if (unit >= p.units) return;
+    const int K = (int)p.K;
+    const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
+    if (cidx == 0 && p.h0 == nullptr) return;   // zero initial state: nothing to correct
+    const int64_t s = cidx * p.chunk;
+    const int len = (int)imin64(p.chunk, p.L - s);
+
+    unsigned char *wbase = sm_c + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
+    Ring<2> ring;
+    ring.buf = wbase;
+    ring.rowb = ROWB;
+    ring.esz = (int)sizeof(T);
+    ring.tens_bytes = TENS;
+    ring.stage_bytes = 2 * TENS;
+    ring.ns = p.ns;
+    ring.bulk = p.bulk != 0;
+    float *ybuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes) + 2 * kPbStride;
+    ring.bar0 = smem_u32(ybuf + kYbufFloats);
+    const int64_t seq_row0 = bh * p.L;
+    ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * ROWB;
+    ring.src[1] = reinterpret_cast<const unsigned char *>(p.c) + seq_row0 * ROWB;
+    ring_init_bars(ring.bar0, p.ns, lane);
+
+    const int ntiles = (len + kTS - 1) / kTS;
+    for (int i = 0; i < p.ns && i < ntiles; ++i)
+        ring.issue(i, s + (int64_t)i * kTS, min(kTS, len - i * kTS), 2, lane);
+    for (int i = p.ns; i < p.ns + kPrefetchTiles && i < ntiles; ++i)
+        ring.prefetch(s + (int64_t)i * kTS, min(kTS, len - i * kTS), 2, lane);
+
+    const uint32_t map_s = smem_u32(sd.map), yb_lane = smem_u32(ybuf) + lane * 4;
+    float w[NPL];
+    int pos4[NPL];
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        const int e = lane * NPL + r;
+        pos4[r] = e * 4;
+        w[r] = cidx == 0 ? p.h0[bh * p.N + e] : p.Hc[(unit - 1) * p.N + e];
+    }
+    const int32_t *kp = p.k + seq_row0 + s;
+    float *yp = p.y + seq_row0 + s;
+    int kreg = load_k(kp, lane, lane < kTS && lane < len, K, p.status);
+
+    for (int i = 0; i < ntiles; ++i) {
+        const int stage = i % p.ns;
+        if (!ring.wait(stage, (uint32_t)((i / p.ns) & 1))) {
+            ring_abort(ring, i, min(ntiles, i + p.ns), p.status, lane);
+            return;
+        }
+        const int t0 = i * kTS;
+        const int n = min(kTS, len - t0);
+        const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
+        const float yold = lane < n ? yp[t0 + lane] : 0.f;
+        uint32_t row = smem_u32(ring.tile(stage, 0));
+        uint32_t yb = yb_lane;
+#pragma unroll 2
+        for (int q = 0; q < n; ++q, row += ROWB, yb += 33 * 4) {
+            const int kk = __shfl_sync(kFull, kreg, q);
+            const uint32_t pk = map_s + kk * (N * 4);
+            float acc = 0.f;
+#pragma unroll
+            for (int r = 0; r < NPL; ++r) {
+                w[r] *= lds_elem<T>(row + elem_off<T>(pos4[r]));
+                pos4[r] = lds_s32(pk + pos4[r]);
+                acc = fmaf(lds_elem<T>(row + TENS + elem_off<T>(pos4[r])), w[r], acc);
+            }
+            sts_f32(yb, acc);
+        }
+        warp_barrier();
+        const float ys = ybuf_row_sum(ybuf, lane, n);
+        if (lane < n) yp[t0 + lane] = yold + ys;
+        warp_barrier();
+        if (i + p.ns < ntiles)
+            ring.issue(stage, s + (int64_t)(i + p.ns) * kTS, min(kTS, len - (i + p.ns) * kTS), 2,
+                       lane);
+        {
+            const int pf = i + p.ns + kPrefetchTiles;
+            if (pf < ntiles) ring.prefetch(s + (int64_t)pf * kTS, min(kTS, len - pf * kTS), 2, lane);
+        }
+        kreg = clamp_k(knext, K, p.status);
+    }
+}
+
+template <typename KernT>
+static cudaError_t launch_fast(KernT kern, const ChunkParams &p, size_t, cudaStream_t st) {
+    return launch_units(kern, p, p.smem_per_warp, st);
+}
+
+bool fast_path(const ChunkParams &p) { return p.N == 32 || p.N == 64; }
+
+cudaError_t launch_phaseA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
+    const int es = dt == PDSSM_BF16 ? 2 : 4;
+    p.smem_per_warp = warp_smem_bytes(p.ns, 3, (int)p.N * es);
+    const size_t smem = 0;
+    if (dt == PDSSM_BF16)
+        return p.N == 64 ? launch_fast(k_phaseA_fast<__nv_bfloat16, 2>, p, smem, st)
+                         : launch_fast(k_phaseA_fast<__nv_bfloat16, 1>, p, smem, st);
+    return p.N == 64 ? launch_fast(k_phaseA_fast<float, 2>, p, smem, st)
+                     : launch_fast(k_phaseA_fast<float, 1>, p, smem, st);
+}
+
+cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
+    const int es = dt == PDSSM_BF16 ? 2 : 4;
+    p.smem_per_warp = warp_smem_bytes(p.ns, 2, (int)p.N * es);
+    const size_t smem = 0;
+    if (dt == PDSSM_BF16)
+        return p.N == 64 ? launch_fast(k_phaseC_fast<__nv_bfloat16, 2>, p, smem, st)
+                         : launch_fast(k_phaseC_fast<__nv_bfloat16, 1>, p, smem, st);
+    return p.N == 64 ? launch_fast(k_phaseC_fast<float, 2>, p, smem, st)
+                     : launch_fast(k_phaseC_fast<float, 1>, p, smem, st);
+}
+
+}  // namespace pdssm

@@ -12,13 +12,15 @@
 //
 // Certification.  Let S = ||u_row||_2 * max_k ||W_hk||_2 >= sum_d |u_d W_kd|
 // (Cauchy-Schwarz).  The tensor-core logit differs from the exact real sum
-// by at most (D * 2^-20 + 2^-16) S (the first term allows every one of the 2D
-// accumulations to lose 4 ulp of fp32), and the contract's fp32 fma chain
-// differs from it by at most D * 2^-24 S.  With eps the sum of both, a
-// tensor-core top-1 that leads the runner-up by more than 2 eps is the strict
-// argmax of the fma chain too.  Otherwise the epilogue recomputes the K fma
-// chains of that (row, head) exactly and takes their first argmax, so k is
-// bit-for-bit the contract's result either way.
+// by at most (D * 2^-21 + 2^-16) S (the first term allows each of the 2D
+// products to lose 2 ulp of fp32 in the accumulation), and the contract's
+// fp32 fma chain differs from it by at most D * 2^-24 S.  With eps the sum of
+// both, any k whose tensor-core logit is below top-1 minus 2 eps has an fma
+// logit strictly below the fma logit of top-1, so the contract's first
+// argmax is among the candidates within 2 eps of the top.  One candidate:
+// it is the answer.  Several: the epilogue evaluates their fp32 fma chains
+// exactly and takes the first maximum, so k is bit-for-bit the contract's
+// result either way.
 //
 // Operand layouts in shared memory (K-major, no swizzle, 16-byte core rows):
 //   A: [D/8 k-chunks][128 rows][8 bf16]     (TMA boxes of 8 x 128)
@@ -33,6 +35,7 @@
 namespace pdssm {
 
 constexpr int kTcRows = 128;
+constexpr int kTcThreads = 256;   // two warps per group of 32 TMEM lanes
 
 __device__ __forceinline__ uint64_t umma_smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
     uint64_t d = 0;
@@ -118,13 +121,15 @@ __host__ __device__ inline size_t tc_smem_bytes(int D, int NP, int H) {
 }
 
 template <int KT>
-__global__ void __launch_bounds__(kTcRows, 1)
+__global__ void __launch_bounds__(kTcThreads, 1)
     k_select_tc(const __grid_constant__ CUtensorMap umap, const TcSelectParams p) {
     extern __shared__ __align__(1024) unsigned char sm_raw[];
     // 1024-byte alignment of the operand region
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int quad = warp & 3, half = warp >> 2;   // TMEM lane group, column half
+    const int rtid = quad * 32 + lane;              // row of the tile this thread reads
     const int D = p.D, NP = p.NP, H = p.H, K = KT;
     const int nkc = D / 8;
     unsigned char *Bs = sm;                               // [2][nkc][NP][8] bf16
@@ -138,7 +143,7 @@ __global__ void __launch_bounds__(kTcRows, 1)
 
     // ---- weights: split into hi/lo bf16 parts in the K-major slab layout ----
     const int HK = H * K;
-    for (int idx = tid; idx < NP * D; idx += kTcRows) {
+    for (int idx = tid; idx < NP * D; idx += kTcThreads) {
         const int n = idx / D, d = idx - n * D;
         const float w = n < HK ? __ldg(p.W + (int64_t)n * D + d) : 0.f;
         const __nv_bfloat16 hi = __float2bfloat16_rn(w);
@@ -148,7 +153,7 @@ __global__ void __launch_bounds__(kTcRows, 1)
         *reinterpret_cast<__nv_bfloat16 *>(Bs + (size_t)nkc * NP * 16 + off) = lo;
     }
     // per-head bound on ||W_hk||_2 (rounded up)
-    for (int h = warp; h < H; h += kTcRows / 32) {
+    for (int h = warp; h < H; h += kTcThreads / 32) {
         float mx = 0.f;
         for (int kk = 0; kk < K; ++kk) {
             float ss = 0.f;
@@ -222,9 +227,9 @@ __global__ void __launch_bounds__(kTcRows, 1)
         ok = mbar_wait_bounded(barM, (uint32_t)(it & 1)) && ok;
         tc_fence_after();
 
-        // ---- epilogue: one row per thread ----
-        const int64_t row = (int64_t)tile * kTcRows + tid;
-        const unsigned char *arow = As + (size_t)buf * abytes + tid * 16;
+        // ---- epilogue: one row per thread, half of the columns per warp ----
+        const int64_t row = (int64_t)tile * kTcRows + rtid;
+        const unsigned char *arow = As + (size_t)buf * abytes + rtid * 16;
         float unorm = 0.f;
         for (int q = 0; q < nkc; ++q) {
             const uint4 v = *reinterpret_cast<const uint4 *>(arow + q * (kTcRows * 16));
@@ -237,43 +242,47 @@ __global__ void __launch_bounds__(kTcRows, 1)
             }
         }
         unorm = __fmul_ru(__fsqrt_ru(unorm), 1.0009765625f);
-        const float ceps = 1.01f * ((float)D * 9.5367431640625e-07f + 1.52587890625e-05f +
-                                    (float)D * 5.9604644775390625e-08f);   // D 2^-20 + 2^-16 + D 2^-24
+        // D 2^-21 + 2^-16 + D 2^-24, with a margin for the rounding of the test
+        const float ceps = 1.01f * ((float)D * 4.76837158203125e-07f + 1.52587890625e-05f +
+                                    (float)D * 5.9604644775390625e-08f);
         const int64_t bb = row / p.L, t = row - bb * p.L;
         const bool live = row < p.rows;
-        // One head: certified tensor-core argmax, else the exact fma chains.
         auto decide = [&](const float *lg, int h) {
+            float b1 = lg[0];
             int best = 0;
-            float b1 = lg[0], b2 = -INFINITY;
 #pragma unroll
-            for (int kk = 1; kk < KT; ++kk) {
-                const float v = lg[kk];
-                if (v > b1) {
-                    b2 = b1;
-                    b1 = v;
+            for (int kk = 1; kk < KT; ++kk)
+                if (lg[kk] > b1) {
+                    b1 = lg[kk];
                     best = kk;
-                } else if (v > b2) {
-                    b2 = v;
                 }
-            }
-            const float eps = __fmul_ru(__fmul_ru(unorm, Wn[h]), ceps);
-            if (!(KT == 1 || b1 - b2 > 2.0f * eps)) {
+            const float thr = b1 - 2.0f * __fmul_ru(__fmul_ru(unorm, Wn[h]), ceps);
+            unsigned cand = 0;
+#pragma unroll
+            for (int kk = 0; kk < KT; ++kk) cand |= (lg[kk] >= thr ? 1u : 0u) << kk;
+            if (__popc(cand) > 1) {
+                // the contract's fp32 fma chains of the candidates, first maximum
                 float bv = 0.f;
-                best = 0;
-                for (int kk = 0; kk < KT; ++kk) {
+                best = -1;
+                while (cand) {
+                    const int kk = __ffs(cand) - 1;
+                    cand &= cand - 1;
                     const float *wr = p.W + ((int64_t)h * KT + kk) * D;
                     float acc = 0.f;
                     for (int q = 0; q < nkc; ++q) {
                         const uint4 v = *reinterpret_cast<const uint4 *>(arow + q * (kTcRows * 16));
                         const __nv_bfloat162 *b2v = reinterpret_cast<const __nv_bfloat162 *>(&v);
+                        const float4 w0 = __ldg(reinterpret_cast<const float4 *>(wr + q * 8));
+                        const float4 w1 = __ldg(reinterpret_cast<const float4 *>(wr + q * 8 + 4));
+                        const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
                             const float2 f = __bfloat1622float2(b2v[i]);
-                            acc = __fmaf_rn(__ldg(wr + q * 8 + 2 * i), f.x, acc);
-                            acc = __fmaf_rn(__ldg(wr + q * 8 + 2 * i + 1), f.y, acc);
+                            acc = __fmaf_rn(wv[2 * i], f.x, acc);
+                            acc = __fmaf_rn(wv[2 * i + 1], f.y, acc);
                         }
                     }
-                    if (kk == 0 || acc > bv) {
+                    if (best < 0 || acc > bv) {
                         bv = acc;
                         best = kk;
                     }
@@ -281,10 +290,11 @@ __global__ void __launch_bounds__(kTcRows, 1)
             }
             if (live) p.k_out[(bb * H + h) * p.L + t] = ok ? best : -1;
         };
-        const uint32_t tlane = tmem + ((uint32_t)(warp * 32) << 16);
+        const uint32_t tlane = tmem + ((uint32_t)(quad * 32) << 16);
         if constexpr (KT <= 16) {
-            // 16 columns per load hold 16 / KT whole heads
-            for (int c = 0; c < NP / 16; ++c) {
+            // 16 columns per load hold 16 / KT whole heads; the two warps of a
+            // lane group take alternate loads
+            for (int c = half; c < NP / 16; c += 2) {
                 float v[16];
                 tmem_ld16(tlane + (uint32_t)(c * 16), v);
 #pragma unroll
@@ -294,7 +304,7 @@ __global__ void __launch_bounds__(kTcRows, 1)
                 }
             }
         } else {
-            for (int h = 0; h < H; ++h) {
+            for (int h = half; h < H; h += 2) {
                 float v[32];
                 tmem_ld16(tlane + (uint32_t)(h * 32), *reinterpret_cast<float(*)[16]>(v));
                 tmem_ld16(tlane + (uint32_t)(h * 32 + 16), *reinterpret_cast<float(*)[16]>(v + 16));
@@ -374,7 +384,7 @@ cudaError_t launch_select_tc(const pdssm_dims &dm, const void *u, const float *W
         cudaError_t e =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<grid, kTcRows, smem, st>>>(map, p);
+        kern<<<grid, kTcThreads, smem, st>>>(map, p);
         return cudaGetLastError();
     };
     switch (p.K) {
