@@ -141,6 +141,37 @@ pdssm_status pdssm_scan_bwd(const pdssm_dims *dims, const int32_t *pi_dict,
                             void *stream);
 
 /*
+ * pdssm_scan_fwd for callers that cannot allocate device memory.  The pages
+ * have no counterpart of this call: it exists for host code that owns no
+ * allocator (device memory held by another framework's pool), must not call
+ * cudaMalloc in its loop (the call can synchronise the device), or runs
+ * where allocation after start-up is forbidden.  Same arguments and results
+ * as pdssm_scan_fwd without `ws`: the workspace is a file-scope device array
+ * of pdssm_noalloc_scratch_bytes() bytes (4 MiB) that every GPU loading the
+ * library holds until the process exits; nothing is allocated.
+ *  * Sizes whose workspace (pdssm_workspace_bytes(..., 0)) exceeds that
+ *    maximum return PDSSM_ERR_UNSUPPORTED before anything is launched.
+ *  * The first call on a device looks up the array's device address (once
+ *    per device, with that device current); make that first call before any
+ *    stream capture.
+ *  * Every call on a device shares the one array and it keeps the last
+ *    call's contents (each call resets what must start at zero).  Calls whose
+ *    work overlaps on the GPU (different streams, no ordering) race on it.
+ *  * The device status word of these calls lives in the shared array and is
+ *    not exposed; check indices with pdssm_validate when in doubt.
+ */
+pdssm_status pdssm_scan_fwd_noalloc(const pdssm_dims *dims,
+                                    const int32_t *pi_dict,
+                                    int64_t pi_head_stride, const int32_t *k,
+                                    const void *d, const void *b,
+                                    const void *c, pdssm_dtype in_dtype,
+                                    const float *h0, float *y, float *h_last,
+                                    int64_t chunk, void *stream);
+
+/* Size in bytes of the static scratch array of pdssm_scan_fwd_noalloc. */
+size_t pdssm_noalloc_scratch_bytes(void);
+
+/*
  * Phase A alone, exposing each chunk's closed PD transfer (for tests of the
  * composed index maps, which must match bit for bit):
  *     h_e = P_{Pi_c} diag(Delta_c) h_{s-1} + v_c   for the chunk s..e.

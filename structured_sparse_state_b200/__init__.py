@@ -34,7 +34,7 @@ STATUS = {0: "PDSSM_OK", 1: "PDSSM_ERR_INVALID_ARG", 2: "PDSSM_ERR_UNSUPPORTED",
 EXPORTS = ("pdssm_status_str", "pdssm_last_error", "pdssm_version",
            "pdssm_workspace_bytes", "pdssm_select", "pdssm_scan_fwd",
            "pdssm_scan_bwd", "pdssm_chunk_transfers", "pdssm_validate",
-           "pdssm_ws_status")
+           "pdssm_ws_status", "pdssm_scan_fwd_noalloc", "pdssm_noalloc_scratch_bytes")
 
 
 class Dims(ctypes.Structure):
@@ -68,6 +68,8 @@ def _load() -> ctypes.CDLL:
         "pdssm_chunk_transfers": (I32, [D, P, I64, P, P, P, I32, I64, P, P, P, P, SZ, P]),
         "pdssm_validate": (I32, [D, P, I64, P, P, SZ, P]),
         "pdssm_ws_status": (I32, [P, SZ, P]),
+        "pdssm_scan_fwd_noalloc": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, I64, P]),
+        "pdssm_noalloc_scratch_bytes": (SZ, []),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -223,6 +225,32 @@ def pdssm_scan_fwd(pi_dict, k, d, b, c, h0=None, chunk=128, ws=None, y=None, h_l
                                _ptr(h_last), int(chunk), _ptr(ws), ws.numel(),
                                _stream(stream)), "pdssm_scan_fwd")
     return y, h_last, ws
+
+
+def pdssm_scan_fwd_noalloc(pi_dict, k, d, b, c, h0=None, chunk=128, y=None, h_last=None,
+                           stream=None):
+    """pdssm_scan_fwd without a workspace argument: for callers that cannot
+    allocate device memory, the scratch is the library's fixed device array
+    (pdssm_noalloc_scratch_bytes()).  Pass preallocated y / h_last to keep the
+    call itself free of allocations.  Returns (y, h_last)."""
+    B, H, L, N, K, stride = _scan_shapes(pi_dict, k, d, b, c)
+    dev = d.device
+    if h0 is not None:
+        _cuda(h0, "h0", (torch.float32,))
+    if y is None:
+        y = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    if h_last is None:
+        h_last = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dm = dims(B, H, L, N, K)
+    _check(_lib.pdssm_scan_fwd_noalloc(ctypes.byref(dm), _ptr(pi_dict), stride, _ptr(k),
+                                       _ptr(d), _ptr(b), _ptr(c), _dtype_code(d), _ptr(h0),
+                                       _ptr(y), _ptr(h_last), int(chunk), _stream(stream)),
+           "pdssm_scan_fwd_noalloc")
+    return y, h_last
+
+
+def pdssm_noalloc_scratch_bytes() -> int:
+    return int(_lib.pdssm_noalloc_scratch_bytes())
 
 
 def pdssm_scan_bwd(pi_dict, k, d, b, c, h0, g_y, ws, chunk=128, g_hlast=None, out=None,
