@@ -135,16 +135,20 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
     const int32_t *src = pi + dk * pi_hs + kk * N;
     uint8_t *t = tab + m * (kDcap * 64);
     for (int i = lane; i < kDcap * 64; i += 32) t[i] = (uint8_t)kZeroSlot;
+    // the map's row, two entries per lane, sanitised once
+    int ta = lane < N ? __ldg(src + lane) : 0;
+    int tb = lane + 32 < N ? __ldg(src + lane + 32) : 0;
+    bool bad = (lane < N && (ta < 0 || ta >= N)) || (lane + 32 < N && (tb < 0 || tb >= N));
+    ta = min(max(ta, 0), N - 1);
+    tb = min(max(tb, 0), N - 1);
+    if (lane < N) dict[m * N + lane] = ta;
+    if (lane + 32 < N) dict[m * N + lane + 32] = tb;
     __syncwarp();
     int cnt0 = 0, cnt1 = 0;   // sources of targets lane and lane + 32
-    bool bad = false;
     for (int j = 0; j < N; ++j) {
-        int tgt = __ldg(src + j);
-        if (tgt < 0 || tgt >= N) {
-            bad = true;
-            tgt = tgt < 0 ? 0 : N - 1;
-        }
-        if (lane == 0) dict[m * N + j] = tgt;
+        const int va = __shfl_sync(kFull, ta, j & 31);
+        const int vb = __shfl_sync(kFull, tb, j & 31);
+        const int tgt = j < 32 ? va : vb;
         if (tgt == lane) {
             if (cnt0 < kDcap) t[cnt0 * 64 + lane] = (uint8_t)j;
             ++cnt0;
@@ -153,6 +157,7 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
             ++cnt1;
         }
     }
+    bad = __any_sync(kFull, bad);
     if (bad && lane == 0) flag_status(status, kStBadIndex);
     const int D = __reduce_max_sync(kFull, max(cnt0, cnt1));
     if (lane == 0) fan[m] = D;
