@@ -48,6 +48,10 @@ def parse():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle cpu_baseline leg")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--batch", type=int, default=0,
+                    help="override B per GPU (small cases for profiler captures)")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override L (small cases for profiler captures)")
     return ap.parse_args()
 
 
@@ -459,7 +463,12 @@ def run_reference(args, cfg):
 
 def main():
     args = parse()
-    cfg = gen.workload(workload_index(args.workload))
+    over = {}
+    if args.batch:
+        over["B"] = args.batch
+    if args.seq_len:
+        over["L"] = args.seq_len
+    cfg = gen.workload(workload_index(args.workload), **over)
     if args.impl == "reference":
         out = run_reference(args, cfg)
     else:

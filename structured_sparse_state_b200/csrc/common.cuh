@@ -425,6 +425,21 @@ __device__ __forceinline__ void pd_gather_step(float (&h)[NPL], const float (&dv
     for (int r = 0; r < NPL; ++r) h[r] = (FULL || lane * NPL + r < N) ? acc[r] + bv[r] : 0.f;
 }
 
+// Sum over the warp of per-step partials staged in ybuf[q][33] (kTS = 8
+// rows): lane l adds 8 entries of row l / 4, two shuffles combine the four
+// quarters, and lane 4 q ends up with the total of row q.  Conflict-free.
+// Caller synchronises before; every lane must call it.
+__device__ __forceinline__ float ybuf_quad_sum(const float *ybuf, int lane) {
+    static_assert(kTS == 8, "quarter-row reduction assumes 8 rows");
+    const float *src = ybuf + (lane >> 2) * 33 + (lane & 3) * 8;
+    float s = src[0];
+#pragma unroll
+    for (int i = 1; i < 8; ++i) s += src[i];
+    s += __shfl_xor_sync(kFull, s, 1);
+    s += __shfl_xor_sync(kFull, s, 2);
+    return s;
+}
+
 // Sum over the warp of per-step partials staged in ybuf[q][33] (rows
 // q < n): lane q < n returns the total of row q.  Caller synchronises.
 __device__ __forceinline__ float ybuf_row_sum(const float *ybuf, int lane, int n) {
@@ -651,15 +666,20 @@ template <int NPL>
 __device__ __forceinline__ void step_any(float (&h)[NPL], const float (&dv)[NPL],
                                          const float (&bv)[NPL], uint32_t pb, uint32_t tl,
                                          int Dk, uint32_t pk, int lane) {
-    if (Dk <= 1) {
-        step_slots<NPL, 1>(h, dv, bv, pb, tl, lane);
-    } else if (Dk <= 2) {
-        step_slots<NPL, 2>(h, dv, bv, pb, tl, lane);
-    } else if (Dk <= 4) {
-        step_slots<NPL, 4>(h, dv, bv, pb, tl, lane);
-    } else if (Dk <= kDcap) {
-        step_slots<NPL, kDcap>(h, dv, bv, pb, tl, lane);
-    } else {
+    static_assert(kDcap == 8, "fan-in classes below are written for kDcap = 8");
+    switch (Dk) {
+        case 0:
+        case 1: step_slots<NPL, 1>(h, dv, bv, pb, tl, lane); return;
+        case 2: step_slots<NPL, 2>(h, dv, bv, pb, tl, lane); return;
+        case 3: step_slots<NPL, 3>(h, dv, bv, pb, tl, lane); return;
+        case 4: step_slots<NPL, 4>(h, dv, bv, pb, tl, lane); return;
+        case 5: step_slots<NPL, 5>(h, dv, bv, pb, tl, lane); return;
+        case 6: step_slots<NPL, 6>(h, dv, bv, pb, tl, lane); return;
+        case 7:
+        case kDcap: step_slots<NPL, kDcap>(h, dv, bv, pb, tl, lane); return;
+        default: break;
+    }
+    {
         constexpr int N = 32 * NPL;
         if constexpr (NPL == 1)
             sts_f32(pb + lane * 4, dv[0] * h[0]);
@@ -720,7 +740,7 @@ inline cudaError_t launch_units(KernT kern, ChunkParams p, int per_warp, cudaStr
 // ---------------------------------------------------------------------------
 cudaError_t launch_select(const pdssm_dims &dm, const void *u, pdssm_dtype ut, const float *W,
                           int32_t *k_out, cudaStream_t st);
-bool select_tc_supported(const pdssm_dims &dm, pdssm_dtype ut, const void *u);
+bool select_tc_supported(const pdssm_dims &dm, pdssm_dtype ut, const void *u, const float *W);
 bool select_tc_enabled();
 cudaError_t launch_select_tc(const pdssm_dims &dm, const void *u, const float *W, int32_t *k_out,
                              cudaStream_t st);

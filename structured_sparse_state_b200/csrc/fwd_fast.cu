@@ -91,6 +91,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA_fast(const ChunkParams 
         if (with_y) lds_own<T, NPL>(row + own_off + 2 * TENS, cv);
         int Dk = lds_s32(fan_s + kk * 4);
         uint32_t tl = tab_lane + kk * (kDcap * 64);
+#pragma unroll 2
         for (int q = 0; q < n; ++q, row += ROWB, yb += 33 * 4) {
             // transfer tracking: Delta picks up d at the column's current
             // position, then the selected map moves the column
@@ -100,11 +101,14 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA_fast(const ChunkParams 
                 pos4[r] = lds_s32(pk + pos4[r]);
             }
             step_any<NPL>(h, dv, bv, pb_s + (q & 1) * (kPbStride * 4), tl, Dk, pk, lane);
-            // next step's state-independent values
-            const int q1 = q + 1 < n ? q + 1 : q;
-            const int kk_n = __shfl_sync(kFull, kreg, q1);
+            // next step's state-independent values.  After the last step of
+            // a tile these read one row past the tile (still inside this
+            // warp's staging area: the next stage, or the buffers behind the
+            // ring) and the index held by lane n (a valid map: lanes past
+            // the tile hold 0); the values are never used.
+            const int kk_n = __shfl_sync(kFull, kreg, q + 1);
             const uint32_t pk_n = map_s + kk_n * (N * 4);
-            const uint32_t row_n = row + (q + 1 < n ? ROWB : 0);
+            const uint32_t row_n = row + ROWB;
             float dv_n[NPL], bv_n[NPL], cv_n[NPL];
             lds_own<T, NPL>(row_n + own_off, dv_n);
             lds_own<T, NPL>(row_n + own_off + TENS, bv_n);
@@ -130,8 +134,8 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA_fast(const ChunkParams 
         }
         warp_barrier();
         if (with_y) {
-            const float ys = ybuf_row_sum(ybuf, lane, n);
-            if (lane < n) p.y[seq_row0 + s + t0 + lane] = ys;
+            const float ys = ybuf_quad_sum(ybuf, lane);
+            if ((lane & 3) == 0 && (lane >> 2) < n) p.y[seq_row0 + s + t0 + (lane >> 2)] = ys;
         }
         warp_barrier();
         if (i + p.ns < ntiles)
@@ -213,7 +217,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
         const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
-        const float yold = lane < n ? yp[t0 + lane] : 0.f;
+        const float yold = ((lane & 3) == 0 && (lane >> 2) < n) ? yp[t0 + (lane >> 2)] : 0.f;
         uint32_t row = smem_u32(ring.tile(stage, 0));
         uint32_t yb = yb_lane;
 #pragma unroll 2
@@ -230,8 +234,8 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
             sts_f32(yb, acc);
         }
         warp_barrier();
-        const float ys = ybuf_row_sum(ybuf, lane, n);
-        if (lane < n) yp[t0 + lane] = yold + ys;
+        const float ys = ybuf_quad_sum(ybuf, lane);
+        if ((lane & 3) == 0 && (lane >> 2) < n) yp[t0 + (lane >> 2)] = yold + ys;
         warp_barrier();
         if (i + p.ns < ntiles)
             ring.issue(stage, s + (int64_t)(i + p.ns) * kTS, min(kTS, len - (i + p.ns) * kTS), 2,
