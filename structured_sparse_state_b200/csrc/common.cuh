@@ -37,7 +37,7 @@ enum : int { kStBadIndex = 1, kStTimeout = 2 };
 // workspace layout (all offsets 256-byte aligned)
 // ---------------------------------------------------------------------------
 struct WsLayout {
-    size_t status, dict, tab, fan, Pi, Dl, v, Hc, wc, lam, total;
+    size_t status, dict, tab, fan, seg, Pi, Dl, v, Hc, wc, lam, total;
     int64_t C, Hd;
 };
 
@@ -57,6 +57,7 @@ inline WsLayout ws_layout(const pdssm_dims &dm, int64_t pi_hs, int64_t chunk,
     w.dict = o;   o = align256(o + (size_t)(w.Hd * dm.K * dm.N) * 4);
     w.tab = o;    o = align256(o + (size_t)(w.Hd * dm.K * kDcap * 64));
     w.fan = o;    o = align256(o + (size_t)(w.Hd * dm.K) * 4);
+    w.seg = o;    o = align256(o + (size_t)(w.Hd * dm.K) * 32 * 8);
     w.Pi = o;     o = align256(o + vecs);
     w.Dl = o;     o = align256(o + vecs);
     w.v = o;      o = align256(o + vecs);
@@ -78,6 +79,9 @@ struct ChunkParams {
     const int32_t *dict;      // sanitised dictionary [Hd][K][N]
     const uint8_t *tab;       // slot tables [Hd][K][kDcap][64]: s-th source of each target
     const int32_t *fan;       // largest fan-in of each map [Hd][K]
+    const uint2 *seg;         // segment tables [Hd][K][32 lanes] (N = 32 or 64)
+    const int *seg_maxdist;   // largest lane distance inside a segment, all maps
+    int dict_content;         // parts of the dictionary staged in shared memory
     const int32_t *k;
     const void *d, *b, *c;
     const float *h0;
@@ -185,6 +189,11 @@ __device__ __forceinline__ float lds_f32(uint32_t a) {
 __device__ __forceinline__ float2 lds_f32x2(uint32_t a) {
     float2 v;
     asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds_u32x2(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
     return v;
 }
 __device__ __forceinline__ int lds_s32(uint32_t a) {
@@ -525,6 +534,65 @@ struct Ring {
     }
 };
 
+// Two-stage bulk-copy ring with compile-time geometry, for the fast-path
+// kernels (N = 32 / 64, aligned rows): tile i of a chunk goes to stage i & 1
+// and completes phase (i >> 1) & 1 of that stage's mbarrier.  NT tensors are
+// allocated per stage; the first `nt` of them are copied.
+constexpr int kFastStages = 2;
+
+__device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    return mbar_wait_bounded(bar, parity);
+}
+
+template <int NT, int ROWB>
+struct FastRing {
+    static constexpr int TENS = kTS * ROWB;
+    static constexpr int STAGEB = NT * TENS;
+    uint32_t ring_s;                  // shared address of stage 0, tensor 0
+    uint32_t bar0;                    // mbarrier of stage 0 (8 bytes each)
+    int len;                          // rows of this chunk
+    int nt;                           // tensors copied per tile
+    const unsigned char *src[NT];     // row 0 of this chunk, per tensor
+
+    __device__ uint32_t tile(int i) const { return ring_s + (uint32_t)((i & 1) * STAGEB); }
+
+    __device__ void issue(int i, int lane) const {
+        if (lane == 0) {
+            const int stage = i & 1;
+            const uint32_t bytes = (uint32_t)(min(kTS, len - i * kTS) * ROWB);
+            const uint32_t bar = bar0 + 8u * stage;
+            mbar_expect_tx(bar, bytes * (uint32_t)nt);
+#pragma unroll
+            for (int q = 0; q < NT; ++q)
+                if (q < nt)
+                    bulk_g2s(ring_s + (uint32_t)(stage * STAGEB + q * TENS),
+                             src[q] + (size_t)i * TENS, bytes, bar);
+        }
+    }
+
+    __device__ void prefetch(int i, int lane) const {
+        if (lane == 0) {
+            const uint32_t bytes = (uint32_t)(min(kTS, len - i * kTS) * ROWB);
+#pragma unroll
+            for (int q = 0; q < NT; ++q)
+                if (q < nt) bulk_prefetch_l2(src[q] + (size_t)i * TENS, bytes);
+        }
+    }
+
+    __device__ bool wait(int i) const {
+        return mbar_wait_fast(bar0 + 8u * (uint32_t)(i & 1), (uint32_t)((i >> 1) & 1));
+    }
+
+    // After a wait gave up on tile i: record it, then wait (bounded) for the
+    // copies still in flight (tiles i and i + 1) so none lands after exit.
+    __device__ void abort(int i, int ntiles, int *status, int lane) const {
+        if (lane == 0) flag_status(status, kStTimeout);
+        for (int j = i; j < ntiles && j < i + kFastStages; ++j) wait(j);
+        __syncwarp();
+    }
+};
+
 // Initialise a warp's ns mbarriers (one arrival each: the expect_tx).
 __device__ __forceinline__ void ring_init_bars(uint32_t bar0, int ns, int lane) {
     if (lane == 0) {
@@ -550,8 +618,21 @@ __device__ void ring_abort(const Ring<NT> &ring, int first, int last, int *statu
 //   warp = [staging ring][exchange buffers 2 x kPbStride floats]
 //          [readout buffer kTS x 33 floats][extra][barriers]
 constexpr int kYbufFloats = kTS * 33;
-__host__ __device__ inline int dict_slot_bytes(int K, int N) {
-    return (K * N * 4 + K * kDcap * 64 + K * 4 + 127) / 128 * 128;
+// Parts of the dictionary a kernel stages in shared memory (bit mask; 0
+// means map + slot tables).
+enum : int { kDictMap = 1, kDictTab = 2, kDictSeg = 4 };
+__host__ __device__ inline int dict_parts(int content) {
+    return content ? content : (kDictMap | kDictTab);
+}
+__host__ __device__ inline int dict_map_bytes(int K, int N) { return K * N * 4; }
+__host__ __device__ inline int dict_tab_bytes(int K) { return K * kDcap * 64 + K * 4; }
+__host__ __device__ inline int dict_seg_bytes(int K) { return K * 32 * 8; }
+__host__ __device__ inline int dict_slot_bytes(int K, int N, int content = 0) {
+    const int c = dict_parts(content);
+    int b = dict_map_bytes(K, N);
+    if (c & kDictTab) b += dict_tab_bytes(K);
+    if (c & kDictSeg) b = (b + 7) / 8 * 8 + dict_seg_bytes(K);
+    return (b + 127) / 128 * 128;
 }
 __host__ __device__ inline int warp_smem_bytes(int ns, int nt, int rowb, int extra = 0) {
     return (ns * nt * kTS * rowb + 2 * kPbStride * 4 + kYbufFloats * 4 + extra + kMaxStages * 8 +
@@ -562,20 +643,32 @@ struct SmemDict {
     const int *map;        // [K][N]
     const uint8_t *tab;    // [K][kDcap][64]
     const int *fan;        // [K]
+    const uint2 *seg;      // [K][32]
 };
 
 __device__ __forceinline__ void copy_slot(unsigned char *dst, const ChunkParams &p, int64_t dk,
                                           int tid, int nthr, int scale) {
     const int K = (int)p.K, N = (int)p.N;
+    const int c = dict_parts(p.dict_content);
     int *m = reinterpret_cast<int *>(dst);
-    uint32_t *t = reinterpret_cast<uint32_t *>(dst + K * N * 4);
-    int *f = reinterpret_cast<int *>(dst + K * N * 4 + K * kDcap * 64);
     const int32_t *gm = p.dict + dk * K * N;
-    const uint32_t *gt = reinterpret_cast<const uint32_t *>(p.tab + dk * K * kDcap * 64);
-    const int32_t *gf = p.fan + dk * K;
     for (int i = tid; i < K * N; i += nthr) m[i] = __ldg(gm + i) * scale;
-    for (int i = tid; i < K * kDcap * 16; i += nthr) t[i] = __ldg(gt + i);
-    for (int i = tid; i < K; i += nthr) f[i] = __ldg(gf + i);
+    int off = dict_map_bytes(K, N);
+    if (c & kDictTab) {
+        uint32_t *t = reinterpret_cast<uint32_t *>(dst + off);
+        int *f = reinterpret_cast<int *>(dst + off + K * kDcap * 64);
+        const uint32_t *gt = reinterpret_cast<const uint32_t *>(p.tab + dk * K * kDcap * 64);
+        const int32_t *gf = p.fan + dk * K;
+        for (int i = tid; i < K * kDcap * 16; i += nthr) t[i] = __ldg(gt + i);
+        for (int i = tid; i < K; i += nthr) f[i] = __ldg(gf + i);
+        off += dict_tab_bytes(K);
+    }
+    if (c & kDictSeg) {
+        off = (off + 7) / 8 * 8;
+        uint2 *g = reinterpret_cast<uint2 *>(dst + off);
+        const uint2 *gs = p.seg + dk * K * 32;
+        for (int i = tid; i < K * 32; i += nthr) g[i] = __ldg(gs + i);
+    }
 }
 
 // Loads the dictionary used by this CTA's warps into shared memory and
@@ -584,7 +677,8 @@ __device__ __forceinline__ void copy_slot(unsigned char *dst, const ChunkParams 
 __device__ __forceinline__ SmemDict stage_dict(const ChunkParams &p, unsigned char *smem,
                                                int warp, int lane, int scale = 1) {
     const int K = (int)p.K, N = (int)p.N;
-    const int slot = dict_slot_bytes(K, N);
+    const int c = dict_parts(p.dict_content);
+    const int slot = dict_slot_bytes(K, N, p.dict_content);
     unsigned char *mine = smem;
     if (p.dict_hs == 0) {
         copy_slot(smem, p, 0, threadIdx.x, blockDim.x, scale);
@@ -596,13 +690,21 @@ __device__ __forceinline__ SmemDict stage_dict(const ChunkParams &p, unsigned ch
     __syncthreads();
     SmemDict sd;
     sd.map = reinterpret_cast<const int *>(mine);
-    sd.tab = mine + K * N * 4;
-    sd.fan = reinterpret_cast<const int *>(mine + K * N * 4 + K * kDcap * 64);
+    int off = dict_map_bytes(K, N);
+    sd.tab = nullptr;
+    sd.fan = nullptr;
+    sd.seg = nullptr;
+    if (c & kDictTab) {
+        sd.tab = mine + off;
+        sd.fan = reinterpret_cast<const int *>(mine + off + K * kDcap * 64);
+        off += dict_tab_bytes(K);
+    }
+    if (c & kDictSeg) sd.seg = reinterpret_cast<const uint2 *>(mine + (off + 7) / 8 * 8);
     return sd;
 }
 
 __host__ __device__ inline int dict_region_bytes(const ChunkParams &p) {
-    return (p.dict_hs == 0 ? 1 : p.wpc) * dict_slot_bytes((int)p.K, (int)p.N);
+    return (p.dict_hs == 0 ? 1 : p.wpc) * dict_slot_bytes((int)p.K, (int)p.N, p.dict_content);
 }
 
 // ---------------------------------------------------------------------------
@@ -701,9 +803,73 @@ __device__ __forceinline__ void step_any(float (&h)[NPL], const float (&dv)[NPL]
     }
 }
 
+// The PD step through the map's segment table.  The sources of the step's
+// map, sorted by target (ascending j within a target), are dealt out NPL
+// per lane in order, so every target's sources form one segment of
+// consecutive entries.  Each lane loads its entries' d * h, a segmented
+// inclusive scan over the lanes (LV shuffle levels; 2^LV must exceed the
+// largest lane distance inside a segment) sums every segment, the entry
+// that ends a segment stores the sum under its target, and the owners read
+// their targets back.  The cost does not depend on the fan-in, and the sum
+// of each target follows a fixed tree, so the step is deterministic.
+//
+// Entry word e (per map and lane):
+//   e.x: byte offsets (index * 4) of source a, source b, target a, target b
+//   e.y: bits 0-7 lane distance back to the start of b's segment;
+//        bit 8 a and b share a target; bit 9 a continues the previous
+//        lane's segment; bit 10 b ends its segment; bits 11, 12 this lane's
+//        own targets (NPL e, NPL e + 1) have sources.
+// With NPL = 1 a lane holds only entry b.  pb holds d * h by element, ob the
+// segment sums by target; the two barriers keep them single-buffered.
+template <int NPL, int LV>
+__device__ __forceinline__ void step_seg(float (&h)[NPL], const float (&dv)[NPL],
+                                         const float (&bv)[NPL], uint32_t pb, uint32_t ob,
+                                         uint2 e, int lane) {
+    if constexpr (NPL == 1)
+        sts_f32(pb + lane * 4, dv[0] * h[0]);
+    else
+        sts_f32x2(pb + lane * 8, dv[0] * h[0], dv[1] * h[1]);
+    warp_barrier();
+    const uint32_t w0 = e.x, w1 = e.y;
+    const float zb = lds_f32(pb + ((w0 >> 8) & 0xffu));
+    float za = 0.f, v = zb;
+    bool ab_same = false;
+    if constexpr (NPL == 2) {
+        za = lds_f32(pb + (w0 & 0xffu));
+        ab_same = (w1 >> 8) & 1u;
+        if (ab_same) v = za + zb;
+    }
+    const int dist = (int)(w1 & 0xffu);
+#pragma unroll
+    for (int o = 1; o < (1 << LV); o <<= 1) {
+        const float t = __shfl_up_sync(kFull, v, o);
+        if (dist >= o) v = t + v;
+    }
+    if constexpr (NPL == 2) {
+        const float left = __shfl_up_sync(kFull, v, 1);
+        if (!ab_same) sts_f32(ob + ((w0 >> 16) & 0xffu), ((w1 >> 9) & 1u) ? left + za : za);
+    }
+    if ((w1 >> 10) & 1u) sts_f32(ob + (w0 >> 24), v);
+    warp_barrier();
+    if constexpr (NPL == 1) {
+        const float o0 = lds_f32(ob + lane * 4);
+        h[0] = ((w1 >> 11) & 1u ? o0 : 0.f) + bv[0];
+    } else {
+        const float2 o2 = lds_f32x2(ob + lane * 8);
+        h[0] = ((w1 >> 11) & 1u ? o2.x : 0.f) + bv[0];
+        h[1] = ((w1 >> 12) & 1u ? o2.y : 0.f) + bv[1];
+    }
+}
+
+// Shuffle levels the segment tables need: the smallest LV in {1, 2, 3, 5}
+// with 2^LV > the largest lane distance inside a segment.
+__device__ __forceinline__ int seg_levels(int maxdist) {
+    return maxdist < 2 ? 1 : maxdist < 4 ? 2 : maxdist < 8 ? 3 : 5;
+}
+
 // Warps per CTA for a chunk kernel with `per_warp` bytes of shared memory
 // per warp: 4 or 8, whichever keeps more warps resident per SM (the
-// dictionary region is paid once per CTA); assumes <= 64 registers/thread.
+// dictionary region is paid once per CTA); assumes <= 80 registers/thread.
 inline int choose_wpc(const ChunkParams &p, int per_warp) {
     const int budget = 227 * 1024;
     int best = 4, best_warps = -1;
@@ -745,6 +911,7 @@ bool select_tc_enabled();
 cudaError_t launch_select_tc(const pdssm_dims &dm, const void *u, const float *W, int32_t *k_out,
                              cudaStream_t st);
 cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
+                        uint2 *seg, int *seg_maxdist,
                         uint8_t *tab, int32_t *fan, int64_t Hd, int *status, cudaStream_t st);
 cudaError_t launch_validate(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs,
                             const int32_t *k, int *counts, cudaStream_t st);

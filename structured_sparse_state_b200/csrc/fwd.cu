@@ -238,203 +238,298 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC(const ChunkParams p) {
 
 // ---------------------------------------------------------------------------
 // phase B: one CTA of nw warps per (b, h).  Chunks are split into nw
-// contiguous segments: (1) each warp composes its segment's transfers,
-// (2) warp 0 chains the segment aggregates from h0, (3) each warp re-applies
-// its segment's transfers from its segment carry and stores every H_c.
+// contiguous segments: (1) each warp composes its segment's transfers into
+// one aggregate, (2) the aggregates are combined by an inclusive
+// Hillis-Steele scan (log2 nw rounds) and applied to h0, which gives every
+// segment's carry, (3) each warp re-applies its segment's transfers from its
+// carry and stores every H_c.
+//
+// Element layout inside a warp: lane l holds elements j = l and j = l + 32
+// (slot 1 is padding when N <= 32).  Padding elements carry index 63, factor
+// 0 and offset 0; with N < 64 no real index reaches 63, and with N = 64 there
+// is no padding, so padding never touches a stored entry.
 // ---------------------------------------------------------------------------
 
-// out = P_P diag(D) x + V for an arbitrary (composed) index map P: every
-// lane scans all N sources in ascending j (maps composed over a chunk often
-// collapse onto a few targets, so no bounded fan-in can be assumed).
-// sP, sZ are this warp's scratch rows.  x and out may alias.
-template <int NPL>
-__device__ __forceinline__ void apply_scatter(const int (&P)[NPL], const float (&D)[NPL],
-                                              const float (&V)[NPL], const float (&x)[NPL],
-                                              float (&out)[NPL], int *sP, float *sZ, int N,
-                                              int lane) {
+constexpr int kPadIdx = 63;
+
+// Per-warp scratch of the scatter (64 entries each).
+struct ScatterScratch {
+    int cnt[64];
+    int off[64];
+    int key[64];
+    float val[64];
+    float sum[64];
+};
+
+// out[i] = V[i] + sum_{j : P[j] = i} Z[j] over the warp's 64 elements, for an
+// arbitrary index map (maps composed over a chunk often send most columns to
+// one target, so no bounded fan-in is assumed).  Deterministic: the entries
+// are sorted by target (ascending j within a target, by counting ranks), and
+// each target's entries are summed by a segmented scan over the sorted
+// order, whose tree of additions depends only on the map.
+__device__ __forceinline__ void warp_scatter(const int (&P)[2], const float (&Z)[2],
+                                             const float (&V)[2], float (&out)[2],
+                                             ScatterScratch &sc, int lane) {
+    const unsigned lt = (1u << lane) - 1u;
+    const unsigned m0 = __match_any_sync(kFull, P[0]);
+    const unsigned m1 = __match_any_sync(kFull, P[1]);
+    const int r0 = __popc(m0 & lt), r1 = __popc(m1 & lt);
+    sc.cnt[lane] = 0;
+    sc.cnt[lane + 32] = 0;
+    __syncwarp();
+    if (r0 == 0) sc.cnt[P[0]] = __popc(m0);   // one writer per index
+    __syncwarp();
+    const int rank1 = sc.cnt[P[1]] + r1;       // slot-1 entries follow slot-0 ones
+    __syncwarp();
+    if (r1 == 0) sc.cnt[P[1]] += __popc(m1);
+    __syncwarp();
+    // exclusive scan of the 64 counts, bins 2 l and 2 l + 1 per lane
+    const int c0 = sc.cnt[2 * lane], c1 = sc.cnt[2 * lane + 1];
+    int incl = c0 + c1;
 #pragma unroll
-    for (int r = 0; r < NPL; ++r) {
-        const int e = lane * NPL + r;
-        if (e < N) {
-            sP[e] = P[r];
-            sZ[e] = D[r] * x[r];
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(kFull, incl, o);
+        if (lane >= o) incl += y;
+    }
+    const int ex = incl - c0 - c1;
+    sc.off[2 * lane] = ex;
+    sc.off[2 * lane + 1] = ex + c0;
+    __syncwarp();
+    const int pos0 = sc.off[P[0]] + r0, pos1 = sc.off[P[1]] + rank1;
+    sc.key[pos0] = P[0];
+    sc.val[pos0] = Z[0];
+    sc.key[pos1] = P[1];
+    sc.val[pos1] = Z[1];
+    __syncwarp();
+    // segmented inclusive scan over sorted entries 2 l, 2 l + 1
+    const int ka = sc.key[2 * lane], kb = sc.key[2 * lane + 1];
+    const float za = sc.val[2 * lane], zb = sc.val[2 * lane + 1];
+    const int kprev = __shfl_up_sync(kFull, kb, 1);     // entry 2 l - 1
+    const int knext = __shfl_down_sync(kFull, ka, 1);   // entry 2 l + 2
+    const bool joins_left = lane > 0 && kprev == ka;    // entry 2 l continues a segment
+    float sv = ka == kb ? za + zb : zb;
+    int sf = (ka != kb || !joins_left) ? 1 : 0;          // segment of 2 l + 1 starts here
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float yv = __shfl_up_sync(kFull, sv, o);
+        const int yf = __shfl_up_sync(kFull, sf, o);
+        if (lane >= o && !sf) {
+            sv = yv + sv;
+            sf = yf;
         }
     }
+    const float sprev = __shfl_up_sync(kFull, sv, 1);
+    if (ka != kb) sc.sum[ka] = joins_left ? sprev + za : za;   // entry 2 l ends a segment
+    if (lane == 31 || knext != kb) sc.sum[kb] = sv;          // entry 2 l + 1 ends a segment
     __syncwarp();
-    float acc[NPL];
 #pragma unroll
-    for (int r = 0; r < NPL; ++r) acc[r] = 0.f;
-#pragma unroll 4
-    for (int j = 0; j < N; ++j) {
-        const int pj = sP[j];
-        const float zj = sZ[j];
-#pragma unroll
-        for (int r = 0; r < NPL; ++r)
-            if (pj == lane * NPL + r) acc[r] += zj;
+    for (int r = 0; r < 2; ++r) {
+        const int i = lane + 32 * r;
+        out[r] = sc.cnt[i] > 0 ? sc.sum[i] + V[r] : V[r];
     }
     __syncwarp();
-#pragma unroll
-    for (int r = 0; r < NPL; ++r) out[r] = lane * NPL + r < N ? acc[r] + V[r] : 0.f;
 }
 
-template <int NPL>
-__device__ __forceinline__ void load_transfer(const ChunkParams &p, int64_t unit, int lane,
-                                              int (&P)[NPL], float (&D)[NPL], float (&V)[NPL]) {
+// Chunk transfer `unit` in the phase-B layout.
+__device__ __forceinline__ void load_transfer2(const ChunkParams &p, int64_t unit, int lane,
+                                               int (&P)[2], float (&D)[2], float (&V)[2]) {
     const int64_t o = unit * p.N;
 #pragma unroll
-    for (int r = 0; r < NPL; ++r) {
-        const int e = lane * NPL + r;
+    for (int r = 0; r < 2; ++r) {
+        const int e = lane + 32 * r;
         if (e < p.N) {
-            P[r] = p.Pi[o + e];
-            D[r] = p.Dl[o + e];
-            V[r] = p.v[o + e];
+            P[r] = __ldg(p.Pi + o + e);
+            D[r] = __ldg(p.Dl + o + e);
+            V[r] = __ldg(p.v + o + e);
         } else {
-            P[r] = 0;
+            P[r] = kPadIdx;
             D[r] = 0.f;
             V[r] = 0.f;
         }
     }
 }
 
-template <int NPL>
-__global__ void k_phaseB(const ChunkParams p) {
+// Aggregate (P, D, V) of a run of chunks in one warp, laid out as above.
+struct Agg {
+    int P[2];
+    float D[2], V[2];
+};
+
+// a <- T o a (a first, then T), where T's index map and factors are staged
+// in shared memory (tP, tD) for the gathers and (TP, TD, TV) are this lane's
+// entries of T.
+__device__ __forceinline__ void compose_after(Agg &a, const int *tP, const float *tD,
+                                              const int (&TP)[2], const float (&TD)[2],
+                                              const float (&TV)[2], ScatterScratch &sc,
+                                              int lane) {
+    float z[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) z[r] = TD[r] * a.V[r];
+    float nv[2];
+    warp_scatter(TP, z, TV, nv, sc, lane);
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int q = a.P[r];
+        a.D[r] = a.D[r] * tD[q];
+        a.P[r] = tP[q];
+        a.V[r] = nv[r];
+    }
+}
+
+constexpr int kBGroup = 2;   // transfers loaded together
+
+__global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p) {
     extern __shared__ __align__(16) unsigned char sm_b[];
     const int nw = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int N = (int)p.N;
     const int64_t bh = blockIdx.x;
     const int64_t C = p.C;
-    int *sPall = reinterpret_cast<int *>(sm_b);                    // [nw][64]
-    float *sZall = reinterpret_cast<float *>(sPall + nw * kMaxN);  // [nw][64]
-    float *sDall = sZall + nw * kMaxN;                             // [nw][64]
-    int *aggP = reinterpret_cast<int *>(sDall + nw * kMaxN);       // [nw][64]
-    float *aggD = reinterpret_cast<float *>(aggP + nw * kMaxN);
-    float *aggV = aggD + nw * kMaxN;
-    float *carry = aggV + nw * kMaxN;                              // [nw][64]
-    int *sP = sPall + warp * kMaxN;
-    float *sZ = sZall + warp * kMaxN;
-    float *sD = sDall + warp * kMaxN;
+    // [2 buffers][nw][64] aggregates, [nw][64] carries, [nw] scratch
+    int *aggP = reinterpret_cast<int *>(sm_b);
+    float *aggD = reinterpret_cast<float *>(aggP + 2 * nw * 64);
+    float *aggV = aggD + 2 * nw * 64;
+    float *carry = aggV + 2 * nw * 64;
+    ScatterScratch *scr = reinterpret_cast<ScatterScratch *>(carry + nw * 64);
+    ScatterScratch &sc = scr[warp];
+    // the staged chunk transfer of the level-1 gathers reuses key / val
+    int *tP = sc.key;
+    float *tD = sc.val;
 
     const int64_t c0 = C * warp / nw, c1 = C * (warp + 1) / nw;
     const int64_t u0 = bh * C;
 
-    // (1) segment aggregate: T_{c1-1} o ... o T_{c0}
-    if (c0 < c1) {
-        int aP[NPL];
-        float aD[NPL], aV[NPL];
-        load_transfer<NPL>(p, u0 + c0, lane, aP, aD, aV);
-        int P2[NPL];
-        float D2[NPL], V2[NPL];
-        if (c0 + 1 < c1) load_transfer<NPL>(p, u0 + c0 + 1, lane, P2, D2, V2);
-        for (int64_t c = c0 + 1; c < c1; ++c) {
-            int Pn[NPL];
-            float Dn[NPL], Vn[NPL];
-            if (c + 1 < c1) load_transfer<NPL>(p, u0 + c + 1, lane, Pn, Dn, Vn);
+    // (1) segment aggregate T_{c1-1} o ... o T_{c0}; identity for an empty segment
+    Agg a;
 #pragma unroll
-            for (int r = 0; r < NPL; ++r) {
-                const int e = lane * NPL + r;
-                if (e < N) {
-                    sP[e] = P2[r];
-                    sD[e] = D2[r];
-                }
+    for (int r = 0; r < 2; ++r) {
+        const int e = lane + 32 * r;
+        a.P[r] = e < p.N ? e : kPadIdx;
+        a.D[r] = e < p.N ? 1.f : 0.f;
+        a.V[r] = 0.f;
+    }
+    for (int64_t g = c0; g < c1; g += kBGroup) {
+        int TP[kBGroup][2];
+        float TD[kBGroup][2], TV[kBGroup][2];
+#pragma unroll
+        for (int i = 0; i < kBGroup; ++i)
+            if (g + i < c1) load_transfer2(p, u0 + g + i, lane, TP[i], TD[i], TV[i]);
+#pragma unroll
+        for (int i = 0; i < kBGroup; ++i) {
+            if (g + i >= c1) break;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                tP[lane + 32 * r] = TP[i][r];
+                tD[lane + 32 * r] = TD[i][r];
             }
             __syncwarp();
-            int nP[NPL];
-            float nD[NPL];
+            // the gathers read tP / tD before the scatter overwrites them
+            int gP[2];
+            float gD[2];
 #pragma unroll
-            for (int r = 0; r < NPL; ++r) {
-                nP[r] = sP[aP[r]];
-                nD[r] = aD[r] * sD[aP[r]];
+            for (int r = 0; r < 2; ++r) {
+                gP[r] = tP[a.P[r]];
+                gD[r] = tD[a.P[r]];
             }
             __syncwarp();
-            apply_scatter<NPL>(P2, D2, V2, aV, aV, sP, sZ, N, lane);
+            float z[2], nv[2];
 #pragma unroll
-            for (int r = 0; r < NPL; ++r) {
-                aP[r] = nP[r];
-                aD[r] = nD[r];
-                if (c + 1 < c1) {
-                    P2[r] = Pn[r];
-                    D2[r] = Dn[r];
-                    V2[r] = Vn[r];
-                }
+            for (int r = 0; r < 2; ++r) z[r] = TD[i][r] * a.V[r];
+            warp_scatter(TP[i], z, TV[i], nv, sc, lane);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                a.D[r] *= gD[r];
+                a.P[r] = gP[r];
+                a.V[r] = nv[r];
             }
         }
+    }
+    // (2) inclusive scan of the aggregates: after round d, warp w holds
+    // A_w o A_{w-1} o ... o A_{max(0, w - 2d + 1)}
+    int cur = 0;
 #pragma unroll
-        for (int r = 0; r < NPL; ++r) {
-            const int e = lane * NPL + r;
-            if (e < N) {
-                aggP[warp * kMaxN + e] = aP[r];
-                aggD[warp * kMaxN + e] = aD[r];
-                aggV[warp * kMaxN + e] = aV[r];
+    for (int r = 0; r < 2; ++r) {
+        const int e = lane + 32 * r;
+        aggP[(cur * nw + warp) * 64 + e] = a.P[r];
+        aggD[(cur * nw + warp) * 64 + e] = a.D[r];
+        aggV[(cur * nw + warp) * 64 + e] = a.V[r];
+    }
+    __syncthreads();
+    for (int d = 1; d < nw; d <<= 1) {
+        if (warp >= d) {
+            // this warp's aggregate goes after warp (warp - d)'s
+            const int src = (cur * nw + warp - d) * 64;
+            Agg lo;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int e = lane + 32 * r;
+                lo.P[r] = aggP[src + e];
+                lo.D[r] = aggD[src + e];
+                lo.V[r] = aggV[src + e];
             }
+            const int *hP = aggP + (cur * nw + warp) * 64;
+            const float *hD = aggD + (cur * nw + warp) * 64;
+            compose_after(lo, hP, hD, a.P, a.D, a.V, sc, lane);
+            a = lo;
+        }
+        const int nxt = cur ^ 1;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int e = lane + 32 * r;
+            aggP[(nxt * nw + warp) * 64 + e] = a.P[r];
+            aggD[(nxt * nw + warp) * 64 + e] = a.D[r];
+            aggV[(nxt * nw + warp) * 64 + e] = a.V[r];
+        }
+        cur = nxt;
+        __syncthreads();
+    }
+    // carry at the end of this warp's segment: (prefix aggregate)(h0)
+    float S[2];
+    if (p.h0) {
+        float z[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int e = lane + 32 * r;
+            z[r] = a.D[r] * (e < p.N ? p.h0[bh * p.N + e] : 0.f);
+        }
+        warp_scatter(a.P, z, a.V, S, sc, lane);
+    } else {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) S[r] = a.V[r];
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) carry[warp * 64 + lane + 32 * r] = S[r];
+    if (warp == nw - 1 && p.h_last) {
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int e = lane + 32 * r;
+            if (e < p.N) p.h_last[bh * p.N + e] = S[r];
         }
     }
     __syncthreads();
-    // (2) chain the segment aggregates
-    if (warp == 0) {
-        float S[NPL];
+    // (3) re-apply this warp's transfers from its carry-in, storing every H_c
+    float x[2];
 #pragma unroll
-        for (int r = 0; r < NPL; ++r) {
-            const int e = lane * NPL + r;
-            S[r] = (e < N && p.h0) ? p.h0[bh * p.N + e] : 0.f;
-        }
-        for (int w = 0; w < nw; ++w) {
-#pragma unroll
-            for (int r = 0; r < NPL; ++r) {
-                const int e = lane * NPL + r;
-                if (e < N) carry[w * kMaxN + e] = S[r];
-            }
-            if (C * w / nw < C * (w + 1) / nw) {
-                int P[NPL];
-                float D[NPL], V[NPL];
-#pragma unroll
-                for (int r = 0; r < NPL; ++r) {
-                    const int e = lane * NPL + r;
-                    P[r] = e < N ? aggP[w * kMaxN + e] : 0;
-                    D[r] = e < N ? aggD[w * kMaxN + e] : 0.f;
-                    V[r] = e < N ? aggV[w * kMaxN + e] : 0.f;
-                }
-                apply_scatter<NPL>(P, D, V, S, S, sP, sZ, N, lane);
-            }
-        }
-        if (p.h_last) {
-#pragma unroll
-            for (int r = 0; r < NPL; ++r) {
-                const int e = lane * NPL + r;
-                if (e < N) p.h_last[bh * p.N + e] = S[r];
-            }
-        }
+    for (int r = 0; r < 2; ++r) {
+        const int e = lane + 32 * r;
+        x[r] = warp > 0 ? carry[(warp - 1) * 64 + e] : (p.h0 && e < p.N ? p.h0[bh * p.N + e] : 0.f);
     }
-    __syncthreads();
-    // (3) fill the carries of this warp's segment
-    float x[NPL];
+    for (int64_t g = c0; g < c1; g += kBGroup) {
+        int TP[kBGroup][2];
+        float TD[kBGroup][2], TV[kBGroup][2];
 #pragma unroll
-    for (int r = 0; r < NPL; ++r) {
-        const int e = lane * NPL + r;
-        x[r] = e < N ? carry[warp * kMaxN + e] : 0.f;
-    }
-    if (c0 < c1) {
-        int P[NPL];
-        float D[NPL], V[NPL];
-        load_transfer<NPL>(p, u0 + c0, lane, P, D, V);
-        for (int64_t c = c0; c < c1; ++c) {
-            int Pn[NPL];
-            float Dn[NPL], Vn[NPL];
+        for (int i = 0; i < kBGroup; ++i)
+            if (g + i < c1) load_transfer2(p, u0 + g + i, lane, TP[i], TD[i], TV[i]);
 #pragma unroll
-            for (int r = 0; r < NPL; ++r) {
-                Pn[r] = 0;
-                Dn[r] = 0.f;
-                Vn[r] = 0.f;
-            }
-            if (c + 1 < c1) load_transfer<NPL>(p, u0 + c + 1, lane, Pn, Dn, Vn);
-            apply_scatter<NPL>(P, D, V, x, x, sP, sZ, N, lane);
+        for (int i = 0; i < kBGroup; ++i) {
+            if (g + i >= c1) break;
+            float z[2];
 #pragma unroll
-            for (int r = 0; r < NPL; ++r) {
-                const int e = lane * NPL + r;
-                if (e < N) p.Hc[(u0 + c) * p.N + e] = x[r];
-                P[r] = Pn[r];
-                D[r] = Dn[r];
-                V[r] = Vn[r];
+            for (int r = 0; r < 2; ++r) z[r] = TD[i][r] * x[r];
+            warp_scatter(TP[i], z, TV[i], x, sc, lane);
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int e = lane + 32 * r;
+                if (e < p.N) p.Hc[(u0 + g + i) * p.N + e] = x[r];
             }
         }
     }
@@ -488,20 +583,12 @@ cudaError_t launch_phaseC(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st)
 cudaError_t launch_phaseB(const ChunkParams &p, cudaStream_t st) {
     if (p.units == 0) return cudaSuccess;
     const int nw = (int)imin64(32, p.C);
-    const size_t smem = (size_t)nw * kMaxN * 4 * 7;
+    const size_t smem = (size_t)nw * 64 * 4 * 7 + (size_t)nw * sizeof(ScatterScratch);
     const int64_t BH = p.B * p.H;
-    cudaError_t e;
-    if (p.N > 32) {
-        e = cudaFuncSetAttribute(k_phaseB<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-        if (e != cudaSuccess) return e;
-        k_phaseB<2><<<(unsigned)BH, nw * 32, smem, st>>>(p);
-    } else {
-        e = cudaFuncSetAttribute(k_phaseB<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-        if (e != cudaSuccess) return e;
-        k_phaseB<1><<<(unsigned)BH, nw * 32, smem, st>>>(p);
-    }
+    cudaError_t e =
+        cudaFuncSetAttribute(k_phaseB, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_phaseB<<<(unsigned)BH, nw * 32, smem, st>>>(p);
     return cudaGetLastError();
 }
 

@@ -11,16 +11,14 @@
 
 namespace pdssm {
 
-template <typename T, int NPL>
-__global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA_fast(const ChunkParams p) {
-    extern __shared__ __align__(128) unsigned char sm_a[];
+// Phase A of one chunk (this warp's unit) with LV shuffle levels in the
+// segment-table step.
+template <typename T, int NPL, int LV>
+__device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const SmemDict &sd,
+                                                 unsigned char *wbase, int64_t unit, int lane) {
     constexpr int N = 32 * NPL;
     constexpr int ROWB = N * (int)sizeof(T);
     constexpr int TENS = kTS * ROWB;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const SmemDict sd = stage_dict(p, sm_a, warp, lane, 4);
-    const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
-    if (unit >= p.units) return;
     const int K = (int)p.K;
     const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
     const int64_t s = cidx * p.chunk;
@@ -28,35 +26,30 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA_fast(const ChunkParams 
     const bool with_y = p.y != nullptr;
     const int nt = with_y ? 3 : 2;
 
-    unsigned char *wbase = sm_a + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
-    Ring<3> ring;
-    ring.buf = wbase;
-    ring.rowb = ROWB;
-    ring.esz = (int)sizeof(T);
-    ring.tens_bytes = TENS;
-    ring.stage_bytes = 3 * TENS;
-    ring.ns = p.ns;
-    ring.bulk = p.bulk != 0;
-    float *pbuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes);
+    using RingT = FastRing<3, ROWB>;
+    float *pbuf = reinterpret_cast<float *>(wbase + kFastStages * RingT::STAGEB);
     float *ybuf = pbuf + 2 * kPbStride;
+    RingT ring;
+    ring.ring_s = smem_u32(wbase);
     ring.bar0 = smem_u32(ybuf + kYbufFloats);
-    const int64_t seq_row0 = bh * p.L;
-    ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * ROWB;
-    ring.src[1] = reinterpret_cast<const unsigned char *>(p.b) + seq_row0 * ROWB;
-    ring.src[2] = with_y ? reinterpret_cast<const unsigned char *>(p.c) + seq_row0 * ROWB
+    ring.len = len;
+    ring.nt = nt;
+    const int64_t row0 = bh * p.L + s;
+    ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + row0 * ROWB;
+    ring.src[1] = reinterpret_cast<const unsigned char *>(p.b) + row0 * ROWB;
+    ring.src[2] = with_y ? reinterpret_cast<const unsigned char *>(p.c) + row0 * ROWB
                          : ring.src[1];
-    ring_init_bars(ring.bar0, p.ns, lane);
+    ring_init_bars(ring.bar0, kFastStages, lane);
 
     const int ntiles = (len + kTS - 1) / kTS;
-    for (int i = 0; i < p.ns && i < ntiles; ++i)
-        ring.issue(i, s + (int64_t)i * kTS, min(kTS, len - i * kTS), nt, lane);
-    for (int i = p.ns; i < p.ns + kPrefetchTiles && i < ntiles; ++i)
-        ring.prefetch(s + (int64_t)i * kTS, min(kTS, len - i * kTS), nt, lane);
-    clear_pb(pbuf, lane);
+    for (int i = 0; i < kFastStages && i < ntiles; ++i) ring.issue(i, lane);
+    for (int i = kFastStages; i < kFastStages + kPrefetchTiles && i < ntiles; ++i)
+        ring.prefetch(i, lane);
 
-    const uint32_t map_s = smem_u32(sd.map), fan_s = smem_u32(sd.fan);
-    const uint32_t tab_lane = smem_u32(sd.tab) + lane * NPL;
-    const uint32_t pb_s = smem_u32(pbuf), yb_lane = smem_u32(ybuf) + lane * 4;
+    const uint32_t map_s = smem_u32(sd.map);
+    const uint32_t seg_lane = smem_u32(sd.seg) + lane * 8;
+    const uint32_t pb_s = smem_u32(pbuf), ob_s = pb_s + kPbStride * 4;
+    const uint32_t yb_lane = smem_u32(ybuf) + lane * 4;
     const uint32_t own_off = lane * NPL * (uint32_t)sizeof(T);
 
     float h[NPL], Dl[NPL];
@@ -67,30 +60,29 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA_fast(const ChunkParams 
         Dl[r] = 1.f;
         pos4[r] = (lane * NPL + r) * 4;
     }
-    const int32_t *kp = p.k + seq_row0 + s;
+    const int32_t *kp = p.k + row0;
+    float *yp = with_y ? p.y + row0 : nullptr;
     int kreg = load_k(kp, lane, lane < kTS && lane < len, K, p.status);
 
     for (int i = 0; i < ntiles; ++i) {
-        const int stage = i % p.ns;
-        if (!ring.wait(stage, (uint32_t)((i / p.ns) & 1))) {
-            ring_abort(ring, i, min(ntiles, i + p.ns), p.status, lane);
+        if (!ring.wait(i)) {
+            ring.abort(i, ntiles, p.status, lane);
             return;
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
         const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
-        uint32_t row = smem_u32(ring.tile(stage, 0));
+        uint32_t row = ring.tile(i);
         uint32_t yb = yb_lane;
         // values of step q that do not depend on the state, loaded one step
-        // ahead so their latency overlaps the previous step's gather
+        // ahead so their latency overlaps the previous step's work
         int kk = __shfl_sync(kFull, kreg, 0);
         uint32_t pk = map_s + kk * (N * 4);
         float dv[NPL], bv[NPL], cv[NPL];
         lds_own<T, NPL>(row + own_off, dv);
         lds_own<T, NPL>(row + own_off + TENS, bv);
         if (with_y) lds_own<T, NPL>(row + own_off + 2 * TENS, cv);
-        int Dk = lds_s32(fan_s + kk * 4);
-        uint32_t tl = tab_lane + kk * (kDcap * 64);
+        uint2 e = lds_u32x2(seg_lane + kk * 256);
 #pragma unroll 2
         for (int q = 0; q < n; ++q, row += ROWB, yb += 33 * 4) {
             // transfer tracking: Delta picks up d at the column's current
@@ -100,7 +92,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA_fast(const ChunkParams 
                 Dl[r] *= lds_elem<T>(row + elem_off<T>(pos4[r]));
                 pos4[r] = lds_s32(pk + pos4[r]);
             }
-            step_any<NPL>(h, dv, bv, pb_s + (q & 1) * (kPbStride * 4), tl, Dk, pk, lane);
+            step_seg<NPL, LV>(h, dv, bv, pb_s, ob_s, e, lane);
             // next step's state-independent values.  After the last step of
             // a tile these read one row past the tile (still inside this
             // warp's staging area: the next stage, or the buffers behind the
@@ -113,8 +105,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA_fast(const ChunkParams 
             lds_own<T, NPL>(row_n + own_off, dv_n);
             lds_own<T, NPL>(row_n + own_off + TENS, bv_n);
             if (with_y) lds_own<T, NPL>(row_n + own_off + 2 * TENS, cv_n);
-            const int Dk_n = lds_s32(fan_s + kk_n * 4);
-            const uint32_t tl_n = tab_lane + kk_n * (kDcap * 64);
+            const uint2 e_n = lds_u32x2(seg_lane + kk_n * 256);
             if (with_y) {
                 float ya = cv[0] * h[0];
 #pragma unroll
@@ -123,8 +114,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA_fast(const ChunkParams 
             }
             kk = kk_n;
             pk = pk_n;
-            Dk = Dk_n;
-            tl = tl_n;
+            e = e_n;
 #pragma unroll
             for (int r = 0; r < NPL; ++r) {
                 dv[r] = dv_n[r];
@@ -135,25 +125,37 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseA_fast(const ChunkParams 
         warp_barrier();
         if (with_y) {
             const float ys = ybuf_quad_sum(ybuf, lane);
-            if ((lane & 3) == 0 && (lane >> 2) < n) p.y[seq_row0 + s + t0 + (lane >> 2)] = ys;
+            if ((lane & 3) == 0 && (lane >> 2) < n) yp[t0 + (lane >> 2)] = ys;
         }
         warp_barrier();
-        if (i + p.ns < ntiles)
-            ring.issue(stage, s + (int64_t)(i + p.ns) * kTS, min(kTS, len - (i + p.ns) * kTS), nt,
-                       lane);
-        {
-            const int pf = i + p.ns + kPrefetchTiles;
-            if (pf < ntiles) ring.prefetch(s + (int64_t)pf * kTS, min(kTS, len - pf * kTS), nt, lane);
-        }
+        if (i + kFastStages < ntiles) ring.issue(i + kFastStages, lane);
+        if (i + kFastStages + kPrefetchTiles < ntiles)
+            ring.prefetch(i + kFastStages + kPrefetchTiles, lane);
         kreg = clamp_k(knext, K, p.status);
     }
     const int64_t o = unit * p.N;
 #pragma unroll
     for (int r = 0; r < NPL; ++r) {
-        const int e = lane * NPL + r;
-        p.Pi[o + e] = pos4[r] >> 2;
-        p.Dl[o + e] = Dl[r];
-        p.v[o + e] = h[r];
+        const int e2 = lane * NPL + r;
+        p.Pi[o + e2] = pos4[r] >> 2;
+        p.Dl[o + e2] = Dl[r];
+        p.v[o + e2] = h[r];
+    }
+}
+
+template <typename T, int NPL>
+__global__ void __launch_bounds__(kMaxWPC * 32, 3) k_phaseA_fast(const ChunkParams p) {
+    extern __shared__ __align__(128) unsigned char sm_a[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const SmemDict sd = stage_dict(p, sm_a, warp, lane, 4);
+    const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
+    if (unit >= p.units) return;
+    unsigned char *wbase = sm_a + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
+    switch (seg_levels(__ldg(p.seg_maxdist))) {
+        case 1: phaseA_fast_unit<T, NPL, 1>(p, sd, wbase, unit, lane); break;
+        case 2: phaseA_fast_unit<T, NPL, 2>(p, sd, wbase, unit, lane); break;
+        case 3: phaseA_fast_unit<T, NPL, 3>(p, sd, wbase, unit, lane); break;
+        default: phaseA_fast_unit<T, NPL, 5>(p, sd, wbase, unit, lane); break;
     }
 }
 
@@ -174,26 +176,23 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
     const int len = (int)imin64(p.chunk, p.L - s);
 
     unsigned char *wbase = sm_c + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
-    Ring<2> ring;
-    ring.buf = wbase;
-    ring.rowb = ROWB;
-    ring.esz = (int)sizeof(T);
-    ring.tens_bytes = TENS;
-    ring.stage_bytes = 2 * TENS;
-    ring.ns = p.ns;
-    ring.bulk = p.bulk != 0;
-    float *ybuf = reinterpret_cast<float *>(wbase + p.ns * ring.stage_bytes) + 2 * kPbStride;
+    using RingT = FastRing<2, ROWB>;
+    float *ybuf = reinterpret_cast<float *>(wbase + kFastStages * RingT::STAGEB) + 2 * kPbStride;
+    RingT ring;
+    ring.ring_s = smem_u32(wbase);
     ring.bar0 = smem_u32(ybuf + kYbufFloats);
+    ring.len = len;
+    ring.nt = 2;
     const int64_t seq_row0 = bh * p.L;
-    ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + seq_row0 * ROWB;
-    ring.src[1] = reinterpret_cast<const unsigned char *>(p.c) + seq_row0 * ROWB;
-    ring_init_bars(ring.bar0, p.ns, lane);
+    const int64_t row0 = seq_row0 + s;
+    ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + row0 * ROWB;
+    ring.src[1] = reinterpret_cast<const unsigned char *>(p.c) + row0 * ROWB;
+    ring_init_bars(ring.bar0, kFastStages, lane);
 
     const int ntiles = (len + kTS - 1) / kTS;
-    for (int i = 0; i < p.ns && i < ntiles; ++i)
-        ring.issue(i, s + (int64_t)i * kTS, min(kTS, len - i * kTS), 2, lane);
-    for (int i = p.ns; i < p.ns + kPrefetchTiles && i < ntiles; ++i)
-        ring.prefetch(s + (int64_t)i * kTS, min(kTS, len - i * kTS), 2, lane);
+    for (int i = 0; i < kFastStages && i < ntiles; ++i) ring.issue(i, lane);
+    for (int i = kFastStages; i < kFastStages + kPrefetchTiles && i < ntiles; ++i)
+        ring.prefetch(i, lane);
 
     const uint32_t map_s = smem_u32(sd.map), yb_lane = smem_u32(ybuf) + lane * 4;
     float w[NPL];
@@ -204,21 +203,20 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
         pos4[r] = e * 4;
         w[r] = cidx == 0 ? p.h0[bh * p.N + e] : p.Hc[(unit - 1) * p.N + e];
     }
-    const int32_t *kp = p.k + seq_row0 + s;
-    float *yp = p.y + seq_row0 + s;
+    const int32_t *kp = p.k + row0;
+    float *yp = p.y + row0;
     int kreg = load_k(kp, lane, lane < kTS && lane < len, K, p.status);
 
     for (int i = 0; i < ntiles; ++i) {
-        const int stage = i % p.ns;
-        if (!ring.wait(stage, (uint32_t)((i / p.ns) & 1))) {
-            ring_abort(ring, i, min(ntiles, i + p.ns), p.status, lane);
+        if (!ring.wait(i)) {
+            ring.abort(i, ntiles, p.status, lane);
             return;
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
         const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
         const float yold = ((lane & 3) == 0 && (lane >> 2) < n) ? yp[t0 + (lane >> 2)] : 0.f;
-        uint32_t row = smem_u32(ring.tile(stage, 0));
+        uint32_t row = ring.tile(i);
         uint32_t yb = yb_lane;
 #pragma unroll 2
         for (int q = 0; q < n; ++q, row += ROWB, yb += 33 * 4) {
@@ -237,13 +235,9 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
         const float ys = ybuf_quad_sum(ybuf, lane);
         if ((lane & 3) == 0 && (lane >> 2) < n) yp[t0 + (lane >> 2)] = yold + ys;
         warp_barrier();
-        if (i + p.ns < ntiles)
-            ring.issue(stage, s + (int64_t)(i + p.ns) * kTS, min(kTS, len - (i + p.ns) * kTS), 2,
-                       lane);
-        {
-            const int pf = i + p.ns + kPrefetchTiles;
-            if (pf < ntiles) ring.prefetch(s + (int64_t)pf * kTS, min(kTS, len - pf * kTS), 2, lane);
-        }
+        if (i + kFastStages < ntiles) ring.issue(i + kFastStages, lane);
+        if (i + kFastStages + kPrefetchTiles < ntiles)
+            ring.prefetch(i + kFastStages + kPrefetchTiles, lane);
         kreg = clamp_k(knext, K, p.status);
     }
 }
@@ -253,10 +247,14 @@ static cudaError_t launch_fast(KernT kern, const ChunkParams &p, size_t, cudaStr
     return launch_units(kern, p, p.smem_per_warp, st);
 }
 
-bool fast_path(const ChunkParams &p) { return p.N == 32 || p.N == 64; }
+// The fast kernels stage with bulk copies through a two-stage ring.
+bool fast_path(const ChunkParams &p) {
+    return (p.N == 32 || p.N == 64) && p.bulk && p.ns == kFastStages;
+}
 
 cudaError_t launch_phaseA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
     const int es = dt == PDSSM_BF16 ? 2 : 4;
+    p.dict_content = kDictMap | kDictSeg;
     p.smem_per_warp = warp_smem_bytes(p.ns, 3, (int)p.N * es);
     const size_t smem = 0;
     if (dt == PDSSM_BF16)
@@ -268,6 +266,7 @@ cudaError_t launch_phaseA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
 
 cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
     const int es = dt == PDSSM_BF16 ? 2 : 4;
+    p.dict_content = kDictMap;
     p.smem_per_warp = warp_smem_bytes(p.ns, 2, (int)p.N * es);
     const size_t smem = 0;
     if (dt == PDSSM_BF16)

@@ -125,11 +125,17 @@ cudaError_t launch_select(const pdssm_dims &dm, const void *u, pdssm_dtype ut, c
 //   * its largest fan-in (the number of slots a step must visit; above kDcap
 //     the kernels scan all sources instead).
 // ---------------------------------------------------------------------------
+constexpr int kPrepWarps = 4;
+
 __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *__restrict__ dict,
+                       uint2 *__restrict__ seg, int *__restrict__ seg_maxdist,
                        uint8_t *__restrict__ tab, int32_t *__restrict__ fan, int64_t nmaps,
                        int K, int N, int *status) {
-    const int lane = threadIdx.x & 31;
-    const int64_t m = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    __shared__ int s_off[kPrepWarps][65];   // first sorted entry of each target (+ total)
+    __shared__ int s_src[kPrepWarps][64];   // sorted entries: source
+    __shared__ int s_tgt[kPrepWarps][64];   // sorted entries: target
+    const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+    const int64_t m = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib;
     if (m >= nmaps) return;
     const int64_t dk = m / K, kk = m - dk * K;
     const int32_t *src = pi + dk * pi_hs + kk * N;
@@ -144,7 +150,9 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
     if (lane < N) dict[m * N + lane] = ta;
     if (lane + 32 < N) dict[m * N + lane + 32] = tb;
     __syncwarp();
-    int cnt0 = 0, cnt1 = 0;   // sources of targets lane and lane + 32
+    // slot tables (targets lane, lane + 32), entries below each target and
+    // ranks of this lane's sources among the sources of their target
+    int cnt0 = 0, cnt1 = 0, below0 = 0, below1 = 0, rank_a = 0, rank_b = 0;
     for (int j = 0; j < N; ++j) {
         const int va = __shfl_sync(kFull, ta, j & 31);
         const int vb = __shfl_sync(kFull, tb, j & 31);
@@ -156,20 +164,71 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
             if (cnt1 < kDcap) t[cnt1 * 64 + lane + 32] = (uint8_t)j;
             ++cnt1;
         }
+        below0 += tgt < lane;
+        below1 += tgt < lane + 32;
+        rank_a += (j < lane && tgt == ta);
+        rank_b += (j < lane + 32 && tgt == tb);
     }
     bad = __any_sync(kFull, bad);
     if (bad && lane == 0) flag_status(status, kStBadIndex);
     const int D = __reduce_max_sync(kFull, max(cnt0, cnt1));
     if (lane == 0) fan[m] = D;
+
+    // segment table (fast path only: N = 32 or 64)
+    if (N != 32 && N != 64) return;
+    s_off[wib][lane] = below0;
+    if (lane + 32 < N) s_off[wib][lane + 32] = below1;
+    if (lane == 0) s_off[wib][N] = N;
+    __syncwarp();
+    if (lane < N) {
+        const int pa = s_off[wib][ta] + rank_a;
+        s_src[wib][pa] = lane;
+        s_tgt[wib][pa] = ta;
+    }
+    if (lane + 32 < N) {
+        const int pb = s_off[wib][tb] + rank_b;
+        s_src[wib][pb] = lane + 32;
+        s_tgt[wib][pb] = tb;
+    }
+    __syncwarp();
+    const int npl = N / 32;
+    uint32_t w0, w1;
+    int dist;
+    if (npl == 2) {
+        const int ea = 2 * lane, eb = 2 * lane + 1;
+        const int sa = s_src[wib][ea], sb = s_src[wib][eb];
+        const int ga = s_tgt[wib][ea], gb = s_tgt[wib][eb];
+        const bool ab_same = ga == gb;
+        const bool a_cont = lane > 0 && s_tgt[wib][ea - 1] == ga;
+        const bool b_end = eb + 1 >= N || s_tgt[wib][eb + 1] != gb;
+        dist = lane - (s_off[wib][gb] >> 1);
+        const bool has0 = s_off[wib][ea + 1] > s_off[wib][ea];
+        const bool has1 = s_off[wib][eb + 1] > s_off[wib][eb];
+        w0 = (uint32_t)(sa * 4) | (uint32_t)(sb * 4) << 8 | (uint32_t)(ga * 4) << 16 |
+             (uint32_t)(gb * 4) << 24;
+        w1 = (uint32_t)dist | (ab_same ? 1u : 0u) << 8 | (a_cont ? 1u : 0u) << 9 |
+             (b_end ? 1u : 0u) << 10 | (has0 ? 1u : 0u) << 11 | (has1 ? 1u : 0u) << 12;
+    } else {
+        const int e = lane;
+        const int sb = s_src[wib][e], gb = s_tgt[wib][e];
+        const bool b_end = e + 1 >= N || s_tgt[wib][e + 1] != gb;
+        dist = lane - s_off[wib][gb];
+        const bool has0 = s_off[wib][e + 1] > s_off[wib][e];
+        w0 = (uint32_t)(sb * 4) << 8 | (uint32_t)(gb * 4) << 24;
+        w1 = (uint32_t)dist | (b_end ? 1u : 0u) << 10 | (has0 ? 1u : 0u) << 11;
+    }
+    seg[m * 32 + lane] = make_uint2(w0, w1);
+    const int md = __reduce_max_sync(kFull, dist);
+    if (lane == 0) atomicMax(seg_maxdist, md);
 }
 
 cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
+                        uint2 *seg, int *seg_maxdist,
                         uint8_t *tab, int32_t *fan, int64_t Hd, int *status, cudaStream_t st) {
     const int64_t nmaps = Hd * dm.K;
-    const int wpb = 4;
-    const int64_t grid = (nmaps + wpb - 1) / wpb;
-    k_prep<<<(unsigned)grid, 32 * wpb, 0, st>>>(pi, pi_hs, dict, tab, fan, nmaps, (int)dm.K,
-                                                (int)dm.N, status);
+    const int64_t grid = (nmaps + kPrepWarps - 1) / kPrepWarps;
+    k_prep<<<(unsigned)grid, 32 * kPrepWarps, 0, st>>>(pi, pi_hs, dict, seg, seg_maxdist, tab, fan,
+                                                       nmaps, (int)dm.K, (int)dm.N, status);
     return cudaGetLastError();
 }
 
