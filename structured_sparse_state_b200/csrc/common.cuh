@@ -191,6 +191,40 @@ __device__ __forceinline__ float2 lds_f32x2(uint32_t a) {
     asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
     return v;
 }
+// Shared loads at a compile-time byte offset from a register address.
+template <int OFF>
+__device__ __forceinline__ unsigned lds_u16_at(uint32_t a) {
+    unsigned short v;
+    asm volatile("ld.shared.u16 %0, [%1+%2];" : "=h"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF>
+__device__ __forceinline__ float lds_f32_at(uint32_t a) {
+    float v;
+    asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+// element of a staged row at byte address a + OFF, as float
+template <typename T, int OFF>
+__device__ __forceinline__ float lds_elem_at(uint32_t a) {
+    if constexpr (sizeof(T) == 4)
+        return lds_f32_at<OFF>(a);
+    else
+        return __uint_as_float(lds_u16_at<OFF>(a) << 16);
+}
+// next column position (a byte offset idx * sizeof(T)) through a map staged
+// with entries of sizeof(T) bytes
+template <typename T>
+__device__ __forceinline__ int lds_next_pos(uint32_t a) {
+    if constexpr (sizeof(T) == 4) {
+        int v;
+        asm volatile("ld.shared.s32 %0, [%1];" : "=r"(v) : "r"(a));
+        return v;
+    } else {
+        return (int)lds_u16_at<0>(a);
+    }
+}
+
 __device__ __forceinline__ uint2 lds_u32x2(uint32_t a) {
     uint2 v;
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
@@ -557,28 +591,31 @@ struct FastRing {
 
     __device__ uint32_t tile(int i) const { return ring_s + (uint32_t)((i & 1) * STAGEB); }
 
-    __device__ void issue(int i, int lane) const {
+    // Copy chunk tile ti (first ntc tensors) into stage m & 1.
+    __device__ void issue_tile(int m, int ti, int ntc, int lane) const {
         if (lane == 0) {
-            const int stage = i & 1;
-            const uint32_t bytes = (uint32_t)(min(kTS, len - i * kTS) * ROWB);
+            const int stage = m & 1;
+            const uint32_t bytes = (uint32_t)(min(kTS, len - ti * kTS) * ROWB);
             const uint32_t bar = bar0 + 8u * stage;
-            mbar_expect_tx(bar, bytes * (uint32_t)nt);
+            mbar_expect_tx(bar, bytes * (uint32_t)ntc);
 #pragma unroll
             for (int q = 0; q < NT; ++q)
-                if (q < nt)
+                if (q < ntc)
                     bulk_g2s(ring_s + (uint32_t)(stage * STAGEB + q * TENS),
-                             src[q] + (size_t)i * TENS, bytes, bar);
+                             src[q] + (size_t)ti * TENS, bytes, bar);
         }
     }
+    __device__ void issue(int i, int lane) const { issue_tile(i, i, nt, lane); }
 
-    __device__ void prefetch(int i, int lane) const {
+    __device__ void prefetch_tile(int ti, int ntc, int lane) const {
         if (lane == 0) {
-            const uint32_t bytes = (uint32_t)(min(kTS, len - i * kTS) * ROWB);
+            const uint32_t bytes = (uint32_t)(min(kTS, len - ti * kTS) * ROWB);
 #pragma unroll
             for (int q = 0; q < NT; ++q)
-                if (q < nt) bulk_prefetch_l2(src[q] + (size_t)i * TENS, bytes);
+                if (q < ntc) bulk_prefetch_l2(src[q] + (size_t)ti * TENS, bytes);
         }
     }
+    __device__ void prefetch(int i, int lane) const { prefetch_tile(i, nt, lane); }
 
     __device__ bool wait(int i) const {
         return mbar_wait_fast(bar0 + 8u * (uint32_t)(i & 1), (uint32_t)((i >> 1) & 1));
@@ -620,16 +657,19 @@ __device__ void ring_abort(const Ring<NT> &ring, int first, int last, int *statu
 constexpr int kYbufFloats = kTS * 33;
 // Parts of the dictionary a kernel stages in shared memory (bit mask; 0
 // means map + slot tables).
-enum : int { kDictMap = 1, kDictTab = 2, kDictSeg = 4 };
+// kDictMap16: the map with 2-byte entries (for bf16 rows: entry = index * 2).
+enum : int { kDictMap = 1, kDictTab = 2, kDictSeg = 4, kDictMap16 = 8 };
 __host__ __device__ inline int dict_parts(int content) {
     return content ? content : (kDictMap | kDictTab);
 }
-__host__ __device__ inline int dict_map_bytes(int K, int N) { return K * N * 4; }
+__host__ __device__ inline int dict_map_bytes(int K, int N, int content = 0) {
+    return (content & kDictMap16) ? (K * N * 2 + 7) / 8 * 8 : K * N * 4;
+}
 __host__ __device__ inline int dict_tab_bytes(int K) { return K * kDcap * 64 + K * 4; }
 __host__ __device__ inline int dict_seg_bytes(int K) { return K * 32 * 8; }
 __host__ __device__ inline int dict_slot_bytes(int K, int N, int content = 0) {
     const int c = dict_parts(content);
-    int b = dict_map_bytes(K, N);
+    int b = dict_map_bytes(K, N, c);
     if (c & kDictTab) b += dict_tab_bytes(K);
     if (c & kDictSeg) b = (b + 7) / 8 * 8 + dict_seg_bytes(K);
     return (b + 127) / 128 * 128;
@@ -640,7 +680,7 @@ __host__ __device__ inline int warp_smem_bytes(int ns, int nt, int rowb, int ext
 }
 
 struct SmemDict {
-    const int *map;        // [K][N]
+    const int *map;        // [K][N] (2-byte entries with kDictMap16)
     const uint8_t *tab;    // [K][kDcap][64]
     const int *fan;        // [K]
     const uint2 *seg;      // [K][32]
@@ -650,10 +690,15 @@ __device__ __forceinline__ void copy_slot(unsigned char *dst, const ChunkParams 
                                           int tid, int nthr, int scale) {
     const int K = (int)p.K, N = (int)p.N;
     const int c = dict_parts(p.dict_content);
-    int *m = reinterpret_cast<int *>(dst);
     const int32_t *gm = p.dict + dk * K * N;
-    for (int i = tid; i < K * N; i += nthr) m[i] = __ldg(gm + i) * scale;
-    int off = dict_map_bytes(K, N);
+    if (c & kDictMap16) {
+        uint16_t *m = reinterpret_cast<uint16_t *>(dst);
+        for (int i = tid; i < K * N; i += nthr) m[i] = (uint16_t)(__ldg(gm + i) * scale);
+    } else {
+        int *m = reinterpret_cast<int *>(dst);
+        for (int i = tid; i < K * N; i += nthr) m[i] = __ldg(gm + i) * scale;
+    }
+    int off = dict_map_bytes(K, N, c);
     if (c & kDictTab) {
         uint32_t *t = reinterpret_cast<uint32_t *>(dst + off);
         int *f = reinterpret_cast<int *>(dst + off + K * kDcap * 64);
@@ -690,7 +735,7 @@ __device__ __forceinline__ SmemDict stage_dict(const ChunkParams &p, unsigned ch
     __syncthreads();
     SmemDict sd;
     sd.map = reinterpret_cast<const int *>(mine);
-    int off = dict_map_bytes(K, N);
+    int off = dict_map_bytes(K, N, c);
     sd.tab = nullptr;
     sd.fan = nullptr;
     sd.seg = nullptr;

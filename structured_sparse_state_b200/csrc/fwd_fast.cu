@@ -52,13 +52,14 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
     const uint32_t yb_lane = smem_u32(ybuf) + lane * 4;
     const uint32_t own_off = lane * NPL * (uint32_t)sizeof(T);
 
+    constexpr int ES = (int)sizeof(T);
     float h[NPL], Dl[NPL];
-    int pos4[NPL];
+    int posb[NPL];   // column positions as byte offsets into a staged row
 #pragma unroll
     for (int r = 0; r < NPL; ++r) {
         h[r] = 0.f;
         Dl[r] = 1.f;
-        pos4[r] = (lane * NPL + r) * 4;
+        posb[r] = (lane * NPL + r) * ES;
     }
     const int32_t *kp = p.k + row0;
     float *yp = with_y ? p.y + row0 : nullptr;
@@ -77,7 +78,7 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
         // values of step q that do not depend on the state, loaded one step
         // ahead so their latency overlaps the previous step's work
         int kk = __shfl_sync(kFull, kreg, 0);
-        uint32_t pk = map_s + kk * (N * 4);
+        uint32_t pk = map_s + kk * (N * ES);
         float dv[NPL], bv[NPL], cv[NPL];
         lds_own<T, NPL>(row + own_off, dv);
         lds_own<T, NPL>(row + own_off + TENS, bv);
@@ -89,8 +90,8 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
             // position, then the selected map moves the column
 #pragma unroll
             for (int r = 0; r < NPL; ++r) {
-                Dl[r] *= lds_elem<T>(row + elem_off<T>(pos4[r]));
-                pos4[r] = lds_s32(pk + pos4[r]);
+                Dl[r] *= lds_elem_at<T, 0>(row + posb[r]);
+                posb[r] = lds_next_pos<T>(pk + posb[r]);
             }
             step_seg<NPL, LV>(h, dv, bv, pb_s, ob_s, e, lane);
             // next step's state-independent values.  After the last step of
@@ -99,7 +100,7 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
             // ring) and the index held by lane n (a valid map: lanes past
             // the tile hold 0); the values are never used.
             const int kk_n = __shfl_sync(kFull, kreg, q + 1);
-            const uint32_t pk_n = map_s + kk_n * (N * 4);
+            const uint32_t pk_n = map_s + kk_n * (N * ES);
             const uint32_t row_n = row + ROWB;
             float dv_n[NPL], bv_n[NPL], cv_n[NPL];
             lds_own<T, NPL>(row_n + own_off, dv_n);
@@ -137,7 +138,7 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
 #pragma unroll
     for (int r = 0; r < NPL; ++r) {
         const int e2 = lane * NPL + r;
-        p.Pi[o + e2] = pos4[r] >> 2;
+        p.Pi[o + e2] = posb[r] / ES;
         p.Dl[o + e2] = Dl[r];
         p.v[o + e2] = h[r];
     }
@@ -147,7 +148,7 @@ template <typename T, int NPL>
 __global__ void __launch_bounds__(kMaxWPC * 32, 3) k_phaseA_fast(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_a[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const SmemDict sd = stage_dict(p, sm_a, warp, lane, 4);
+    const SmemDict sd = stage_dict(p, sm_a, warp, lane, (int)sizeof(T));
     const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
     if (unit >= p.units) return;
     unsigned char *wbase = sm_a + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
@@ -166,7 +167,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
     constexpr int ROWB = N * (int)sizeof(T);
     constexpr int TENS = kTS * ROWB;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const SmemDict sd = stage_dict(p, sm_c, warp, lane, 4);
+    const SmemDict sd = stage_dict(p, sm_c, warp, lane, (int)sizeof(T));
     const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
     if (unit >= p.units) return;
     const int K = (int)p.K;
@@ -195,12 +196,13 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
         ring.prefetch(i, lane);
 
     const uint32_t map_s = smem_u32(sd.map), yb_lane = smem_u32(ybuf) + lane * 4;
+    constexpr int ES = (int)sizeof(T);
     float w[NPL];
-    int pos4[NPL];
+    int posb[NPL];   // column positions as byte offsets into a staged row
 #pragma unroll
     for (int r = 0; r < NPL; ++r) {
         const int e = lane * NPL + r;
-        pos4[r] = e * 4;
+        posb[r] = e * ES;
         w[r] = cidx == 0 ? p.h0[bh * p.N + e] : p.Hc[(unit - 1) * p.N + e];
     }
     const int32_t *kp = p.k + row0;
@@ -221,13 +223,13 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
 #pragma unroll 2
         for (int q = 0; q < n; ++q, row += ROWB, yb += 33 * 4) {
             const int kk = __shfl_sync(kFull, kreg, q);
-            const uint32_t pk = map_s + kk * (N * 4);
+            const uint32_t pk = map_s + kk * (N * ES);
             float acc = 0.f;
 #pragma unroll
             for (int r = 0; r < NPL; ++r) {
-                w[r] *= lds_elem<T>(row + elem_off<T>(pos4[r]));
-                pos4[r] = lds_s32(pk + pos4[r]);
-                acc = fmaf(lds_elem<T>(row + TENS + elem_off<T>(pos4[r])), w[r], acc);
+                w[r] *= lds_elem_at<T, 0>(row + posb[r]);
+                posb[r] = lds_next_pos<T>(pk + posb[r]);
+                acc = fmaf(lds_elem_at<T, TENS>(row + posb[r]), w[r], acc);
             }
             sts_f32(yb, acc);
         }
@@ -254,7 +256,7 @@ bool fast_path(const ChunkParams &p) {
 
 cudaError_t launch_phaseA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
     const int es = dt == PDSSM_BF16 ? 2 : 4;
-    p.dict_content = kDictMap | kDictSeg;
+    p.dict_content = (dt == PDSSM_BF16 ? kDictMap16 : kDictMap) | kDictSeg;
     p.smem_per_warp = warp_smem_bytes(p.ns, 3, (int)p.N * es);
     const size_t smem = 0;
     if (dt == PDSSM_BF16)
@@ -266,7 +268,7 @@ cudaError_t launch_phaseA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
 
 cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
     const int es = dt == PDSSM_BF16 ? 2 : 4;
-    p.dict_content = kDictMap;
+    p.dict_content = dt == PDSSM_BF16 ? kDictMap16 : kDictMap;
     p.smem_per_warp = warp_smem_bytes(p.ns, 2, (int)p.N * es);
     const size_t smem = 0;
     if (dt == PDSSM_BF16)
