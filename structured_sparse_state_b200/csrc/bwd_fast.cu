@@ -80,8 +80,6 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_bwdA_fast(const ChunkParams p)
     const int ntiles = (len + kTS - 1) / kTS;
     // tiles in reverse order: slot j holds chunk tile ntiles - 1 - j
     for (int j = 0; j < kFastStages && j < ntiles; ++j) ring.issue_tile(j, ntiles - 1 - j, 2, lane);
-    for (int j = kFastStages; j < kFastStages + kPrefetchTiles && j < ntiles; ++j)
-        ring.prefetch_tile(ntiles - 1 - j, 2, lane);
     const uint32_t map_s = smem_u32(sd.map), lb_s = smem_u32(lbuf);
     const uint32_t own_off = lane * NPL * (uint32_t)sizeof(T);
     const int32_t *kp = p.k + row0;
@@ -123,8 +121,6 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_bwdA_fast(const ChunkParams p)
         }
         warp_barrier();
         if (j + kFastStages < ntiles) ring.issue_tile(j + kFastStages, ntiles - 1 - (j + kFastStages), 2, lane);
-        if (j + kFastStages + kPrefetchTiles < ntiles)
-            ring.prefetch_tile(ntiles - 1 - (j + kFastStages + kPrefetchTiles), 2, lane);
         kreg = clamp_k(knext, K, p.status);
         gyreg = gynext;
     }
@@ -174,8 +170,6 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
     auto tile_of = [&](int m) { return m < ntiles ? m : 2 * ntiles - 1 - m; };
     auto nt_of = [&](int m) { return m < ntiles ? 2 : 3; };
     for (int m = 0; m < kFastStages && m < total; ++m) ring.issue_tile(m, tile_of(m), nt_of(m), lane);
-    for (int m = kFastStages; m < kFastStages + kPrefetchTiles && m < ntiles; ++m)
-        ring.prefetch_tile(m, 3, lane);
 
     const uint32_t map_s = smem_u32(sd.map);
     const uint32_t seg_lane = smem_u32(sd.seg) + lane * 8;
@@ -276,8 +270,6 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
             const int mn = m + kFastStages;
             ring.issue_tile(mn, tile_of(mn), nt_of(mn), lane);
         }
-        if (m + kFastStages + kPrefetchTiles < ntiles)
-            ring.prefetch_tile(m + kFastStages + kPrefetchTiles, 3, lane);
         kreg = clamp_k(knext, K, p.status);
         gyreg = gynext;
     }

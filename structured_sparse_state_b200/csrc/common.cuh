@@ -11,6 +11,7 @@
 
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
+#include <mutex>
 #include <stdint.h>
 
 #include <type_traits>
@@ -571,7 +572,8 @@ struct Ring {
 // Two-stage bulk-copy ring with compile-time geometry, for the fast-path
 // kernels (N = 32 / 64, aligned rows): tile i of a chunk goes to stage i & 1
 // and completes phase (i >> 1) & 1 of that stage's mbarrier.  NT tensors are
-// allocated per stage; the first `nt` of them are copied.
+// allocated per stage; the first `nt` of them are copied.  (No L2 prefetch
+// ahead of the ring: with many warps per SM in flight it measured slower.)
 constexpr int kFastStages = 2;
 
 __device__ __forceinline__ bool mbar_wait_fast(uint32_t bar, uint32_t parity) {
@@ -606,16 +608,6 @@ struct FastRing {
         }
     }
     __device__ void issue(int i, int lane) const { issue_tile(i, i, nt, lane); }
-
-    __device__ void prefetch_tile(int ti, int ntc, int lane) const {
-        if (lane == 0) {
-            const uint32_t bytes = (uint32_t)(min(kTS, len - ti * kTS) * ROWB);
-#pragma unroll
-            for (int q = 0; q < NT; ++q)
-                if (q < ntc) bulk_prefetch_l2(src[q] + (size_t)ti * TENS, bytes);
-        }
-    }
-    __device__ void prefetch(int i, int lane) const { prefetch_tile(i, nt, lane); }
 
     __device__ bool wait(int i) const {
         return mbar_wait_fast(bar0 + 8u * (uint32_t)(i & 1), (uint32_t)((i >> 1) & 1));
@@ -865,15 +857,21 @@ __device__ __forceinline__ void step_any(float (&h)[NPL], const float (&dv)[NPL]
 //        lane's segment; bit 10 b ends its segment; bits 11, 12 this lane's
 //        own targets (NPL e, NPL e + 1) have sources.
 // With NPL = 1 a lane holds only entry b.  pb holds d * h by element, ob the
-// segment sums by target; the two barriers keep them single-buffered.
+// segment sums by target (zero for targets without sources); the two
+// barriers keep them single-buffered.
 template <int NPL, int LV>
 __device__ __forceinline__ void step_seg(float (&h)[NPL], const float (&dv)[NPL],
                                          const float (&bv)[NPL], uint32_t pb, uint32_t ob,
                                          uint2 e, int lane) {
-    if constexpr (NPL == 1)
+    // d * h by element, and zero sums for this lane's own targets (targets
+    // without sources keep them)
+    if constexpr (NPL == 1) {
         sts_f32(pb + lane * 4, dv[0] * h[0]);
-    else
+        sts_f32(ob + lane * 4, 0.f);
+    } else {
         sts_f32x2(pb + lane * 8, dv[0] * h[0], dv[1] * h[1]);
+        sts_f32x2(ob + lane * 8, 0.f, 0.f);
+    }
     warp_barrier();
     const uint32_t w0 = e.x, w1 = e.y;
     const float zb = lds_f32(pb + ((w0 >> 8) & 0xffu));
@@ -897,12 +895,11 @@ __device__ __forceinline__ void step_seg(float (&h)[NPL], const float (&dv)[NPL]
     if ((w1 >> 10) & 1u) sts_f32(ob + (w0 >> 24), v);
     warp_barrier();
     if constexpr (NPL == 1) {
-        const float o0 = lds_f32(ob + lane * 4);
-        h[0] = ((w1 >> 11) & 1u ? o0 : 0.f) + bv[0];
+        h[0] = lds_f32(ob + lane * 4) + bv[0];
     } else {
         const float2 o2 = lds_f32x2(ob + lane * 8);
-        h[0] = ((w1 >> 11) & 1u ? o2.x : 0.f) + bv[0];
-        h[1] = ((w1 >> 12) & 1u ? o2.y : 0.f) + bv[1];
+        h[0] = o2.x + bv[0];
+        h[1] = o2.y + bv[1];
     }
 }
 
@@ -913,30 +910,58 @@ __device__ __forceinline__ int seg_levels(int maxdist) {
 }
 
 // Warps per CTA for a chunk kernel with `per_warp` bytes of shared memory
-// per warp: 4 or 8, whichever keeps more warps resident per SM (the
-// dictionary region is paid once per CTA); assumes <= 80 registers/thread.
-inline int choose_wpc(const ChunkParams &p, int per_warp) {
+// per warp: 4 or 8, whichever keeps more warps resident per SM by the
+// runtime's occupancy calculation (registers, shared memory with the
+// dictionary region paid once per CTA, and the per-SM limits).  Answers are
+// cached per (kernel, shared-memory sizes).
+struct WpcCacheEntry {
+    const void *kern;
+    int per_warp, dict_bytes, wpc;
+};
+
+template <typename KernT>
+inline int choose_wpc(KernT kern, const ChunkParams &p, int per_warp) {
+    static WpcCacheEntry cache[64];
+    static int used = 0;
+    static std::mutex mu;
+    const void *key = reinterpret_cast<const void *>(kern);
+    ChunkParams q = p;
+    q.wpc = 4;
+    const int dict4 = dict_region_bytes(q);
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        for (int i = 0; i < used; ++i)
+            if (cache[i].kern == key && cache[i].per_warp == per_warp &&
+                cache[i].dict_bytes == dict4)
+                return cache[i].wpc;
+    }
     const int budget = 227 * 1024;
     int best = 4, best_warps = -1;
     for (int wpc = 4; wpc <= kMaxWPC; wpc *= 2) {
-        ChunkParams q = p;
         q.wpc = wpc;
-        const int cta = dict_region_bytes(q) + wpc * per_warp + 1024;
-        if (cta > budget) continue;
-        int warps = (228 * 1024 / cta) * wpc;
-        warps = warps > 32 ? 32 : warps;
-        if (warps >= best_warps) {
-            best_warps = warps;
+        const int smem = dict_region_bytes(q) + wpc * per_warp;
+        if (smem > budget) continue;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+            continue;
+        int blocks = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&blocks, kern, wpc * 32, smem) !=
+            cudaSuccess)
+            continue;
+        if (blocks * wpc >= best_warps) {
+            best_warps = blocks * wpc;
             best = wpc;
         }
     }
+    std::lock_guard<std::mutex> lock(mu);
+    if (used < 64) cache[used++] = WpcCacheEntry{key, per_warp, dict4, best};
     return best;
 }
 
 template <typename KernT>
 inline cudaError_t launch_units(KernT kern, ChunkParams p, int per_warp, cudaStream_t st) {
     p.smem_per_warp = per_warp;
-    p.wpc = choose_wpc(p, per_warp);
+    p.wpc = choose_wpc(kern, p, per_warp);
     const size_t smem = (size_t)dict_region_bytes(p) + (size_t)p.wpc * per_warp;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

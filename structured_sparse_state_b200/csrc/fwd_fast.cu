@@ -43,8 +43,6 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
 
     const int ntiles = (len + kTS - 1) / kTS;
     for (int i = 0; i < kFastStages && i < ntiles; ++i) ring.issue(i, lane);
-    for (int i = kFastStages; i < kFastStages + kPrefetchTiles && i < ntiles; ++i)
-        ring.prefetch(i, lane);
 
     const uint32_t map_s = smem_u32(sd.map);
     const uint32_t seg_lane = smem_u32(sd.seg) + lane * 8;
@@ -130,8 +128,6 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
         }
         warp_barrier();
         if (i + kFastStages < ntiles) ring.issue(i + kFastStages, lane);
-        if (i + kFastStages + kPrefetchTiles < ntiles)
-            ring.prefetch(i + kFastStages + kPrefetchTiles, lane);
         kreg = clamp_k(knext, K, p.status);
     }
     const int64_t o = unit * p.N;
@@ -192,8 +188,6 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
 
     const int ntiles = (len + kTS - 1) / kTS;
     for (int i = 0; i < kFastStages && i < ntiles; ++i) ring.issue(i, lane);
-    for (int i = kFastStages; i < kFastStages + kPrefetchTiles && i < ntiles; ++i)
-        ring.prefetch(i, lane);
 
     const uint32_t map_s = smem_u32(sd.map), yb_lane = smem_u32(ybuf) + lane * 4;
     constexpr int ES = (int)sizeof(T);
@@ -238,8 +232,6 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
         if ((lane & 3) == 0 && (lane >> 2) < n) yp[t0 + (lane >> 2)] = yold + ys;
         warp_barrier();
         if (i + kFastStages < ntiles) ring.issue(i + kFastStages, lane);
-        if (i + kFastStages + kPrefetchTiles < ntiles)
-            ring.prefetch(i + kFastStages + kPrefetchTiles, lane);
         kreg = clamp_k(knext, K, p.status);
     }
 }
