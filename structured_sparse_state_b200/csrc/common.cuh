@@ -15,6 +15,7 @@
 #include <stdint.h>
 
 #include <type_traits>
+#include <utility>
 
 #include "../../include/pdssm.h"
 
@@ -134,6 +135,9 @@ __device__ __forceinline__ void fence_mbar_init() {
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
 __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar),
                  "r"(bytes)
@@ -283,6 +287,41 @@ template <>
 __device__ __forceinline__ float2 lds_pair<__nv_bfloat16>(uint32_t a) {
     const unsigned w = lds_u32(a);
     return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+
+// The same loads and stores at a compile-time byte offset from a register
+// address (for fully unrolled tiles).
+template <int OFF>
+__device__ __forceinline__ unsigned lds_u32_at(uint32_t a) {
+    unsigned v;
+    asm volatile("ld.shared.u32 %0, [%1+%2];" : "=r"(v) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF>
+__device__ __forceinline__ float2 lds_f32x2_at(uint32_t a) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2+%3];" : "=f"(v.x), "=f"(v.y) : "r"(a), "n"(OFF));
+    return v;
+}
+template <int OFF>
+__device__ __forceinline__ void sts_f32_at(uint32_t a, float v) {
+    asm volatile("st.shared.f32 [%0+%1], %2;" ::"r"(a), "n"(OFF), "f"(v) : "memory");
+}
+template <typename T, int OFF>
+__device__ __forceinline__ float2 lds_pair_at(uint32_t a) {
+    if constexpr (sizeof(T) == 4) {
+        return lds_f32x2_at<OFF>(a);
+    } else {
+        const unsigned w = lds_u32_at<OFF>(a);
+        return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+    }
+}
+
+// Calls f(std::integral_constant<int, Q>) for Q = 0 .. sizeof...(Qs) - 1 in
+// order (a loop unrolled at compile time).
+template <typename F, int... Qs>
+__device__ __forceinline__ void for_each_q(F &&f, std::integer_sequence<int, Qs...>) {
+    (f(std::integral_constant<int, Qs>{}), ...);
 }
 
 // Reduce-scatter of 16 per-lane partials: lane l (and l + 16) returns
@@ -753,6 +792,17 @@ __device__ __forceinline__ void lds_own(uint32_t a, float (&v)[NPL]) {
         v[0] = lds_elem<T>(a);
     } else {
         const float2 q = lds_pair<T>(a);
+        v[0] = q.x;
+        v[1] = q.y;
+    }
+}
+
+template <typename T, int NPL, int OFF>
+__device__ __forceinline__ void lds_own_at(uint32_t a, float (&v)[NPL]) {
+    if constexpr (NPL == 1) {
+        v[0] = lds_elem_at<T, OFF>(a);
+    } else {
+        const float2 q = lds_pair_at<T, OFF>(a);
         v[0] = q.x;
         v[1] = q.y;
     }

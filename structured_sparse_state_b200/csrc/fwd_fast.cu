@@ -71,47 +71,33 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
         const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
-        uint32_t row = ring.tile(i);
-        uint32_t yb = yb_lane;
+        const uint32_t row0s = ring.tile(i);
         // values of step q that do not depend on the state, loaded one step
         // ahead so their latency overlaps the previous step's work
         int kk = __shfl_sync(kFull, kreg, 0);
         uint32_t pk = map_s + kk * (N * ES);
         float dv[NPL], bv[NPL], cv[NPL];
-        lds_own<T, NPL>(row + own_off, dv);
-        lds_own<T, NPL>(row + own_off + TENS, bv);
-        if (with_y) lds_own<T, NPL>(row + own_off + 2 * TENS, cv);
+        lds_own<T, NPL>(row0s + own_off, dv);
+        lds_own<T, NPL>(row0s + own_off + TENS, bv);
+        if (with_y) lds_own<T, NPL>(row0s + own_off + 2 * TENS, cv);
         uint2 e = lds_u32x2(seg_lane + kk * 256);
-#pragma unroll 2
-        for (int q = 0; q < n; ++q, row += ROWB, yb += 33 * 4) {
-            // transfer tracking: Delta picks up d at the column's current
-            // position, then the selected map moves the column
-#pragma unroll
-            for (int r = 0; r < NPL; ++r) {
-                Dl[r] *= lds_elem_at<T, 0>(row + posb[r]);
-                posb[r] = lds_next_pos<T>(pk + posb[r]);
-            }
-            step_seg<NPL, LV>(h, dv, bv, pb_s, ob_s, e, lane);
-            // next step's state-independent values.  After the last step of
-            // a tile these read one row past the tile (still inside this
-            // warp's staging area: the next stage, or the buffers behind the
-            // ring) and the index held by lane n (a valid map: lanes past
-            // the tile hold 0); the values are never used.
-            const int kk_n = __shfl_sync(kFull, kreg, q + 1);
-            const uint32_t pk_n = map_s + kk_n * (N * ES);
-            const uint32_t row_n = row + ROWB;
-            float dv_n[NPL], bv_n[NPL], cv_n[NPL];
-            lds_own<T, NPL>(row_n + own_off, dv_n);
-            lds_own<T, NPL>(row_n + own_off + TENS, bv_n);
-            if (with_y) lds_own<T, NPL>(row_n + own_off + 2 * TENS, cv_n);
-            const uint2 e_n = lds_u32x2(seg_lane + kk_n * 256);
+        // One step: transfer tracking (Delta picks up d at the column's
+        // current position, then the selected map moves the column), the PD
+        // step, the next step's state-independent values, the readout
+        // partial.  After the last step of a tile the next-step loads read one
+        // row past the tile (still inside this warp's staging area: the next
+        // stage, or the buffers behind the ring) and the index held by lane n
+        // (a valid map: lanes past the tile hold 0); they are never used.
+        auto finish_step = [&](int q_next, const float (&dv_n)[NPL], const float (&bv_n)[NPL],
+                               const float (&cv_n)[NPL], uint2 e_n, uint32_t pk_n,
+                               uint32_t yb_addr) {
             if (with_y) {
                 float ya = cv[0] * h[0];
 #pragma unroll
                 for (int r = 1; r < NPL; ++r) ya = fmaf(cv[r], h[r], ya);
-                sts_f32(yb, ya);
+                sts_f32(yb_addr, ya);
             }
-            kk = kk_n;
+            (void)q_next;
             pk = pk_n;
             e = e_n;
 #pragma unroll
@@ -119,6 +105,47 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
                 dv[r] = dv_n[r];
                 bv[r] = bv_n[r];
                 cv[r] = cv_n[r];
+            }
+        };
+        if (n == kTS) {
+            // full tile: steps unrolled, row and readout offsets immediate
+            for_each_q(
+                [&](auto qc) {
+                    constexpr int Q = decltype(qc)::value;
+#pragma unroll
+                    for (int r = 0; r < NPL; ++r) {
+                        Dl[r] *= lds_elem_at<T, Q * ROWB>(row0s + posb[r]);
+                        posb[r] = lds_next_pos<T>(pk + posb[r]);
+                    }
+                    step_seg<NPL, LV>(h, dv, bv, pb_s, ob_s, e, lane);
+                    const int kk_n = __shfl_sync(kFull, kreg, Q + 1);
+                    float dv_n[NPL], bv_n[NPL], cv_n[NPL];
+                    lds_own_at<T, NPL, (Q + 1) * ROWB>(row0s + own_off, dv_n);
+                    lds_own_at<T, NPL, (Q + 1) * ROWB + TENS>(row0s + own_off, bv_n);
+                    if (with_y) lds_own_at<T, NPL, (Q + 1) * ROWB + 2 * TENS>(row0s + own_off, cv_n);
+                    const uint2 e_n = lds_u32x2(seg_lane + kk_n * 256);
+                    finish_step(Q + 1, dv_n, bv_n, cv_n, e_n, map_s + kk_n * (N * ES),
+                                yb_lane + Q * 33 * 4);
+                },
+                std::make_integer_sequence<int, kTS>{});
+        } else {
+            uint32_t row = row0s;
+            for (int q = 0; q < n; ++q, row += ROWB) {
+#pragma unroll
+                for (int r = 0; r < NPL; ++r) {
+                    Dl[r] *= lds_elem_at<T, 0>(row + posb[r]);
+                    posb[r] = lds_next_pos<T>(pk + posb[r]);
+                }
+                step_seg<NPL, LV>(h, dv, bv, pb_s, ob_s, e, lane);
+                const int kk_n = __shfl_sync(kFull, kreg, q + 1);
+                const uint32_t row_n = row + ROWB;
+                float dv_n[NPL], bv_n[NPL], cv_n[NPL];
+                lds_own<T, NPL>(row_n + own_off, dv_n);
+                lds_own<T, NPL>(row_n + own_off + TENS, bv_n);
+                if (with_y) lds_own<T, NPL>(row_n + own_off + 2 * TENS, cv_n);
+                const uint2 e_n = lds_u32x2(seg_lane + kk_n * 256);
+                finish_step(q + 1, dv_n, bv_n, cv_n, e_n, map_s + kk_n * (N * ES),
+                            yb_lane + q * 33 * 4);
             }
         }
         warp_barrier();
@@ -212,20 +239,39 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
         const int n = min(kTS, len - t0);
         const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
         const float yold = ((lane & 3) == 0 && (lane >> 2) < n) ? yp[t0 + (lane >> 2)] : 0.f;
-        uint32_t row = ring.tile(i);
-        uint32_t yb = yb_lane;
-#pragma unroll 2
-        for (int q = 0; q < n; ++q, row += ROWB, yb += 33 * 4) {
-            const int kk = __shfl_sync(kFull, kreg, q);
-            const uint32_t pk = map_s + kk * (N * ES);
-            float acc = 0.f;
+        const uint32_t row0s = ring.tile(i);
+        if (n == kTS) {
+            // full tile: steps unrolled, row and readout offsets immediate
+            for_each_q(
+                [&](auto qc) {
+                    constexpr int Q = decltype(qc)::value;
+                    const int kk = __shfl_sync(kFull, kreg, Q);
+                    const uint32_t pk = map_s + kk * (N * ES);
+                    float acc = 0.f;
 #pragma unroll
-            for (int r = 0; r < NPL; ++r) {
-                w[r] *= lds_elem_at<T, 0>(row + posb[r]);
-                posb[r] = lds_next_pos<T>(pk + posb[r]);
-                acc = fmaf(lds_elem_at<T, TENS>(row + posb[r]), w[r], acc);
+                    for (int r = 0; r < NPL; ++r) {
+                        w[r] *= lds_elem_at<T, Q * ROWB>(row0s + posb[r]);
+                        posb[r] = lds_next_pos<T>(pk + posb[r]);
+                        acc = fmaf(lds_elem_at<T, Q * ROWB + TENS>(row0s + posb[r]), w[r], acc);
+                    }
+                    sts_f32_at<Q * 33 * 4>(yb_lane, acc);
+                },
+                std::make_integer_sequence<int, kTS>{});
+        } else {
+            uint32_t row = row0s;
+            uint32_t yb = yb_lane;
+            for (int q = 0; q < n; ++q, row += ROWB, yb += 33 * 4) {
+                const int kk = __shfl_sync(kFull, kreg, q);
+                const uint32_t pk = map_s + kk * (N * ES);
+                float acc = 0.f;
+#pragma unroll
+                for (int r = 0; r < NPL; ++r) {
+                    w[r] *= lds_elem_at<T, 0>(row + posb[r]);
+                    posb[r] = lds_next_pos<T>(pk + posb[r]);
+                    acc = fmaf(lds_elem_at<T, TENS>(row + posb[r]), w[r], acc);
+                }
+                sts_f32(yb, acc);
             }
-            sts_f32(yb, acc);
         }
         warp_barrier();
         const float ys = ybuf_quad_sum(ybuf, lane);
