@@ -168,7 +168,8 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
 }
 
 template <typename T, int NPL>
-__global__ void __launch_bounds__(kMaxWPC * 32, 3) k_phaseA_fast(const ChunkParams p) {
+__global__ void __launch_bounds__(kMaxWPC * 32, (sizeof(T) == 4 && NPL == 2) ? 2 : 3)
+    k_phaseA_fast(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_a[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const SmemDict sd = stage_dict(p, sm_a, warp, lane, (int)sizeof(T));

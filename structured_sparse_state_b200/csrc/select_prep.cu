@@ -134,6 +134,8 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
     __shared__ int s_off[kPrepWarps][65];   // first sorted entry of each target (+ total)
     __shared__ int s_src[kPrepWarps][64];   // sorted entries: source
     __shared__ int s_tgt[kPrepWarps][64];   // sorted entries: target
+    __shared__ int s_cnt0[kPrepWarps][64];  // sources of each target among j < 32
+    __shared__ int s_cnt[kPrepWarps][64];   // sources of each target
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int64_t m = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib;
     if (m >= nmaps) return;
@@ -150,25 +152,43 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
     if (lane < N) dict[m * N + lane] = ta;
     if (lane + 32 < N) dict[m * N + lane + 32] = tb;
     __syncwarp();
-    // slot tables (targets lane, lane + 32), entries below each target and
-    // ranks of this lane's sources among the sources of their target
-    int cnt0 = 0, cnt1 = 0, below0 = 0, below1 = 0, rank_a = 0, rank_b = 0;
-    for (int j = 0; j < N; ++j) {
-        const int va = __shfl_sync(kFull, ta, j & 31);
-        const int vb = __shfl_sync(kFull, tb, j & 31);
-        const int tgt = j < 32 ? va : vb;
-        if (tgt == lane) {
-            if (cnt0 < kDcap) t[cnt0 * 64 + lane] = (uint8_t)j;
-            ++cnt0;
-        } else if (tgt == lane + 32) {
-            if (cnt1 < kDcap) t[cnt1 * 64 + lane + 32] = (uint8_t)j;
-            ++cnt1;
+    // Ranks of this lane's sources among the sources of their target
+    // (ascending j): sources j = lane first, then j = lane + 32.  Lanes past N
+    // carry keys no real target has.
+    const unsigned lt = (1u << lane) - 1u;
+    const int key_a = lane < N ? ta : 64 + lane;
+    const int key_b = lane + 32 < N ? tb : 128 + lane;
+    const unsigned m_a = __match_any_sync(kFull, key_a);
+    const unsigned m_b = __match_any_sync(kFull, key_b);
+    s_cnt0[wib][lane] = 0;
+    s_cnt0[wib][lane + 32] = 0;
+    s_cnt[wib][lane] = 0;
+    s_cnt[wib][lane + 32] = 0;
+    __syncwarp();
+    if (lane < N && (m_a & lt) == 0) s_cnt0[wib][ta] = __popc(m_a);   // one writer per target
+    __syncwarp();
+    const int rank_a = __popc(m_a & lt);
+    const int rank_b = lane + 32 < N ? s_cnt0[wib][tb] + __popc(m_b & lt) : 0;
+    if (lane < N && (m_a & lt) == 0) s_cnt[wib][ta] = __popc(m_a);
+    __syncwarp();
+    if (lane + 32 < N && (m_b & lt) == 0) s_cnt[wib][tb] += __popc(m_b);
+    __syncwarp();
+    const int cnt0 = s_cnt[wib][lane], cnt1 = s_cnt[wib][lane + 32];   // fan-in of targets lane, lane + 32
+    // slot tables: the r-th source of target t at t[r * 64 + t]
+    if (lane < N && rank_a < kDcap) t[rank_a * 64 + ta] = (uint8_t)lane;
+    if (lane + 32 < N && rank_b < kDcap) t[rank_b * 64 + tb] = (uint8_t)(lane + 32);
+    // entries below each target: exclusive scan of the counts
+    int inc0 = cnt0, inc1 = cnt1;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y0 = __shfl_up_sync(kFull, inc0, o), y1 = __shfl_up_sync(kFull, inc1, o);
+        if (lane >= o) {
+            inc0 += y0;
+            inc1 += y1;
         }
-        below0 += tgt < lane;
-        below1 += tgt < lane + 32;
-        rank_a += (j < lane && tgt == ta);
-        rank_b += (j < lane + 32 && tgt == tb);
     }
+    const int total0 = __shfl_sync(kFull, inc0, 31);
+    const int below0 = inc0 - cnt0, below1 = total0 + inc1 - cnt1;
     bad = __any_sync(kFull, bad);
     if (bad && lane == 0) flag_status(status, kStBadIndex);
     const int D = __reduce_max_sync(kFull, max(cnt0, cnt1));
