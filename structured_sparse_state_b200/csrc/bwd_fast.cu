@@ -51,7 +51,8 @@ __device__ __forceinline__ void stg_own(float *row, int lane, const float (&v)[N
 // ---------------------------------------------------------------------------
 template <typename T, int NPL>
 __global__ void __launch_bounds__(kMaxWPC * 32) k_bwdA_fast(const ChunkParams p) {
-    extern __shared__ __align__(128) unsigned char sm_ba[];
+    extern __shared__ __align__(128) unsigned char sm_ba_raw[];
+    unsigned char *sm_ba = smem_base256(sm_ba_raw);
     constexpr int N = 32 * NPL;
     constexpr int ROWB = N * (int)sizeof(T);
     constexpr int TENS = kTS * ROWB;
@@ -173,7 +174,7 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
 
     const uint32_t map_s = smem_u32(sd.map);
     const uint32_t seg_lane = smem_u32(sd.seg) + lane * 8;
-    const uint32_t pb_s = smem_u32(pbuf), ob_s = pb_s + kPbStride * 4, lb_s = smem_u32(lbuf);
+    const uint32_t pb_s = smem_u32(pbuf), ob_s = pb_s + 256, lb_s = smem_u32(lbuf);   // pb, ob 256-byte aligned
     const uint32_t hs_lane = smem_u32(hsm) + lane * NPL * 4;
     const uint32_t own_off = lane * NPL * (uint32_t)sizeof(T);
     const int32_t *kp = p.k + row0;
@@ -277,7 +278,8 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
 
 template <typename T, int NPL>
 __global__ void __launch_bounds__(kMaxWPC * 32, 3) k_bwdC_fast(const ChunkParams p) {
-    extern __shared__ __align__(128) unsigned char sm_bc[];
+    extern __shared__ __align__(128) unsigned char sm_bc_raw[];
+    unsigned char *sm_bc = smem_base256(sm_bc_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const SmemDict sd = stage_dict(p, sm_bc, warp, lane, 4);
     const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
@@ -311,7 +313,9 @@ cudaError_t launch_bwdA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
 cudaError_t launch_bwdC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
     const int es = dt == PDSSM_BF16 ? 2 : 4;
     p.dict_content = kDictMap | kDictSeg;
-    p.smem_per_warp = warp_smem_bytes(kFastStages, 3, (int)p.N * es, kBwdFastExtraFloats * 4);
+    // ring, exchange buffers pb / ob and lbuf, the tile's states, barriers
+    p.smem_per_warp = (kFastStages * 3 * kTS * (int)p.N * es + kBwdFastExtraFloats * 4 +
+                       2 * kPbStride * 4 + kFastStages * 8 + 255) / 256 * 256;
     const size_t smem = 0;
     if (dt == PDSSM_BF16)
         return p.N == 64 ? launch_bfast(k_bwdC_fast<__nv_bfloat16, 2>, p, smem, st)

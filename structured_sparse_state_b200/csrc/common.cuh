@@ -703,11 +703,18 @@ __host__ __device__ inline int dict_slot_bytes(int K, int N, int content = 0) {
     int b = dict_map_bytes(K, N, c);
     if (c & kDictTab) b += dict_tab_bytes(K);
     if (c & kDictSeg) b = (b + 7) / 8 * 8 + dict_seg_bytes(K);
-    return (b + 127) / 128 * 128;
+    return (b + 255) / 256 * 256;
 }
 __host__ __device__ inline int warp_smem_bytes(int ns, int nt, int rowb, int extra = 0) {
     return (ns * nt * kTS * rowb + 2 * kPbStride * 4 + kYbufFloats * 4 + extra + kMaxStages * 8 +
-            127) / 128 * 128;
+            255) / 256 * 256;
+}
+// The dynamic shared memory of the chunk kernels, rounded up to 256 bytes
+// (launches add 256 bytes of slack), so that the per-warp regions, whose
+// sizes are multiples of 256, start 256-byte aligned.
+__device__ __forceinline__ unsigned char *smem_base256(unsigned char *raw) {
+    return reinterpret_cast<unsigned char *>((reinterpret_cast<uintptr_t>(raw) + 255) &
+                                             ~uintptr_t(255));
 }
 
 struct SmemDict {
@@ -907,8 +914,9 @@ __device__ __forceinline__ void step_any(float (&h)[NPL], const float (&dv)[NPL]
 //        lane's segment; bit 10 b ends its segment; bits 11, 12 this lane's
 //        own targets (NPL e, NPL e + 1) have sources.
 // With NPL = 1 a lane holds only entry b.  pb holds d * h by element, ob the
-// segment sums by target (zero for targets without sources); the two
-// barriers keep them single-buffered.
+// segment sums by target (zero for targets without sources); both are
+// 256-byte aligned shared addresses, and the two barriers keep them
+// single-buffered.
 template <int NPL, int LV>
 __device__ __forceinline__ void step_seg(float (&h)[NPL], const float (&dv)[NPL],
                                          const float (&bv)[NPL], uint32_t pb, uint32_t ob,
@@ -923,12 +931,14 @@ __device__ __forceinline__ void step_seg(float (&h)[NPL], const float (&dv)[NPL]
         sts_f32x2(ob + lane * 8, 0.f, 0.f);
     }
     warp_barrier();
+    // pb and ob are 256-byte aligned: an entry's byte offset replaces the low
+    // byte of the buffer address (one byte permute per address)
     const uint32_t w0 = e.x, w1 = e.y;
-    const float zb = lds_f32(pb + ((w0 >> 8) & 0xffu));
+    const float zb = lds_f32(__byte_perm(w0, pb, 0x7651));
     float za = 0.f, v = zb;
     bool ab_same = false;
     if constexpr (NPL == 2) {
-        za = lds_f32(pb + (w0 & 0xffu));
+        za = lds_f32(__byte_perm(w0, pb, 0x7650));
         ab_same = (w1 >> 8) & 1u;
         if (ab_same) v = za + zb;
     }
@@ -940,9 +950,9 @@ __device__ __forceinline__ void step_seg(float (&h)[NPL], const float (&dv)[NPL]
     }
     if constexpr (NPL == 2) {
         const float left = __shfl_up_sync(kFull, v, 1);
-        if (!ab_same) sts_f32(ob + ((w0 >> 16) & 0xffu), ((w1 >> 9) & 1u) ? left + za : za);
+        if (!ab_same) sts_f32(__byte_perm(w0, ob, 0x7652), ((w1 >> 9) & 1u) ? left + za : za);
     }
-    if ((w1 >> 10) & 1u) sts_f32(ob + (w0 >> 24), v);
+    if ((w1 >> 10) & 1u) sts_f32(__byte_perm(w0, ob, 0x7653), v);
     warp_barrier();
     if constexpr (NPL == 1) {
         h[0] = lds_f32(ob + lane * 4) + bv[0];
@@ -989,7 +999,7 @@ inline int choose_wpc(KernT kern, const ChunkParams &p, int per_warp) {
     int best = 4, best_warps = -1;
     for (int wpc = 4; wpc <= kMaxWPC; wpc *= 2) {
         q.wpc = wpc;
-        const int smem = dict_region_bytes(q) + wpc * per_warp;
+        const int smem = dict_region_bytes(q) + wpc * per_warp + 256;
         if (smem > budget) continue;
         if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
             cudaSuccess)
@@ -1012,7 +1022,7 @@ template <typename KernT>
 inline cudaError_t launch_units(KernT kern, ChunkParams p, int per_warp, cudaStream_t st) {
     p.smem_per_warp = per_warp;
     p.wpc = choose_wpc(kern, p, per_warp);
-    const size_t smem = (size_t)dict_region_bytes(p) + (size_t)p.wpc * per_warp;
+    const size_t smem = (size_t)dict_region_bytes(p) + (size_t)p.wpc * per_warp + 256;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

@@ -46,7 +46,7 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
 
     const uint32_t map_s = smem_u32(sd.map);
     const uint32_t seg_lane = smem_u32(sd.seg) + lane * 8;
-    const uint32_t pb_s = smem_u32(pbuf), ob_s = pb_s + kPbStride * 4;
+    const uint32_t pb_s = smem_u32(pbuf), ob_s = pb_s + 256;   // both 256-byte aligned
     const uint32_t yb_lane = smem_u32(ybuf) + lane * 4;
     const uint32_t own_off = lane * NPL * (uint32_t)sizeof(T);
 
@@ -170,7 +170,8 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
 template <typename T, int NPL>
 __global__ void __launch_bounds__(kMaxWPC * 32, (sizeof(T) == 4 && NPL == 2) ? 2 : 3)
     k_phaseA_fast(const ChunkParams p) {
-    extern __shared__ __align__(128) unsigned char sm_a[];
+    extern __shared__ __align__(128) unsigned char sm_a_raw[];
+    unsigned char *sm_a = smem_base256(sm_a_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const SmemDict sd = stage_dict(p, sm_a, warp, lane, (int)sizeof(T));
     const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
@@ -186,7 +187,8 @@ __global__ void __launch_bounds__(kMaxWPC * 32, (sizeof(T) == 4 && NPL == 2) ? 2
 
 template <typename T, int NPL>
 __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams p) {
-    extern __shared__ __align__(128) unsigned char sm_c[];
+    extern __shared__ __align__(128) unsigned char sm_c_raw[];
+    unsigned char *sm_c = smem_base256(sm_c_raw);
     constexpr int N = 32 * NPL;
     constexpr int ROWB = N * (int)sizeof(T);
     constexpr int TENS = kTS * ROWB;
