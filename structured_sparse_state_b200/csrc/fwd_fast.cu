@@ -204,7 +204,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
 
     unsigned char *wbase = sm_c + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
     using RingT = FastRing<2, ROWB>;
-    float *ybuf = reinterpret_cast<float *>(wbase + kFastStages * RingT::STAGEB) + 2 * kPbStride;
+    float *ybuf = reinterpret_cast<float *>(wbase + kFastStages * RingT::STAGEB);   // [kTS][33]
     RingT ring;
     ring.ring_s = smem_u32(wbase);
     ring.bar0 = smem_u32(ybuf + kYbufFloats);
@@ -310,7 +310,9 @@ cudaError_t launch_phaseA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
 cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
     const int es = dt == PDSSM_BF16 ? 2 : 4;
     p.dict_content = dt == PDSSM_BF16 ? kDictMap16 : kDictMap;
-    p.smem_per_warp = warp_smem_bytes(p.ns, 2, (int)p.N * es);
+    // ring, readout buffer, barriers (no exchange buffers: no scatter here)
+    p.smem_per_warp =
+        (kFastStages * 2 * kTS * (int)p.N * es + kYbufFloats * 4 + kFastStages * 8 + 255) / 256 * 256;
     const size_t smem = 0;
     if (dt == PDSSM_BF16)
         return p.N == 64 ? launch_fast(k_phaseC_fast<__nv_bfloat16, 2>, p, smem, st)
