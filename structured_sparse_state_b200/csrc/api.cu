@@ -77,7 +77,7 @@ ChunkParams make_params(const pdssm_dims *dm, const WsLayout &w, void *ws, int64
     p.tab = reinterpret_cast<const uint8_t *>(base + w.tab);
     p.fan = reinterpret_cast<const int32_t *>(base + w.fan);
     p.seg = reinterpret_cast<const uint2 *>(base + w.seg);
-    p.seg_maxdist = reinterpret_cast<const int *>(base + w.status) + 1;
+    p.dict_stats = reinterpret_cast<const int *>(base + w.status) + 1;
     p.k = k;
     p.d = d;
     p.b = b;
@@ -174,8 +174,9 @@ static pdssm_status run_prep(const pdssm_dims *dims, const int32_t *pi_dict,
                              int64_t pi_head_stride, const WsLayout &w, void *ws,
                              cudaStream_t st) {
     unsigned char *base = reinterpret_cast<unsigned char *>(ws);
-    // status word and the segment tables' largest lane distance
-    cudaError_t e = cudaMemsetAsync(base + w.status, 0, 8, st);
+    // status word and the dictionary statistics (largest segment lane
+    // distance, largest fan-in)
+    cudaError_t e = cudaMemsetAsync(base + w.status, 0, 16, st);
     if (e != cudaSuccess) return cuda_fail(e, "status reset");
     e = launch_prep(*dims, pi_dict, pi_head_stride, reinterpret_cast<int32_t *>(base + w.dict),
                     reinterpret_cast<uint2 *>(base + w.seg),

@@ -219,7 +219,7 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
                 float dv[NPL], bv[NPL];
                 lds_own<T, NPL>(row + own_off, dv);
                 lds_own<T, NPL>(row + own_off + TENS, bv);
-                step_seg<NPL, LV>(h, dv, bv, pb_s, ob_s, lds_u32x2(seg_lane + kk * 256), lane);
+                pd_step<NPL, LV>(h, dv, bv, pb_s, ob_s, lds_u32x2(seg_lane + kk * 256), lane, q & 1);
             }
         } else {
             // pass 2: states of this tile, hsm[q] = h_{t0+q-1}
@@ -232,7 +232,7 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
                 float dv[NPL], bv[NPL];
                 lds_own<T, NPL>(row + own_off, dv);
                 lds_own<T, NPL>(row + own_off + TENS, bv);
-                step_seg<NPL, LV>(x, dv, bv, pb_s, ob_s, lds_u32x2(seg_lane + kk * 256), lane);
+                pd_step<NPL, LV>(x, dv, bv, pb_s, ob_s, lds_u32x2(seg_lane + kk * 256), lane, q & 1);
                 sts_own<NPL>(hs_lane + (q + 1) * (kMaxN * 4), x);
             }
             row = tile + (n - 1) * ROWB;
@@ -285,7 +285,8 @@ __global__ void __launch_bounds__(kMaxWPC * 32, 3) k_bwdC_fast(const ChunkParams
     const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
     if (unit >= p.units) return;
     unsigned char *wbase = sm_bc + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
-    switch (seg_levels(__ldg(p.seg_maxdist))) {
+    switch (step_variant(p.dict_stats)) {
+        case 0: bwdC_fast_unit<T, NPL, 0>(p, sd, wbase, unit, lane); break;
         case 1: bwdC_fast_unit<T, NPL, 1>(p, sd, wbase, unit, lane); break;
         case 2: bwdC_fast_unit<T, NPL, 2>(p, sd, wbase, unit, lane); break;
         case 3: bwdC_fast_unit<T, NPL, 3>(p, sd, wbase, unit, lane); break;

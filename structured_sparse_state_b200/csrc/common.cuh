@@ -82,7 +82,8 @@ struct ChunkParams {
     const uint8_t *tab;       // slot tables [Hd][K][kDcap][64]: s-th source of each target
     const int32_t *fan;       // largest fan-in of each map [Hd][K]
     const uint2 *seg;         // segment tables [Hd][K][32 lanes] (N = 32 or 64)
-    const int *seg_maxdist;   // largest lane distance inside a segment, all maps
+    const int *dict_stats;    // over all maps: [0] largest lane distance inside a
+                              // segment, [1] largest fan-in (1: all permutations)
     int dict_content;         // parts of the dictionary staged in shared memory
     const int32_t *k;
     const void *d, *b, *c;
@@ -963,10 +964,46 @@ __device__ __forceinline__ void step_seg(float (&h)[NPL], const float (&dv)[NPL]
     }
 }
 
-// Shuffle levels the segment tables need: the smallest LV in {1, 2, 3, 5}
-// with 2^LV > the largest lane distance inside a segment.
-__device__ __forceinline__ int seg_levels(int maxdist) {
-    return maxdist < 2 ? 1 : maxdist < 4 ? 2 : maxdist < 8 ? 3 : 5;
+// The PD step when every map of the dictionary is a permutation (fan-in 1):
+// a map's segment table then lists, for this lane's own targets, their only
+// sources (entries NPL*lane .. NPL*lane+NPL-1 are the lane's targets).  With
+// N = 32 the source's d * h comes by one shuffle; with N = 64 through the
+// exchange buffer pb, which callers alternate between two 256-byte aligned
+// buffers on consecutive steps (one barrier per step).
+template <int NPL>
+__device__ __forceinline__ void step_perm(float (&h)[NPL], const float (&dv)[NPL],
+                                          const float (&bv)[NPL], uint32_t pb, uint2 e,
+                                          int lane) {
+    if constexpr (NPL == 1) {
+        const float hd = dv[0] * h[0];
+        h[0] = __shfl_sync(kFull, hd, (int)((e.x >> 10) & 31u)) + bv[0];
+    } else {
+        sts_f32x2(pb + lane * 8, dv[0] * h[0], dv[1] * h[1]);
+        warp_barrier();
+        h[0] = lds_f32(__byte_perm(e.x, pb, 0x7650)) + bv[0];
+        h[1] = lds_f32(__byte_perm(e.x, pb, 0x7651)) + bv[1];
+    }
+}
+
+// One PD step: LV = 0 selects the permutation step (buffer by step parity),
+// otherwise the segment-table step with LV shuffle levels.
+template <int NPL, int LV>
+__device__ __forceinline__ void pd_step(float (&h)[NPL], const float (&dv)[NPL],
+                                        const float (&bv)[NPL], uint32_t pb, uint32_t ob,
+                                        uint2 e, int lane, int parity) {
+    if constexpr (LV == 0)
+        step_perm<NPL>(h, dv, bv, parity ? ob : pb, e, lane);
+    else
+        step_seg<NPL, LV>(h, dv, bv, pb, ob, e, lane);
+}
+
+// Step variant for a launch: 0 when every map is a permutation, else the
+// shuffle levels of the segment tables: the smallest LV in {1, 2, 3, 5} with
+// 2^LV above the largest lane distance inside a segment.
+__device__ __forceinline__ int step_variant(const int *dict_stats) {
+    if (__ldg(dict_stats + 1) <= 1) return 0;
+    const int md = __ldg(dict_stats);
+    return md < 2 ? 1 : md < 4 ? 2 : md < 8 ? 3 : 5;
 }
 
 // Warps per CTA for a chunk kernel with `per_warp` bytes of shared memory
@@ -1041,7 +1078,7 @@ bool select_tc_enabled();
 cudaError_t launch_select_tc(const pdssm_dims &dm, const void *u, const float *W, int32_t *k_out,
                              cudaStream_t st);
 cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
-                        uint2 *seg, int *seg_maxdist,
+                        uint2 *seg, int *dict_stats,
                         uint8_t *tab, int32_t *fan, int64_t Hd, int *status, cudaStream_t st);
 cudaError_t launch_validate(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs,
                             const int32_t *k, int *counts, cudaStream_t st);

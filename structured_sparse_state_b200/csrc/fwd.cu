@@ -269,7 +269,19 @@ struct ScatterScratch {
 // order, whose tree of additions depends only on the map.
 __device__ __forceinline__ void warp_scatter(const int (&P)[2], const float (&Z)[2],
                                              const float (&V)[2], float (&out)[2],
-                                             ScatterScratch &sc, int lane) {
+                                             ScatterScratch &sc, int lane, bool perm) {
+    if (perm) {
+        // every map is a permutation, so composed maps are too: each target
+        // has one source (padding entries all write 0 to index 63, which no
+        // real target uses when N < 64, and N = 64 has no padding)
+        sc.val[P[0]] = Z[0];
+        sc.val[P[1]] = Z[1];
+        __syncwarp();
+        out[0] = sc.val[lane] + V[0];
+        out[1] = sc.val[lane + 32] + V[1];
+        __syncwarp();
+        return;
+    }
     const unsigned lt = (1u << lane) - 1u;
     const unsigned m0 = __match_any_sync(kFull, P[0]);
     const unsigned m1 = __match_any_sync(kFull, P[1]);
@@ -361,12 +373,12 @@ struct Agg {
 __device__ __forceinline__ void compose_after(Agg &a, const int *tP, const float *tD,
                                               const int (&TP)[2], const float (&TD)[2],
                                               const float (&TV)[2], ScatterScratch &sc,
-                                              int lane) {
+                                              int lane, bool perm) {
     float z[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) z[r] = TD[r] * a.V[r];
     float nv[2];
-    warp_scatter(TP, z, TV, nv, sc, lane);
+    warp_scatter(TP, z, TV, nv, sc, lane, perm);
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         const int q = a.P[r];
@@ -384,6 +396,7 @@ __global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t bh = blockIdx.x;
     const int64_t C = p.C;
+    const bool perm = __ldg(p.dict_stats + 1) <= 1;   // every map a permutation
     // [2 buffers][nw][64] aggregates, [nw][64] carries, [nw] scratch
     int *aggP = reinterpret_cast<int *>(sm_b);
     float *aggD = reinterpret_cast<float *>(aggP + 2 * nw * 64);
@@ -434,7 +447,7 @@ __global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p) {
             float z[2], nv[2];
 #pragma unroll
             for (int r = 0; r < 2; ++r) z[r] = TD[i][r] * a.V[r];
-            warp_scatter(TP[i], z, TV[i], nv, sc, lane);
+            warp_scatter(TP[i], z, TV[i], nv, sc, lane, perm);
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 a.D[r] *= gD[r];
@@ -468,7 +481,7 @@ __global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p) {
             }
             const int *hP = aggP + (cur * nw + warp) * 64;
             const float *hD = aggD + (cur * nw + warp) * 64;
-            compose_after(lo, hP, hD, a.P, a.D, a.V, sc, lane);
+            compose_after(lo, hP, hD, a.P, a.D, a.V, sc, lane, perm);
             a = lo;
         }
         const int nxt = cur ^ 1;
@@ -491,7 +504,7 @@ __global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p) {
             const int e = lane + 32 * r;
             z[r] = a.D[r] * (e < p.N ? p.h0[bh * p.N + e] : 0.f);
         }
-        warp_scatter(a.P, z, a.V, S, sc, lane);
+        warp_scatter(a.P, z, a.V, S, sc, lane, perm);
     } else {
 #pragma unroll
         for (int r = 0; r < 2; ++r) S[r] = a.V[r];
@@ -525,7 +538,7 @@ __global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p) {
             float z[2];
 #pragma unroll
             for (int r = 0; r < 2; ++r) z[r] = TD[i][r] * x[r];
-            warp_scatter(TP[i], z, TV[i], x, sc, lane);
+            warp_scatter(TP[i], z, TV[i], x, sc, lane, perm);
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
                 const int e = lane + 32 * r;

@@ -11,8 +11,8 @@
 
 namespace pdssm {
 
-// Phase A of one chunk (this warp's unit) with LV shuffle levels in the
-// segment-table step.
+// Phase A of one chunk (this warp's unit); LV selects the PD step (0: the
+// permutation step, else the segment-table step with LV shuffle levels).
 template <typename T, int NPL, int LV>
 __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const SmemDict &sd,
                                                  unsigned char *wbase, int64_t unit, int lane) {
@@ -117,7 +117,7 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
                         Dl[r] *= lds_elem_at<T, Q * ROWB>(row0s + posb[r]);
                         posb[r] = lds_next_pos<T>(pk + posb[r]);
                     }
-                    step_seg<NPL, LV>(h, dv, bv, pb_s, ob_s, e, lane);
+                    pd_step<NPL, LV>(h, dv, bv, pb_s, ob_s, e, lane, Q & 1);
                     const int kk_n = __shfl_sync(kFull, kreg, Q + 1);
                     float dv_n[NPL], bv_n[NPL], cv_n[NPL];
                     lds_own_at<T, NPL, (Q + 1) * ROWB>(row0s + own_off, dv_n);
@@ -136,7 +136,7 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
                     Dl[r] *= lds_elem_at<T, 0>(row + posb[r]);
                     posb[r] = lds_next_pos<T>(pk + posb[r]);
                 }
-                step_seg<NPL, LV>(h, dv, bv, pb_s, ob_s, e, lane);
+                pd_step<NPL, LV>(h, dv, bv, pb_s, ob_s, e, lane, q & 1);
                 const int kk_n = __shfl_sync(kFull, kreg, q + 1);
                 const uint32_t row_n = row + ROWB;
                 float dv_n[NPL], bv_n[NPL], cv_n[NPL];
@@ -177,7 +177,8 @@ __global__ void __launch_bounds__(kMaxWPC * 32, (sizeof(T) == 4 && NPL == 2) ? 2
     const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
     if (unit >= p.units) return;
     unsigned char *wbase = sm_a + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
-    switch (seg_levels(__ldg(p.seg_maxdist))) {
+    switch (step_variant(p.dict_stats)) {
+        case 0: phaseA_fast_unit<T, NPL, 0>(p, sd, wbase, unit, lane); break;
         case 1: phaseA_fast_unit<T, NPL, 1>(p, sd, wbase, unit, lane); break;
         case 2: phaseA_fast_unit<T, NPL, 2>(p, sd, wbase, unit, lane); break;
         case 3: phaseA_fast_unit<T, NPL, 3>(p, sd, wbase, unit, lane); break;

@@ -128,7 +128,7 @@ cudaError_t launch_select(const pdssm_dims &dm, const void *u, pdssm_dtype ut, c
 constexpr int kPrepWarps = 4;
 
 __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *__restrict__ dict,
-                       uint2 *__restrict__ seg, int *__restrict__ seg_maxdist,
+                       uint2 *__restrict__ seg, int *__restrict__ dict_stats,
                        uint8_t *__restrict__ tab, int32_t *__restrict__ fan, int64_t nmaps,
                        int K, int N, int *status) {
     __shared__ int s_off[kPrepWarps][65];   // first sorted entry of each target (+ total)
@@ -192,7 +192,10 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
     bad = __any_sync(kFull, bad);
     if (bad && lane == 0) flag_status(status, kStBadIndex);
     const int D = __reduce_max_sync(kFull, max(cnt0, cnt1));
-    if (lane == 0) fan[m] = D;
+    if (lane == 0) {
+        fan[m] = D;
+        atomicMax(dict_stats + 1, D);
+    }
 
     // segment table (fast path only: N = 32 or 64)
     if (N != 32 && N != 64) return;
@@ -239,15 +242,15 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
     }
     seg[m * 32 + lane] = make_uint2(w0, w1);
     const int md = __reduce_max_sync(kFull, dist);
-    if (lane == 0) atomicMax(seg_maxdist, md);
+    if (lane == 0) atomicMax(dict_stats, md);
 }
 
 cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
-                        uint2 *seg, int *seg_maxdist,
+                        uint2 *seg, int *dict_stats,
                         uint8_t *tab, int32_t *fan, int64_t Hd, int *status, cudaStream_t st) {
     const int64_t nmaps = Hd * dm.K;
     const int64_t grid = (nmaps + kPrepWarps - 1) / kPrepWarps;
-    k_prep<<<(unsigned)grid, 32 * kPrepWarps, 0, st>>>(pi, pi_hs, dict, seg, seg_maxdist, tab, fan,
+    k_prep<<<(unsigned)grid, 32 * kPrepWarps, 0, st>>>(pi, pi_hs, dict, seg, dict_stats, tab, fan,
                                                        nmaps, (int)dm.K, (int)dm.N, status);
     return cudaGetLastError();
 }

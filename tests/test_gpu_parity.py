@@ -213,6 +213,17 @@ def test_forward_map_kinds(kind, N):
     check_fwd(small(7, 1, 2, 500, N, 3, kind=kind), chunk=64)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N", [32, 64])
+def test_permutation_dictionaries_forward_and_adjoint(N, dtype):
+    """Every map a permutation: the kernels switch to the permutation step
+    (a shuffle for N = 32, one exchange per step for N = 64)."""
+    inp = small(40 + N, 2, 2, 700, N, 6, kind="perm", dtype=dtype)
+    check_fwd(inp, chunk=96)
+    if dtype == "f32":
+        check_bwd(inp, chunk=96)
+
+
 @pytest.mark.parametrize("fan", [7, 8, 9, 20])
 @pytest.mark.parametrize("N", [24, 64])
 def test_forward_fan_in_around_slot_capacity(fan, N):
