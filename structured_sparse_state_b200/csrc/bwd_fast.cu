@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_bwdA_fast(const ChunkParams p)
 
     const int ntiles = (len + kTS - 1) / kTS;
     // tiles in reverse order: slot j holds chunk tile ntiles - 1 - j
-    for (int j = 0; j < kFastStages && j < ntiles; ++j) ring.issue_tile(j, ntiles - 1 - j, 2, lane);
+    for (int j = 0; j < kFastStages && j < ntiles; ++j) ring.issue_tile(j, ntiles - 1 - j, 3u, lane);
     const uint32_t map_s = smem_u32(sd.map), lb_s = smem_u32(lbuf);
     const uint32_t own_off = lane * NPL * (uint32_t)sizeof(T);
     const int32_t *kp = p.k + row0;
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_bwdA_fast(const ChunkParams p)
             for (int r = 0; r < NPL; ++r) mu[r] = dv[r] * lds_f32(lb + t4[r]);
         }
         warp_barrier();
-        if (j + kFastStages < ntiles) ring.issue_tile(j + kFastStages, ntiles - 1 - (j + kFastStages), 2, lane);
+        if (j + kFastStages < ntiles) ring.issue_tile(j + kFastStages, ntiles - 1 - (j + kFastStages), 3u, lane);
         kreg = clamp_k(knext, K, p.status);
         gyreg = gynext;
     }
@@ -131,12 +131,11 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_bwdA_fast(const ChunkParams p)
 }
 
 // ---------------------------------------------------------------------------
-// bwd phase C: pass 1 runs the chunk forward from its carry and checkpoints
-// the state at every tile start; pass 2 takes the tiles in reverse, recomputes
-// each tile's states from its checkpoint and sweeps back emitting g_b, g_c,
-// g_d.  The checkpoint of tile ti is kept in g_b's row at the tile start: pass
-// 2 reads it before it writes that tile's rows, and earlier tiles' rows are
-// written only after their own checkpoints have been read.
+// bwd phase C: pass 1 runs the chunk forward from its carry and leaves every
+// state h_t in g_c's row t; pass 2 takes the tiles in reverse, reads each
+// tile's states back (prefetched one tile ahead) and sweeps back emitting
+// g_b, g_c, g_d.  Step t of the sweep reads rows t and t - 1 of g_c and then
+// overwrites row t with its gradient; rows below t are still states.
 // ---------------------------------------------------------------------------
 constexpr int kBwdFastExtraFloats = 2 * kPbStride + (kTS + 1) * kMaxN;
 
@@ -169,8 +168,9 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
     const int ntiles = (len + kTS - 1) / kTS;
     const int total = 2 * ntiles;   // pass 1 tiles, then pass 2 tiles (reverse)
     auto tile_of = [&](int m) { return m < ntiles ? m : 2 * ntiles - 1 - m; };
-    auto nt_of = [&](int m) { return m < ntiles ? 2 : 3; };
-    for (int m = 0; m < kFastStages && m < total; ++m) ring.issue_tile(m, tile_of(m), nt_of(m), lane);
+    // pass 1 stages d and b, pass 2 d and c
+    auto mask_of = [&](int m) { return m < ntiles ? 3u : 5u; };
+    for (int m = 0; m < kFastStages && m < total; ++m) ring.issue_tile(m, tile_of(m), mask_of(m), lane);
 
     const uint32_t map_s = smem_u32(sd.map);
     const uint32_t seg_lane = smem_u32(sd.seg) + lane * 8;
@@ -183,13 +183,29 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
     float *gc = p.g_c + row0 * N;
     float *gd = p.g_d + row0 * N;
 
-    float h[NPL], mu[NPL];
+    float h[NPL], hinit[NPL], mu[NPL];
 #pragma unroll
     for (int r = 0; r < NPL; ++r) {
         const int e = lane * NPL + r;
         h[r] = cidx == 0 ? (p.h0 ? p.h0[bh * N + e] : 0.f) : p.Hc[(unit - 1) * N + e];
+        hinit[r] = h[r];
         mu[r] = p.lam[unit * N + e];
     }
+    // states of the next pass-2 tile, rows t0 - 1 .. t0 + n - 1
+    float nst[kTS + 1][NPL];
+    auto load_states = [&](int ti2) {
+        const int t02 = ti2 * kTS, n2 = min(kTS, len - t02);
+#pragma unroll
+        for (int q = 0; q <= kTS; ++q) {
+            if (q > n2) break;
+            if (q == 0 && t02 == 0) {
+#pragma unroll
+                for (int r = 0; r < NPL; ++r) nst[0][r] = hinit[r];
+            } else {
+                ldg_own<NPL>(gc + (int64_t)(t02 + q - 1) * N, lane, nst[q]);
+            }
+        }
+    };
     int kreg = load_k(kp, lane, lane < kTS && lane < len, K, p.status);
     float gyreg = 0.f;
 
@@ -211,8 +227,7 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
         }
         const uint32_t tile = ring.tile(m);
         if (m < ntiles) {
-            // pass 1: checkpoint at the tile start, then advance the state
-            stg_own<NPL>(gb + (int64_t)t0 * N, lane, h);
+            // pass 1: advance the state, leaving h_t in g_c's row t
             uint32_t row = tile;
             for (int q = 0; q < n; ++q, row += ROWB) {
                 const int kk = __shfl_sync(kFull, kreg, q);
@@ -220,22 +235,17 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
                 lds_own<T, NPL>(row + own_off, dv);
                 lds_own<T, NPL>(row + own_off + TENS, bv);
                 pd_step<NPL, LV>(h, dv, bv, pb_s, ob_s, lds_u32x2(seg_lane + kk * 256), lane, q & 1);
+                stg_own<NPL>(gc + (int64_t)(t0 + q) * N, lane, h);
             }
         } else {
             // pass 2: states of this tile, hsm[q] = h_{t0+q-1}
-            float x[NPL];
-            ldg_own<NPL>(gb + (int64_t)t0 * N, lane, x);
-            sts_own<NPL>(hs_lane, x);
-            uint32_t row = tile;
-            for (int q = 0; q < n; ++q, row += ROWB) {
-                const int kk = __shfl_sync(kFull, kreg, q);
-                float dv[NPL], bv[NPL];
-                lds_own<T, NPL>(row + own_off, dv);
-                lds_own<T, NPL>(row + own_off + TENS, bv);
-                pd_step<NPL, LV>(x, dv, bv, pb_s, ob_s, lds_u32x2(seg_lane + kk * 256), lane, q & 1);
-                sts_own<NPL>(hs_lane + (q + 1) * (kMaxN * 4), x);
+#pragma unroll
+            for (int q = 0; q <= kTS; ++q) {
+                if (q > n) break;
+                sts_own<NPL>(hs_lane + q * (kMaxN * 4), nst[q]);
             }
-            row = tile + (n - 1) * ROWB;
+            __syncwarp();
+            uint32_t row = tile + (n - 1) * ROWB;
             for (int q = n - 1; q >= 0; --q, row -= ROWB) {
                 const int kk = __shfl_sync(kFull, kreg, q);
                 const float gy = __shfl_sync(kFull, gyreg, q);
@@ -269,15 +279,17 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
         warp_barrier();
         if (m + kFastStages < total) {
             const int mn = m + kFastStages;
-            ring.issue_tile(mn, tile_of(mn), nt_of(mn), lane);
+            ring.issue_tile(mn, tile_of(mn), mask_of(mn), lane);
         }
+        // the next pass-2 tile's states (written by this lane in pass 1)
+        if (m + 1 >= ntiles && m + 1 < total) load_states(tile_of(m + 1));
         kreg = clamp_k(knext, K, p.status);
         gyreg = gynext;
     }
 }
 
 template <typename T, int NPL>
-__global__ void __launch_bounds__(kMaxWPC * 32, 3) k_bwdC_fast(const ChunkParams p) {
+__global__ void __launch_bounds__(kMaxWPC * 32, 2) k_bwdC_fast(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_bc_raw[];
     unsigned char *sm_bc = smem_base256(sm_bc_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -633,21 +633,22 @@ struct FastRing {
 
     __device__ uint32_t tile(int i) const { return ring_s + (uint32_t)((i & 1) * STAGEB); }
 
-    // Copy chunk tile ti (first ntc tensors) into stage m & 1.
-    __device__ void issue_tile(int m, int ti, int ntc, int lane) const {
+    // Copy chunk tile ti into stage m & 1: the tensors whose bits are set in
+    // `mask` (bit q: tensor q).
+    __device__ void issue_tile(int m, int ti, unsigned mask, int lane) const {
         if (lane == 0) {
             const int stage = m & 1;
             const uint32_t bytes = (uint32_t)(min(kTS, len - ti * kTS) * ROWB);
             const uint32_t bar = bar0 + 8u * stage;
-            mbar_expect_tx(bar, bytes * (uint32_t)ntc);
+            mbar_expect_tx(bar, bytes * (uint32_t)__popc(mask));
 #pragma unroll
             for (int q = 0; q < NT; ++q)
-                if (q < ntc)
+                if ((mask >> q) & 1u)
                     bulk_g2s(ring_s + (uint32_t)(stage * STAGEB + q * TENS),
                              src[q] + (size_t)ti * TENS, bytes, bar);
         }
     }
-    __device__ void issue(int i, int lane) const { issue_tile(i, i, nt, lane); }
+    __device__ void issue(int i, int lane) const { issue_tile(i, i, (1u << nt) - 1u, lane); }
 
     __device__ bool wait(int i) const {
         return mbar_wait_fast(bar0 + 8u * (uint32_t)(i & 1), (uint32_t)((i >> 1) & 1));
