@@ -1007,6 +1007,32 @@ __device__ __forceinline__ int step_variant(const int *dict_stats) {
     return md < 2 ? 1 : md < 4 ? 2 : md < 8 ? 3 : 5;
 }
 
+// Programmatic dependent launch: a kernel launched with launch_pdl may start
+// while its predecessor in the stream finishes; pdl_wait() blocks until the
+// predecessor has completed and its writes are visible (a no-op for a normal
+// launch), and pdl_trigger() lets the successor start launching once every
+// CTA of this grid has issued it.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // Warps per CTA for a chunk kernel with `per_warp` bytes of shared memory
 // per warp: 4 or 8, whichever keeps more warps resident per SM by the
 // runtime's occupancy calculation (registers, shared memory with the
@@ -1057,7 +1083,8 @@ inline int choose_wpc(KernT kern, const ChunkParams &p, int per_warp) {
 }
 
 template <typename KernT>
-inline cudaError_t launch_units(KernT kern, ChunkParams p, int per_warp, cudaStream_t st) {
+inline cudaError_t launch_units(KernT kern, ChunkParams p, int per_warp, cudaStream_t st,
+                                bool pdl = false) {
     p.smem_per_warp = per_warp;
     p.wpc = choose_wpc(kern, p, per_warp);
     const size_t smem = (size_t)dict_region_bytes(p) + (size_t)p.wpc * per_warp + 256;
@@ -1065,6 +1092,7 @@ inline cudaError_t launch_units(KernT kern, ChunkParams p, int per_warp, cudaStr
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int64_t grid = (p.units + p.wpc - 1) / p.wpc;
+    if (pdl) return launch_pdl(kern, dim3((unsigned)grid), dim3(p.wpc * 32), smem, st, p);
     kern<<<(unsigned)grid, p.wpc * 32, smem, st>>>(p);
     return cudaGetLastError();
 }

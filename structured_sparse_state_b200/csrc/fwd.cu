@@ -394,6 +394,8 @@ __global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p) {
     extern __shared__ __align__(16) unsigned char sm_b[];
     const int nw = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    pdl_trigger();
+    pdl_wait();   // the chunk transfers come from the preceding kernel
     const int64_t bh = blockIdx.x;
     const int64_t C = p.C;
     const bool perm = __ldg(p.dict_stats + 1) <= 1;   // every map a permutation
@@ -601,8 +603,7 @@ cudaError_t launch_phaseB(const ChunkParams &p, cudaStream_t st) {
     cudaError_t e =
         cudaFuncSetAttribute(k_phaseB, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_phaseB<<<(unsigned)BH, nw * 32, smem, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(k_phaseB, dim3((unsigned)BH), dim3(nw * 32), smem, st, p);
 }
 
 }  // namespace pdssm

@@ -172,6 +172,8 @@ __global__ void __launch_bounds__(kMaxWPC * 32, (sizeof(T) == 4 && NPL == 2) ? 2
     k_phaseA_fast(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_a_raw[];
     unsigned char *sm_a = smem_base256(sm_a_raw);
+    pdl_trigger();
+    pdl_wait();   // the dictionary tables come from the preceding kernel
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const SmemDict sd = stage_dict(p, sm_a, warp, lane, (int)sizeof(T));
     const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
@@ -190,6 +192,8 @@ template <typename T, int NPL>
 __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_c_raw[];
     unsigned char *sm_c = smem_base256(sm_c_raw);
+    pdl_trigger();
+    pdl_wait();   // the carries come from the preceding kernel
     constexpr int N = 32 * NPL;
     constexpr int ROWB = N * (int)sizeof(T);
     constexpr int TENS = kTS * ROWB;
@@ -288,7 +292,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
 
 template <typename KernT>
 static cudaError_t launch_fast(KernT kern, const ChunkParams &p, size_t, cudaStream_t st) {
-    return launch_units(kern, p, p.smem_per_warp, st);
+    return launch_units(kern, p, p.smem_per_warp, st, true);
 }
 
 // The fast kernels stage with bulk copies through a two-stage ring.

@@ -136,6 +136,7 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
     __shared__ int s_tgt[kPrepWarps][64];   // sorted entries: target
     __shared__ int s_cnt0[kPrepWarps][64];  // sources of each target among j < 32
     __shared__ int s_cnt[kPrepWarps][64];   // sources of each target
+    pdl_trigger();
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int64_t m = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib;
     if (m >= nmaps) return;

@@ -168,6 +168,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     extern __shared__ __align__(1024) unsigned char sm_raw[];
     unsigned char *sm = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(sm_raw) + 1023) & ~uintptr_t(1023));
+    pdl_trigger();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int D = p.D, NP = p.NP, H = p.H, K = KT;
     const int nkc = D / 8;
@@ -279,6 +280,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const uint32_t tmem = *tmem_slot;
     const uint32_t tcols = p.tcols;
 
+    // The weight split and the first copies of u (inputs) may overlap the
+    // preceding kernel; k_out, which it may still read, is written only after
+    // it has completed.
+    pdl_wait();
     bool ok = true;
     if (warp == kTcEpiWarps) {
         // ---- control: MMAs of tile j, then the copy of tile j + 1 into the
@@ -570,8 +575,7 @@ cudaError_t launch_select_tc(const pdssm_dims &dm, const void *u, const float *W
         cudaError_t e =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        kern<<<grid, kTcThreads, smem, st>>>(map, p);
-        return cudaGetLastError();
+        return launch_pdl(kern, dim3(grid), dim3(kTcThreads), smem, st, map, p);
     };
     if (sw) {
         switch (p.K) {
