@@ -5,8 +5,9 @@
 // r < NPL, NPL = ceil(N / 32) in {1, 2}.  Chunk data (rows of d, b, c) are
 // contiguous in HBM, so each warp streams its chunk through shared memory in
 // tiles of kTS steps with 1-D bulk copies (cp.async.bulk, the TMA engine's
-// non-tensor path) completed on per-warp mbarriers, double- or
-// triple-buffered.
+// non-tensor path) completed on per-warp mbarriers: a compile-time two-stage
+// ring in the fast kernels (N = 32 / 64), a ring of p.ns stages with L2
+// prefetch ahead of it in the general kernels.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -25,9 +26,9 @@ constexpr int kTS = 8;         // steps per staged tile = steps per readout grou
 constexpr int kMaxWPC = 8;     // most warps (units) per CTA in the chunk kernels
 constexpr int kMaxN = 64;
 constexpr int kMaxStages = 4;
-constexpr int kBwdMaxChunk = 256;   // checkpoints of one chunk kept in shared memory
+constexpr int kBwdMaxChunk = 256;   // checkpoints of one chunk kept in shared memory (general bwd C)
 constexpr int kDcap = 8;            // sources per target held in the slot table
-constexpr int kPrefetchTiles = 4;   // tiles prefetched into L2 ahead of the staged ones
+constexpr int kPrefetchTiles = 4;   // tiles prefetched into L2 ahead of the staged ones (general kernels)
 constexpr int kZeroSlot = 64;       // exchange-buffer entry that always holds 0
 constexpr int kPbStride = 80;       // floats per exchange buffer (64 + zero slot, padded)
 constexpr unsigned kFull = 0xffffffffu;
@@ -325,40 +326,6 @@ __device__ __forceinline__ void for_each_q(F &&f, std::integer_sequence<int, Qs.
     (f(std::integral_constant<int, Qs>{}), ...);
 }
 
-// Reduce-scatter of 16 per-lane partials: lane l (and l + 16) returns
-// sum over all 32 lanes of v[l & 15].  16 shuffles for 16 values.
-__device__ __forceinline__ float reduce_scatter16(float (&v)[kTS]) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const bool up = lane & 8;
-        const float send = up ? v[i] : v[i + 8];
-        const float keep = up ? v[i + 8] : v[i];
-        v[i] = keep + __shfl_xor_sync(kFull, send, 8);
-    }
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const bool up = lane & 4;
-        const float send = up ? v[i] : v[i + 4];
-        const float keep = up ? v[i + 4] : v[i];
-        v[i] = keep + __shfl_xor_sync(kFull, send, 4);
-    }
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-        const bool up = lane & 2;
-        const float send = up ? v[i] : v[i + 2];
-        const float keep = up ? v[i + 2] : v[i];
-        v[i] = keep + __shfl_xor_sync(kFull, send, 2);
-    }
-    {
-        const bool up = lane & 1;
-        const float send = up ? v[0] : v[1];
-        const float keep = up ? v[1] : v[0];
-        v[0] = keep + __shfl_xor_sync(kFull, send, 1);
-    }
-    return v[0] + __shfl_xor_sync(kFull, v[0], 16);
-}
-
 // Load the NPL elements a lane owns from one staged row (0 beyond N).
 template <typename T, int NPL, bool EVEN>
 __device__ __forceinline__ void load_row(const T *row, int lane, int N, float (&v)[NPL]) {
@@ -409,27 +376,6 @@ __device__ __forceinline__ int load_k_raw(const int32_t *kp, int64_t idx, bool v
 // ---------------------------------------------------------------------------
 // dictionary in shared memory and the PD step as a shared-memory scatter
 // ---------------------------------------------------------------------------
-
-// Targets pi_k(e) of the elements a lane owns (e = lane*NPL + r).
-template <int NPL, bool EVEN>
-__device__ __forceinline__ void own_targets(const int *pk, int lane, int N, int (&tgt)[NPL]) {
-    if constexpr (NPL == 2 && EVEN) {
-        if (2 * lane < N) {
-            const int2 q = *reinterpret_cast<const int2 *>(pk + 2 * lane);
-            tgt[0] = q.x;
-            tgt[1] = q.y;
-        } else {
-            tgt[0] = 0;
-            tgt[1] = 0;
-        }
-    } else {
-#pragma unroll
-        for (int r = 0; r < NPL; ++r) {
-            const int e = lane * NPL + r;
-            tgt[r] = e < N ? pk[e] : 0;
-        }
-    }
-}
 
 // Loads the NPL elements a lane owns from one staged row.  FULL means the
 // state fills the warp (N == 32 * NPL): no guards, vector loads.
@@ -814,88 +760,6 @@ __device__ __forceinline__ void lds_own_at(uint32_t a, float (&v)[NPL]) {
         const float2 q = lds_pair_at<T, OFF>(a);
         v[0] = q.x;
         v[1] = q.y;
-    }
-}
-
-// byte offset of element `pos4 / 4` in a row of T
-template <typename T>
-__device__ __forceinline__ uint32_t elem_off(int pos4) {
-    return sizeof(T) == 4 ? (uint32_t)pos4 : (uint32_t)pos4 >> 1;
-}
-
-// The PD step with the slot gather fully unrolled to S slots (S >= the
-// map's fan-in; padding slots point at the zero entry).  Table entries are
-// read-only, so they are fetched before the warp barrier; the S value loads
-// after it issue back to back, and the sums keep the slot (ascending source)
-// order.
-template <int NPL, int S>
-__device__ __forceinline__ void step_slots(float (&h)[NPL], const float (&dv)[NPL],
-                                           const float (&bv)[NPL], uint32_t pb, uint32_t tl,
-                                           int lane) {
-    unsigned w[S];
-#pragma unroll
-    for (int sl = 0; sl < S; ++sl) w[sl] = NPL == 1 ? lds_u8(tl + sl * 64) : lds_u16(tl + sl * 64);
-    if constexpr (NPL == 1)
-        sts_f32(pb + lane * 4, dv[0] * h[0]);
-    else
-        sts_f32x2(pb + lane * 8, dv[0] * h[0], dv[1] * h[1]);
-    warp_barrier();
-    float v[NPL][S];
-#pragma unroll
-    for (int sl = 0; sl < S; ++sl) {
-        if constexpr (NPL == 1) {
-            v[0][sl] = lds_f32(pb + w[sl] * 4);
-        } else {
-            v[0][sl] = lds_f32(pb + (w[sl] & 0xffu) * 4);
-            v[1][sl] = lds_f32(pb + (w[sl] >> 8) * 4);
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < NPL; ++r) {
-        float acc = v[r][0];
-#pragma unroll
-        for (int sl = 1; sl < S; ++sl) acc += v[r][sl];
-        h[r] = acc + bv[r];
-    }
-}
-
-// Dispatch on the map's fan-in class; above kDcap, scan all sources.
-template <int NPL>
-__device__ __forceinline__ void step_any(float (&h)[NPL], const float (&dv)[NPL],
-                                         const float (&bv)[NPL], uint32_t pb, uint32_t tl,
-                                         int Dk, uint32_t pk, int lane) {
-    static_assert(kDcap == 8, "fan-in classes below are written for kDcap = 8");
-    switch (Dk) {
-        case 0:
-        case 1: step_slots<NPL, 1>(h, dv, bv, pb, tl, lane); return;
-        case 2: step_slots<NPL, 2>(h, dv, bv, pb, tl, lane); return;
-        case 3: step_slots<NPL, 3>(h, dv, bv, pb, tl, lane); return;
-        case 4: step_slots<NPL, 4>(h, dv, bv, pb, tl, lane); return;
-        case 5: step_slots<NPL, 5>(h, dv, bv, pb, tl, lane); return;
-        case 6: step_slots<NPL, 6>(h, dv, bv, pb, tl, lane); return;
-        case 7:
-        case kDcap: step_slots<NPL, kDcap>(h, dv, bv, pb, tl, lane); return;
-        default: break;
-    }
-    {
-        constexpr int N = 32 * NPL;
-        if constexpr (NPL == 1)
-            sts_f32(pb + lane * 4, dv[0] * h[0]);
-        else
-            sts_f32x2(pb + lane * 8, dv[0] * h[0], dv[1] * h[1]);
-        warp_barrier();
-        float acc[NPL];
-#pragma unroll
-        for (int r = 0; r < NPL; ++r) acc[r] = 0.f;
-        for (int j = 0; j < N; ++j) {
-            const int t4 = lds_s32(pk + j * 4);
-            const float vj = lds_f32(pb + j * 4);
-#pragma unroll
-            for (int r = 0; r < NPL; ++r)
-                if (t4 == (lane * NPL + r) * 4) acc[r] += vj;
-        }
-#pragma unroll
-        for (int r = 0; r < NPL; ++r) h[r] = acc[r] + bv[r];
     }
 }
 

@@ -1,12 +1,14 @@
-// Forward phases A and C for a state that fills the warp (N = 32 or 64):
-// the same arithmetic as fwd.cu, written against explicit 32-bit shared
-// addresses so that a step costs few integer instructions:
-//   * the dictionary is staged as byte offsets (entry * 4), so following a
-//     column is one shared load per step;
-//   * the three tensors of a staged row sit at fixed distances, read with
-//     immediate offsets;
+// Forward phases A and C for a state that fills the warp (N = 32 or 64) with
+// 16-byte aligned rows: the arithmetic of fwd.cu, written against explicit
+// 32-bit shared addresses so that a step costs few instructions:
+//   * the maps are staged with entries of the element size holding byte
+//     offsets, so following a column is one shared load per step;
+//   * the PD step goes through the per-map segment tables (or the
+//     permutation step when every map is a permutation);
+//   * full tiles are unrolled at compile time: row, readout and lane offsets
+//     are immediates;
 //   * readout partials go to the per-warp transpose buffer.
-// The general kernels in fwd.cu serve every other N.
+// The general kernels in fwd.cu serve every other N and unaligned rows.
 #include "common.cuh"
 
 namespace pdssm {
