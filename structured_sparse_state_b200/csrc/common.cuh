@@ -768,37 +768,33 @@ __device__ __forceinline__ void lds_own_at(uint32_t a, float (&v)[NPL]) {
 // per lane in order, so every target's sources form one segment of
 // consecutive entries.  Each lane loads its entries' d * h, a segmented
 // inclusive scan over the lanes (LV shuffle levels; 2^LV must exceed the
-// largest lane distance inside a segment) sums every segment, the entry
-// that ends a segment stores the sum under its target, and the owners read
-// their targets back.  The cost does not depend on the fan-in, and the sum
-// of each target follows a fixed tree, so the step is deterministic.
+// largest lane distance inside a segment) sums every segment, and each
+// owner fetches its targets' sums by shuffle from the lane holding the entry
+// that ends the segment, then adds b.  The cost does not depend on the
+// fan-in, and the sum of each target follows a fixed tree, so the step is
+// deterministic.
 //
 // Entry word e (per map and lane):
 //   e.x: byte offsets (index * 4) of source a, source b, target a, target b
 //   e.y: bits 0-7 lane distance back to the start of b's segment;
 //        bit 8 a and b share a target; bit 9 a continues the previous
 //        lane's segment; bit 10 b ends its segment; bits 11, 12 this lane's
-//        own targets (NPL e, NPL e + 1) have sources.
-// With NPL = 1 a lane holds only entry b.  pb holds d * h by element, ob the
-// segment sums by target (zero for targets without sources); both are
-// 256-byte aligned shared addresses, and the two barriers keep them
-// single-buffered.
+//        own targets (NPL e, NPL e + 1) have sources; bits 16-20 / 21 the
+//        lane and entry (0: a, 1: b) ending the first own target's segment,
+//        bits 22-26 / 27 the same for the second.
+// With NPL = 1 a lane holds only entry b.  pb holds d * h by element; it is
+// 256-byte aligned and callers alternate two such buffers on consecutive
+// steps (one barrier per step).
 template <int NPL, int LV>
 __device__ __forceinline__ void step_seg(float (&h)[NPL], const float (&dv)[NPL],
-                                         const float (&bv)[NPL], uint32_t pb, uint32_t ob,
-                                         uint2 e, int lane) {
-    // d * h by element, and zero sums for this lane's own targets (targets
-    // without sources keep them)
-    if constexpr (NPL == 1) {
+                                         const float (&bv)[NPL], uint32_t pb, uint2 e,
+                                         int lane) {
+    if constexpr (NPL == 1)
         sts_f32(pb + lane * 4, dv[0] * h[0]);
-        sts_f32(ob + lane * 4, 0.f);
-    } else {
+    else
         sts_f32x2(pb + lane * 8, dv[0] * h[0], dv[1] * h[1]);
-        sts_f32x2(ob + lane * 8, 0.f, 0.f);
-    }
     warp_barrier();
-    // pb and ob are 256-byte aligned: an entry's byte offset replaces the low
-    // byte of the buffer address (one byte permute per address)
+    // an entry's byte offset replaces the low byte of the buffer address
     const uint32_t w0 = e.x, w1 = e.y;
     const float zb = lds_f32(__byte_perm(w0, pb, 0x7651));
     float za = 0.f, v = zb;
@@ -814,18 +810,20 @@ __device__ __forceinline__ void step_seg(float (&h)[NPL], const float (&dv)[NPL]
         const float t = __shfl_up_sync(kFull, v, o);
         if (dist >= o) v = t + v;
     }
-    if constexpr (NPL == 2) {
-        const float left = __shfl_up_sync(kFull, v, 1);
-        if (!ab_same) sts_f32(__byte_perm(w0, ob, 0x7652), ((w1 >> 9) & 1u) ? left + za : za);
-    }
-    if ((w1 >> 10) & 1u) sts_f32(__byte_perm(w0, ob, 0x7653), v);
-    warp_barrier();
+    // v: the sum of b's segment up to b; sa: the sum of a's segment up to a
     if constexpr (NPL == 1) {
-        h[0] = lds_f32(ob + lane * 4) + bv[0];
+        const float x = __shfl_sync(kFull, v, (int)((w1 >> 16) & 31u));
+        h[0] = ((w1 >> 11) & 1u ? x : 0.f) + bv[0];
     } else {
-        const float2 o2 = lds_f32x2(ob + lane * 8);
-        h[0] = o2.x + bv[0];
-        h[1] = o2.y + bv[1];
+        const float left = __shfl_up_sync(kFull, v, 1);
+        const float sa = ((w1 >> 9) & 1u) ? left + za : za;
+        const int l0 = (int)((w1 >> 16) & 31u), l1 = (int)((w1 >> 22) & 31u);
+        const float a0 = __shfl_sync(kFull, sa, l0), b0 = __shfl_sync(kFull, v, l0);
+        const float a1 = __shfl_sync(kFull, sa, l1), b1 = __shfl_sync(kFull, v, l1);
+        const float x0 = ((w1 >> 21) & 1u) ? b0 : a0;
+        const float x1 = ((w1 >> 27) & 1u) ? b1 : a1;
+        h[0] = ((w1 >> 11) & 1u ? x0 : 0.f) + bv[0];
+        h[1] = ((w1 >> 12) & 1u ? x1 : 0.f) + bv[1];
     }
 }
 
@@ -850,8 +848,9 @@ __device__ __forceinline__ void step_perm(float (&h)[NPL], const float (&dv)[NPL
     }
 }
 
-// One PD step: LV = 0 selects the permutation step (buffer by step parity),
-// otherwise the segment-table step with LV shuffle levels.
+// One PD step: LV = 0 selects the permutation step, otherwise the
+// segment-table step with LV shuffle levels; both take the exchange buffer
+// of the step's parity (pb or ob).
 template <int NPL, int LV>
 __device__ __forceinline__ void pd_step(float (&h)[NPL], const float (&dv)[NPL],
                                         const float (&bv)[NPL], uint32_t pb, uint32_t ob,
@@ -859,7 +858,7 @@ __device__ __forceinline__ void pd_step(float (&h)[NPL], const float (&dv)[NPL],
     if constexpr (LV == 0)
         step_perm<NPL>(h, dv, bv, parity ? ob : pb, e, lane);
     else
-        step_seg<NPL, LV>(h, dv, bv, pb, ob, e, lane);
+        step_seg<NPL, LV>(h, dv, bv, parity ? ob : pb, e, lane);
 }
 
 // Step variant for a launch: 0 when every map is a permutation, else the

@@ -230,16 +230,24 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
         const bool has1 = s_off[wib][eb + 1] > s_off[wib][eb];
         w0 = (uint32_t)(sa * 4) | (uint32_t)(sb * 4) << 8 | (uint32_t)(ga * 4) << 16 |
              (uint32_t)(gb * 4) << 24;
+        // where this lane's own targets' sums end up: the entry that ends
+        // each target's segment (lane = entry / 2; entry odd: a b entry)
+        const int e0 = has0 ? s_off[wib][ea + 1] - 1 : 0;
+        const int e1 = has1 ? s_off[wib][eb + 1] - 1 : 0;
         w1 = (uint32_t)dist | (ab_same ? 1u : 0u) << 8 | (a_cont ? 1u : 0u) << 9 |
-             (b_end ? 1u : 0u) << 10 | (has0 ? 1u : 0u) << 11 | (has1 ? 1u : 0u) << 12;
+             (b_end ? 1u : 0u) << 10 | (has0 ? 1u : 0u) << 11 | (has1 ? 1u : 0u) << 12 |
+             (uint32_t)(e0 >> 1) << 16 | (uint32_t)(e0 & 1) << 21 | (uint32_t)(e1 >> 1) << 22 |
+             (uint32_t)(e1 & 1) << 27;
     } else {
         const int e = lane;
         const int sb = s_src[wib][e], gb = s_tgt[wib][e];
         const bool b_end = e + 1 >= N || s_tgt[wib][e + 1] != gb;
         dist = lane - s_off[wib][gb];
         const bool has0 = s_off[wib][e + 1] > s_off[wib][e];
+        const int e0 = has0 ? s_off[wib][e + 1] - 1 : 0;   // entry ending this lane's target
         w0 = (uint32_t)(sb * 4) << 8 | (uint32_t)(gb * 4) << 24;
-        w1 = (uint32_t)dist | (b_end ? 1u : 0u) << 10 | (has0 ? 1u : 0u) << 11;
+        w1 = (uint32_t)dist | (b_end ? 1u : 0u) << 10 | (has0 ? 1u : 0u) << 11 |
+             (uint32_t)e0 << 16 | 1u << 21;
     }
     seg[m * 32 + lane] = make_uint2(w0, w1);
     const int md = __reduce_max_sync(kFull, dist);
