@@ -60,10 +60,12 @@ def test_select_bit_exact(idx, over):
 
 
 @pytest.mark.parametrize("H,K,D", [(16, 16, 128), (2, 8, 64), (1, 4, 16), (4, 32, 32),
-                                   (3, 2, 48)])
+                                   (3, 2, 48), (4, 16, 192), (2, 8, 256), (5, 1, 64)])
 def test_select_tensor_core_shapes_bit_exact(H, K, D):
     """bf16 u with K a power of two takes the tcgen05 path (certified
-    argmax, exact fma-chain recompute near ties)."""
+    argmax, exact fma-chain recompute near ties); D a multiple of 64 uses
+    the 128-byte swizzled operands (1 to 4 atoms), other D the unswizzled
+    ones; K = 1 has a single candidate per head."""
     rng = np.random.default_rng(H * 1000 + K * 10 + D)
     B, L = 2, 333
     u = gen.round_bf16(rng.standard_normal((B, L, D)).astype(np.float32))
