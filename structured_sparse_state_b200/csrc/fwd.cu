@@ -263,10 +263,11 @@ struct ScatterScratch {
 
 // out[i] = V[i] + sum_{j : P[j] = i} Z[j] over the warp's 64 elements, for an
 // arbitrary index map (maps composed over a chunk often send most columns to
-// one target, so no bounded fan-in is assumed).  Deterministic: the entries
-// are sorted by target (ascending j within a target, by counting ranks), and
+// one target, so no bounded fan-in is assumed).  Deterministic either way:
+// a small image sums each target by a warp butterfly; otherwise the entries
+// are sorted by target (ascending j within a target, by counting ranks) and
 // each target's entries are summed by a segmented scan over the sorted
-// order, whose tree of additions depends only on the map.
+// order.  The trees of additions depend only on the map.
 __device__ __forceinline__ void warp_scatter(const int (&P)[2], const float (&Z)[2],
                                              const float (&V)[2], float (&out)[2],
                                              ScatterScratch &sc, int lane, bool perm) {
@@ -281,6 +282,41 @@ __device__ __forceinline__ void warp_scatter(const int (&P)[2], const float (&Z)
         out[1] = sc.val[lane + 32] + V[1];
         __syncwarp();
         return;
+    }
+    {
+        // Maps composed over whole chunks usually send all columns to one or
+        // two targets: for up to kSmallImage distinct targets, each target's
+        // sum is a warp butterfly over the entries aimed at it (smallest
+        // target first).  A larger image falls through to the sort below.
+        constexpr int kSmallImage = 4;
+        bool p0 = true, p1 = true;   // entries not yet summed
+        float s0 = 0.f, s1 = 0.f;   // sums of this lane's own targets lane, lane + 32
+        bool got0 = false, got1 = false;
+        for (int round = 0; round < kSmallImage; ++round) {
+            const unsigned key = min(p0 ? (unsigned)P[0] : 0xffffu, p1 ? (unsigned)P[1] : 0xffffu);
+            const unsigned t = __reduce_min_sync(kFull, key);
+            if (t == 0xffffu) break;
+            float c = (p0 && (unsigned)P[0] == t) ? Z[0] : 0.f;
+            if (p1 && (unsigned)P[1] == t) c += Z[1];
+#pragma unroll
+            for (int o = 16; o; o >>= 1) c += __shfl_xor_sync(kFull, c, o);
+            if ((int)(t & 31u) == lane) {
+                if (t < 32u) {
+                    s0 = c;
+                    got0 = true;
+                } else {
+                    s1 = c;
+                    got1 = true;
+                }
+            }
+            p0 = p0 && (unsigned)P[0] != t;
+            p1 = p1 && (unsigned)P[1] != t;
+        }
+        if (!__any_sync(kFull, p0 || p1)) {
+            out[0] = (got0 ? s0 : 0.f) + V[0];
+            out[1] = (got1 ? s1 : 0.f) + V[1];
+            return;
+        }
     }
     const unsigned lt = (1u << lane) - 1u;
     const unsigned m0 = __match_any_sync(kFull, P[0]);
