@@ -2,7 +2,7 @@
  * pdssm.h -- C ABI of the B200 (sm_100a) Flash PD-SSM scan library.
  *
  * The recurrence (Flash PD-SSM technical summary, Methodology §1 "hard
- * selection", one-hot column selector; benchmark spec of the path):
+ * selection", one-hot column selector):
  *
  *     k_t    = argmax_k (W_sel u_t)_k
  *     h_t    = P_{k_t} diag(d_t) h_{t-1} + b_t,   P_k[pi_k(j), j] = 1
@@ -24,6 +24,13 @@
  *    device-side problems are recorded in the workspace status word and read
  *    back with pdssm_ws_status().  pdssm_validate() and pdssm_ws_status()
  *    synchronise the stream.
+ *  * Consecutive kernels may overlap (programmatic dependent launch): a
+ *    kernel of this library can start while the previous kernel on the
+ *    stream, when that is one of this library's, is finishing.  Before it
+ *    waits for that kernel it reads only the inputs u, W_sel, d, b, c of its
+ *    own call, so these must not be outputs of the immediately preceding
+ *    call; inputs written by the caller's own kernels or copies are safe
+ *    (those complete first).
  *  * Shapes:   u [B][L][D_in]        W_sel [H][K][D_in] (fp32)
  *              pi_dict: entry (h,k,j) at pi_dict[h*pi_head_stride + k*N + j]
  *                       (pi_head_stride = 0: one [K][N] dictionary for all heads,
