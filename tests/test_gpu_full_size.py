@@ -1,0 +1,137 @@
+"""GPU parity at the full benchmark sizes, in the launch configuration the
+benchmark times: the same entry points with preallocated workspace and
+outputs, two steps issued back to back on one stream (consecutive calls
+overlap through programmatic dependent launch), then a sample of (batch,
+head) rows checked against the oracle.  Every (batch, head) sequence is an
+independent recurrence, so the oracle recomputes only the sampled rows, from
+the generator's inputs (its selection indices included: nothing the CUDA
+path produced is fed to the oracle).
+
+Workloads (their sizes are the generator's defaults):
+  * bf16 selection + forward: B=8, H=16, L=16384, N=64, K=16, D_in=128,
+    chunk 128, uniform random maps;
+  * stiff impulse forward: B=1, H=32, L=131072, N=32, K=8, chunk 256,
+    permutations, d log-uniform in [1e-4, 1];
+  * fp32 forward + adjoint: B=2, H=16, L=65536, N=64, K=16, chunk 128."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import pdssm_inputs as gen
+import structured_sparse_state_b200 as pd
+from parity_util import TOL_F32, floored_relerr, sample_rows, to_device, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _need_gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+
+
+def _rows(B, H, n, seed):
+    """The first and last sequence plus n seeded ones."""
+    return sorted(set([(0, 0), (B - 1, H - 1)] + sample_rows(B, H, n, seed)))
+
+
+def _slice(x, b, h):
+    return None if x is None else x[b:b + 1, h:h + 1]
+
+
+def _buffers(inp, chunk, grad):
+    cfg = inp.cfg
+    B, H, L, N, K = cfg["B"], cfg["H"], cfg["L"], cfg["N"], cfg["K"]
+    dev = torch.device("cuda")
+    ws = pd.make_workspace(B, H, L, N, K, chunk, dev, False, grad)
+    y = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    h_last = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    k_buf = torch.empty((B, H, L), dtype=torch.int32, device=dev)
+    gouts = None
+    if grad:
+        gouts = tuple(torch.empty((B, H, L, N), dtype=torch.float32, device=dev)
+                      for _ in range(3)) + (torch.empty((B, H, N), dtype=torch.float32,
+                                                        device=dev),)
+    return ws, y, h_last, k_buf, gouts
+
+
+def _run_steps(inp, t, chunk, select, grad, steps=2):
+    """The benchmark's step (selection if the workload selects, forward,
+    adjoint if it has one), issued `steps` times without a synchronisation."""
+    ws, y, h_last, k_buf, gouts = _buffers(inp, chunk, grad)
+    stream = torch.cuda.current_stream()
+    for _ in range(steps):
+        k = pd.pdssm_select(t["u"], t["W"], k_out=k_buf, stream=stream) if select else t["k"]
+        pd.pdssm_scan_fwd(t["pi"], k, t["d"], t["b"], t["c"], t["h0"], chunk=chunk, ws=ws, y=y,
+                          h_last=h_last, for_bwd=grad, stream=stream)
+        if grad:
+            pd.pdssm_scan_bwd(t["pi"], k, t["d"], t["b"], t["c"], t["h0"], t["g_y"], ws,
+                              chunk=chunk, out=gouts, stream=stream)
+    torch.cuda.synchronize()
+    assert pd.pdssm_ws_status(ws) == 0
+    return k, y, h_last, gouts
+
+
+def test_full_size_bf16_selection_and_forward():
+    cfg = gen.workload(2)
+    inp = gen.generate(cfg)
+    t = to_device(inp)
+    k, y, h_last, _ = _run_steps(inp, t, cfg["chunk"], select=True, grad=False)
+    assert torch.isfinite(y).all() and torch.isfinite(h_last).all()
+    tol = tol_for(inp)
+    for b, h in _rows(cfg["B"], cfg["H"], 4, seed=2):
+        k_ref = oracle.select(inp.u[b:b + 1], inp.W[h:h + 1])          # [1, 1, L]
+        assert (k[b, h].cpu().numpy() == k_ref[0, 0]).all(), (b, h)
+        y_ref, hl_ref = oracle.scan_fwd(inp.pi, k_ref, _slice(inp.d, b, h), _slice(inp.b, b, h),
+                                        _slice(inp.c, b, h), _slice(inp.h0, b, h))
+        assert floored_relerr(y[b, h].cpu().numpy(), y_ref[0, 0]) <= tol, (b, h)
+        assert floored_relerr(h_last[b, h].cpu().numpy(), hl_ref[0, 0]) <= tol, (b, h)
+
+
+def _stiff_check(a, r, where):
+    """Elementwise relative error 1e-5 where the oracle's value is at least
+    1e-30 in magnitude, and magnitude at most 1e-30 elsewhere; returns how
+    many entries took the relative test."""
+    a = a.cpu().numpy().astype(np.float64)
+    big = np.abs(r) >= 1e-30
+    if big.any():
+        assert np.max(np.abs(a[big] - r[big]) / np.abs(r[big])) <= 1e-5, where
+    assert np.max(np.abs(a[~big]), initial=0.0) <= 1e-30, where
+    return int(big.sum())
+
+
+def test_full_size_stiff_impulse_forward():
+    """The impulse's mass decays along one path through 131072 steps, so most
+    of y and the final state underflow: checked elementwise (_stiff_check)."""
+    cfg = gen.workload(3)
+    inp = gen.generate(cfg)
+    t = to_device(inp)
+    _, y, h_last, _ = _run_steps(inp, t, cfg["chunk"], select=False, grad=False)
+    assert torch.isfinite(y).all() and torch.isfinite(h_last).all()
+    n_big = 0
+    for b, h in _rows(cfg["B"], cfg["H"], 5, seed=3):
+        y_ref, hl_ref = oracle.scan_fwd(inp.pi, _slice(inp.k, b, h), _slice(inp.d, b, h),
+                                        _slice(inp.b, b, h), _slice(inp.c, b, h), None)
+        n_big += _stiff_check(y[b, h], y_ref[0, 0], (b, h))
+        _stiff_check(h_last[b, h], hl_ref[0, 0], (b, h))
+    assert n_big > 8
+
+
+def test_full_size_fp32_forward_and_adjoint():
+    cfg = gen.workload(4)
+    inp = gen.generate(cfg)
+    t = to_device(inp)
+    _, y, h_last, g = _run_steps(inp, t, cfg["chunk"], select=False, grad=True)
+    for x in (y, h_last) + g:
+        assert torch.isfinite(x).all()
+    for b, h in _rows(cfg["B"], cfg["H"], 6, seed=4):
+        args = (inp.pi, _slice(inp.k, b, h), _slice(inp.d, b, h), _slice(inp.b, b, h),
+                _slice(inp.c, b, h), _slice(inp.h0, b, h))
+        y_ref, hl_ref = oracle.scan_fwd(*args)
+        assert floored_relerr(y[b, h].cpu().numpy(), y_ref[0, 0]) <= TOL_F32, (b, h)
+        assert floored_relerr(h_last[b, h].cpu().numpy(), hl_ref[0, 0]) <= TOL_F32, (b, h)
+        g_ref = oracle.scan_bwd(*args, _slice(inp.g_y, b, h))
+        for name, a, r in zip(("g_b", "g_d", "g_c", "g_h0"), g, g_ref):
+            e = floored_relerr(a[b, h].cpu().numpy(), r[0, 0])
+            assert e <= TOL_F32, f"{name} error {e} at {(b, h)}"
