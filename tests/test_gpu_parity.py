@@ -74,6 +74,21 @@ def test_select_tensor_core_shapes_bit_exact(H, K, D):
     assert (k == oracle.select(u, W)).all()
 
 
+@pytest.mark.parametrize("bf16", [True, False])
+def test_select_largest_sizes(bf16):
+    """K = 32 and D_in = 256, the boundary's limits, with H*K = 256 scores per
+    row (the tensor-core kernel's operands would not fit its shared memory,
+    so the fma-chain kernel decides); bit-exact for bf16 and fp32 u."""
+    rng = np.random.default_rng(256)
+    H, K, D, B, L = 8, 32, 256, 2, 300
+    u = rng.standard_normal((B, L, D)).astype(np.float32)
+    if bf16:
+        u = gen.round_bf16(u)
+    W = (rng.standard_normal((H, K, D)) / np.sqrt(D)).astype(np.float32)
+    k = pd.pdssm_select(dev(u, bf16=bf16), dev(W)).cpu().numpy()
+    assert (k == oracle.select(u, W)).all()
+
+
 def test_select_near_ties_take_the_exact_path():
     """Rows of W that differ by ~1e-6 make most top-2 gaps smaller than the
     certification bound, so the exact fma chains decide."""
@@ -241,6 +256,55 @@ def test_forward_fan_in_around_slot_capacity(fan, N):
     inp.pi = pi
     check_fwd(inp, chunk=50)
     check_bwd(inp, chunk=50)
+
+
+def _lane_distance(row, npl):
+    """Largest distance in lanes between the first and the last source of one
+    target, when the sources, ordered by target, are dealt npl per lane."""
+    order = np.argsort(row, kind="stable")
+    tg = row[order]
+    md, s = 0, 0
+    while s < len(tg):
+        e = s
+        while e + 1 < len(tg) and tg[e + 1] == tg[s]:
+            e += 1
+        md = max(md, e // npl - s // npl)
+        s = e + 1
+    return md
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("N,fan,levels", [
+    (32, 2, 1), (32, 3, 2), (32, 5, 3), (32, 9, 5),
+    (64, 3, 1), (64, 5, 2), (64, 9, 3), (64, 17, 5)])
+def test_segment_step_shuffle_levels(N, fan, levels, dtype):
+    """Maps that are permutations except for one target receiving `fan`
+    sources.  The run of that target's sources spans a number of lanes that
+    decides how many shuffle levels the segmented sum of the state update
+    takes (1, 2, 3 or 5 levels for runs spanning under 2, 4, 8 or 32
+    lanes); each case lands in the class named by `levels`."""
+    inp = small(70 + N + fan, 2, 2, 400, N, 5, dtype=dtype)
+    rng = np.random.default_rng(N * 100 + fan)
+    pi = inp.pi.copy()
+    for kk in range(pi.shape[0]):
+        row = rng.permutation(N).astype(np.int32)
+        sel = rng.choice(N, size=fan, replace=False)
+        row[sel] = row[sel[0]]          # that target now has exactly `fan` sources
+        pi[kk] = row
+    inp.pi = pi
+    md = max(_lane_distance(r, N // 32) for r in pi)
+    assert {1: md < 2, 2: 2 <= md < 4, 3: 4 <= md < 8, 5: md >= 8}[levels], md
+    check_fwd(inp, chunk=64)
+    check_bwd(inp, chunk=64)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_largest_dictionary_per_head(dtype):
+    """The largest sizes the boundary accepts for the scan: N = 64 and
+    K = 32 maps per head, a dictionary per head, a ragged last chunk."""
+    inp = small(80, 2, 3, 777, 64, 32, dtype=dtype, per_head=True)
+    check_fwd(inp, chunk=128)
+    check_bwd(inp, chunk=128)
 
 
 @pytest.mark.parametrize("N", [8, 30, 64])
