@@ -18,7 +18,9 @@
  * --------------------------
  *  * All tensor pointers are DEVICE pointers to caller-owned, row-major,
  *    contiguous memory.  The library allocates nothing and keeps no state
- *    between calls; scratch lives in the caller's workspace `ws`.
+ *    between calls; scratch lives in the caller's workspace `ws` (the one
+ *    exception, pdssm_scan_fwd_noalloc, uses a fixed array inside the
+ *    library instead, described there).
  *  * Calls are asynchronous on `stream` (a cudaStream_t; NULL = the legacy
  *    default stream).  A returned PDSSM_OK means the kernels were launched;
  *    device-side problems are recorded in the workspace status word and read
