@@ -63,3 +63,19 @@ def test_l2_note_tells_resident_from_streamed_inputs():
     assert "larger than L2" in bench.l2_note(gen.workload(2))
     assert "larger than L2" in bench.l2_note(gen.workload(3))
     assert "fit in L2" in bench.l2_note(gen.workload(0))
+
+
+def test_oracle_timing_on_one_and_several_threads():
+    """The cpu_baseline leg: the oracle on one thread and on a thread pool
+    over (batch, head) sequences; both count the same pieces of work."""
+    sys.path.insert(0, ROOT)
+    import bench
+    cfg = gen.workload(4, B=1, H=4, L=600)
+    inp = gen.generate(cfg)
+    v1, s1, c1 = bench.time_oracle(cfg, inp, 30.0)
+    v2, s2, c2 = bench.time_oracle(cfg, inp, 30.0, threads=3)
+    assert v1 > 0 and v2 > 0 and (c1, c2) == (1, 3)
+    # the whole small workload fits the budget: every sequence is timed once
+    updates = cfg["B"] * cfg["H"] * cfg["L"] * cfg["N"]
+    assert f"({updates} state updates" in s1 and f"({updates} state updates" in s2
+    assert "single thread" in s1 and "3 threads" in s2
