@@ -15,6 +15,8 @@ Prints one JSON line (rank 0).  ``value`` is whole-job state updates
 with inputs copied from pinned host memory and y / h_last copied back inside
 the timed region.  Multi-GPU runs (torchrun) give every rank its own batch
 (weak scaling, no data-path collective); time is the max over ranks.
+``cpu_baseline`` times the CPU oracle on one host thread and on all of them;
+``--impl reference`` prints the oracle's line (all host cores) instead.
 """
 import argparse
 import hashlib
@@ -496,10 +498,12 @@ def run_reference(args, cfg):
         return None
     inp = gen.generate(cfg)
     budget = max(1.0, 60.0 / max(1, args.steps + args.warmup))
+    threads = len(os.sched_getaffinity(0))   # every host core this process may use
     vals = []
     sample = None
+    cores = threads
     for i in range(args.warmup + args.steps):
-        v, sample, cores = time_oracle(cfg, inp, budget)
+        v, sample, cores = time_oracle(cfg, inp, budget, threads=threads)
         if i >= args.warmup:
             vals.append(v)
     v = float(np.mean(vals)) if vals else 0.0
@@ -510,7 +514,7 @@ def run_reference(args, cfg):
             "scaling": "weak", "vs_baseline": None,
             "dtype": "f64 (oracle arithmetic)", "data": "synthetic (seeded PCG64)",
             "config": config_json(cfg, 1),
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
                              "sample": f"per step: {sample}"},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
             "gpu_launches": 0}
