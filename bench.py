@@ -54,6 +54,8 @@ def parse():
                     help="override B per GPU (small cases for profiler captures)")
     ap.add_argument("--seq-len", type=int, default=0,
                     help="override L (small cases for profiler captures)")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the stiff and forward+adjoint workloads of the default run")
     return ap.parse_args()
 
 
@@ -284,6 +286,33 @@ def run_ours(args, cfg):
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     dev = torch.device("cuda", torch.cuda.current_device())
+    out = measure(args, cfg, torch, pd, dev, world, rank, dist, args.steps,
+                  with_e2e=not args.no_e2e, with_cpu=not args.no_cpu)
+    # the other two benchmark workloads of the method, on the default run
+    # at one GPU: the long stiff forward and the forward + exact adjoint
+    if rank == 0 and out is not None and world == 1 and not args.no_extra and \
+            workload_index(args.workload) == DEFAULT_WORKLOAD and not (args.batch or args.seq_len):
+        out["extra"] = {}
+        for idx in EXTRA_WORKLOADS:
+            xcfg = gen.workload(idx)
+            torch.cuda.empty_cache()
+            x = measure(args, xcfg, torch, pd, dev, 1, 0, dist, max(8, args.steps // 4),
+                        with_e2e=False, with_cpu=not args.no_cpu, cpu_threads_only=True)
+            keep = ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "config",
+                    "roofline", "phases_ms", "clocks", "gpu_launches", "cpu_baseline")
+            out["extra"][xcfg["name"]] = {k: x[k] for k in keep if k in x}
+    if world > 1:
+        dist.destroy_process_group()
+    return out
+
+
+EXTRA_WORKLOADS = (3, 4)
+
+
+def measure(args, cfg, torch, pd, dev, world, rank, dist, K_steps, with_e2e, with_cpu,
+            cpu_threads_only=False):
+    """Times K_steps steps of `cfg` (the whole forward path, plus the adjoint
+    when the workload has one) and returns the JSON object of rank 0."""
     inp = gen.generate(cfg)
     bf = cfg["dtype"] == "bf16"
 
@@ -315,27 +344,50 @@ def run_ours(args, cfg):
                  torch.empty_like(d, dtype=torch.float32),
                  torch.empty((B, H, N), dtype=torch.float32, device=dev))
     stream = torch.cuda.current_stream()
-    launches_per_step = (1 if select else 0) + 4 + (3 if grad else 0)
 
-    ev = None
+    # kernel-level timing on a sample of the timed steps: events recorded
+    # between the kernels of those steps (the other steps run without them,
+    # so their kernels may overlap through programmatic dependent launch)
+    traced = {}
+    launches = {"n": 0}
 
     def step(i=None):
-        k = pd.pdssm_select(u, W, k_out=k_buf, stream=stream) if select else k_given
-        # the scan's own events are recorded on a sample of the timed steps:
-        # an event between two kernels keeps the next one from starting
-        # before the previous finishes (programmatic dependent launch)
-        timed = ev is not None and i in ev
-        if timed:
-            ev[i][0].record(stream)
-        pd.pdssm_scan_fwd(pi, k, d, b, c, h0, chunk=chunk, ws=ws, y=y, h_last=h_last,
-                          for_bwd=grad, stream=stream)
-        if timed:
-            ev[i][1].record(stream)
+        tr = traced.get(i)
+        if select:
+            if tr is not None:
+                tr["sel"][0].record(stream)
+            k = pd.pdssm_select(u, W, k_out=k_buf, stream=stream)
+            if tr is not None:
+                tr["sel"][1].record(stream)
+            launches["n"] += 1
+        else:
+            k = k_given
+        if tr is not None:
+            tr["fwd_res"] = pd.pdssm_scan_fwd_traced(pi, k, d, b, c, h0, chunk, ws, y, h_last,
+                                                     tr["fwd"], stream=stream)
+        else:
+            pd.pdssm_scan_fwd(pi, k, d, b, c, h0, chunk=chunk, ws=ws, y=y, h_last=h_last,
+                              for_bwd=grad, stream=stream)
+        launches["n"] += launches_fwd
         if grad:
-            pd.pdssm_scan_bwd(pi, k, d, b, c, h0, g_y, ws, chunk=chunk, out=gouts,
-                              stream=stream)
+            if tr is not None:
+                tr["bwd_res"] = pd.pdssm_scan_bwd_traced(pi, k, d, b, c, h0, g_y, ws, chunk,
+                                                         gouts, tr["bwd"], stream=stream)
+            else:
+                pd.pdssm_scan_bwd(pi, k, d, b, c, h0, g_y, ws, chunk=chunk, out=gouts,
+                                  stream=stream)
+            launches["n"] += launches_bwd
 
-    # warm-up and a status check of the path
+    # kernels per call, read from one traced call during warm-up
+    probe = {"sel": pd.make_trace_events(2), "fwd": pd.make_trace_events(),
+             "bwd": pd.make_trace_events()}
+    traced[-1] = probe
+    launches_fwd = launches_bwd = 0
+    step(-1)
+    torch.cuda.synchronize()
+    launches_fwd = len(probe["fwd_res"]())
+    launches_bwd = len(probe["bwd_res"]()) if grad else 0
+    del traced[-1]
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -343,10 +395,11 @@ def run_ours(args, cfg):
     if st != 0:
         raise RuntimeError(f"device status {st} after warm-up")
 
-    K_steps = args.steps
     sampled = [i for i in range(K_steps) if K_steps < 4 or i % 4 == 3]
-    ev = {i: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-          for i in sampled}
+    for i in sampled:
+        traced[i] = {"sel": pd.make_trace_events(2), "fwd": pd.make_trace_events(),
+                     "bwd": pd.make_trace_events()}
+    launches["n"] = 0
     start = torch.cuda.Event(enable_timing=True)
     end = torch.cuda.Event(enable_timing=True)
     if world > 1:
@@ -361,7 +414,23 @@ def run_ours(args, cfg):
     if world > 1:
         dist.barrier()
     ms_total = start.elapsed_time(end)
-    scan_ms = sum(a.elapsed_time(bq) for a, bq in ev.values()) / len(ev)
+    # per-kernel means over the sampled steps
+    phases = {}
+    scan_samples = []
+    for i in sampled:
+        tr = traced[i]
+        per = []
+        if select:
+            per.append(("select", tr["sel"][0].elapsed_time(tr["sel"][1])))
+        fwd = tr["fwd_res"]()
+        scan_samples.append(sum(ms for _, ms in fwd))
+        per += fwd
+        if grad:
+            per += [(n, ms) for n, ms in tr["bwd_res"]()]
+        for n, ms in per:
+            phases.setdefault(n, []).append(ms)
+    phases_ms = {n: round(float(np.mean(v)), 5) for n, v in phases.items()}
+    scan_ms = float(np.mean(scan_samples))
     t = torch.tensor([ms_total], dtype=torch.float64, device=dev)
     if world > 1:
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -372,45 +441,52 @@ def run_ours(args, cfg):
 
     # end to end: pinned host inputs -> device -> path -> y, h_last back to host
     e2e = None
-    if not args.no_e2e:
+    if with_e2e:
         e2e = run_e2e(args, cfg, pd, torch, dev, stream, inp, bf, pi, W, world, dist)
 
     if rank != 0:
-        if world > 1:
-            dist.destroy_process_group()
         return None
 
     peaks, peak_kind = measured_peaks()
     fwd_bytes, bwd_bytes, sel_bytes = algorithmic_bytes(cfg)
     achieved = fwd_bytes / (scan_ms * 1e-3) / 1e9
-    roofline = {"kernel": "pdssm_scan_fwd (plans + phase A + phase B + phase C)",
+    fwd_kernels = [n for n, _ in probe["fwd_res"]()]
+    roofline = {"kernel": "pdssm_scan_fwd (" + " + ".join(fwd_kernels) + ")",
                 "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": ncu_traffic(cfg["name"]),
                 "algorithmic_bytes_per_launch": fwd_bytes,
                 "launch_ms": round(scan_ms, 5),
-                "launch_samples": len(ev),
-                "select_ms": round(ms_step - scan_ms, 5) if select and not grad else None}
+                "launch_samples": len(sampled)}
+    if grad:
+        bwd_ms = sum(v for n, v in phases_ms.items() if n.startswith("bwd"))
+        roofline["bwd"] = {"kernel": "pdssm_scan_bwd", "algorithmic_bytes_per_launch": bwd_bytes,
+                           "launch_ms": round(bwd_ms, 5),
+                           "achieved": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9, 1),
+                           "frac": round(bwd_bytes / (bwd_ms * 1e-3) / 1e9 / peaks["hbm_gbs"], 4)}
     out = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
            "steps": K_steps, "warmup": args.warmup, "ms_per_step": ms_step,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "bf16" if bf else "f32", "data": "synthetic (seeded PCG64)",
-           "config": config_json(cfg, world), "roofline": roofline,
-           "gpu_launches": launches_per_step * K_steps, "clocks": clk.report(),
+           "config": config_json(cfg, world), "roofline": roofline, "phases_ms": phases_ms,
+           "gpu_launches": launches["n"], "clocks": clk.report(),
            "e2e": e2e}
-    if not args.no_cpu and world == 1:
-        v, sample, cores = time_oracle(cfg, inp, args.cpu_seconds)
-        out["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
-                               "sample": sample}
+    if with_cpu and world == 1:
         ncores = len(os.sched_getaffinity(0))
+        budget = args.cpu_seconds / (2 if cpu_threads_only else 1)
+        if not cpu_threads_only:
+            v, sample, cores = time_oracle(cfg, inp, budget)
+            out["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                   "sample": sample}
         if ncores > 1:
             # the same oracle on every host core this process may use
-            va, samplea, ca = time_oracle(cfg, inp, args.cpu_seconds, threads=ncores)
-            out["cpu_baseline"]["all_cores"] = {"value": va, "unit": UNIT, "cores": ca,
-                                                "sample": samplea}
-    if world > 1:
-        dist.destroy_process_group()
+            va, samplea, ca = time_oracle(cfg, inp, budget, threads=ncores)
+            allc = {"value": va, "unit": UNIT, "cores": ca, "sample": samplea}
+            if cpu_threads_only:
+                out["cpu_baseline"] = dict(allc, kind="oracle")
+            else:
+                out["cpu_baseline"]["all_cores"] = allc
     return out
 
 

@@ -111,11 +111,51 @@ pdssm_status pdssm_select(const pdssm_dims *dims, const void *u,
                           pdssm_dtype u_dtype, const float *W_sel,
                           int32_t *k_out, void *stream);
 
+/* Arithmetic route of the hard selection (pdssm_select_with). */
+typedef enum pdssm_select_method {
+    PDSSM_SELECT_AUTO = 0,         /* tensor cores where they apply, else the fma chain */
+    PDSSM_SELECT_FMA_CHAIN = 1,    /* the fp32 fma chain on the CUDA cores, any shape */
+    PDSSM_SELECT_TENSOR_CORE = 2   /* tcgen05 logits + certified argmax; bf16 u, D_in a
+                                      multiple of 16, K a power of two, H*K <= 256,
+                                      else PDSSM_ERR_UNSUPPORTED */
+} pdssm_select_method;
+
+/*
+ * pdssm_select with an explicit arithmetic route.  Every route returns the
+ * same k, bit for bit: the tensor-core route bounds the error of its logits
+ * (see pdssm_select_tc_logits), keeps every index within twice that bound of
+ * the top logit as a candidate, and decides several candidates with the
+ * contract's fma chains.  `method` is a pdssm_select_method.
+ */
+pdssm_status pdssm_select_with(const pdssm_dims *dims, const void *u,
+                               pdssm_dtype u_dtype, const float *W_sel,
+                               int32_t *k_out, int method, void *stream);
+
+/*
+ * Test hook of the tensor-core selection: runs pdssm_select_with(...,
+ * PDSSM_SELECT_TENSOR_CORE) on bf16 u and also writes, per row r = b*L + t,
+ *     logits_out[r][h*K + k] = the tensor-core logit (bf16 u times the
+ *                              bf16 hi and lo parts of W_sel, fp32 sums),
+ *     scale_out[r][h]        = ||u_r||_2 * max_k ||W_sel[h][k]||_2, rounded up.
+ * The selection treats |logit - exact sum| <= (D_in 2^-21 + 2^-16) scale as
+ * the tensor cores' error bound; this hook lets a test check that bound
+ * against exact sums.  logits_out: device fp32 [B*L][H*K]; scale_out: device
+ * fp32 [B*L][H].
+ */
+pdssm_status pdssm_select_tc_logits(const pdssm_dims *dims, const void *u,
+                                    const float *W_sel, int32_t *k_out,
+                                    float *logits_out, float *scale_out,
+                                    void *stream);
+
 /*
  * Chunked forward scan (Methodology §3).  Runs phase A0 (sanitised copy of
  * the dictionary), A (per chunk: local readout of the state started from zero,
  * closed PD transfer Pi_c, Delta_c, v_c), B (carry prefix scan H_c, h_last)
- * and C (carry correction of the readout y).  Writes y [B][H][L] and, when
+ * and C (carry correction of the readout y).  For N = 32 or 64 with 16-byte
+ * aligned rows the three phases run as one kernel (one CTA per chunk, in
+ * chunk order: phase A on sub-chunks, their transfers composed in the CTA,
+ * the carry taken from the predecessors by decoupled look-back, then phase
+ * C); other shapes run them as three kernels.  Writes y [B][H][L] and, when
  * non-NULL, h_last [B][H][N] = h_{L-1} (h0 when L = 0).  h0 may be NULL
  * (zero initial state).  ws must hold pdssm_workspace_bytes(dims,
  * pi_head_stride, chunk, 0) bytes, 256-byte aligned; its contents are
@@ -150,6 +190,45 @@ pdssm_status pdssm_scan_bwd(const pdssm_dims *dims, const int32_t *pi_dict,
                             void *stream);
 
 /*
+ * Kernel-level timing of one call (a measurement aid, not part of the
+ * method).  The caller supplies created cudaEvent_t handles; the traced
+ * calls record events[i] on the stream just before the i-th kernel they
+ * launch and events[n_kernels] after the last, and name each kernel in
+ * names[i] (static strings).  Events recorded between the kernels keep them
+ * from overlapping (no programmatic dependent launch across an event), so
+ * traced calls run slightly slower than untraced ones.
+ */
+#define PDSSM_TRACE_MAX_KERNELS 8
+typedef struct pdssm_trace {
+    void *const *events;   /* in: max_events cudaEvent_t handles */
+    int max_events;        /* in: >= 2 */
+    int n_kernels;         /* out */
+    const char *names[PDSSM_TRACE_MAX_KERNELS];   /* out */
+} pdssm_trace;
+
+/* pdssm_scan_fwd, recording `trace` (see above).  Same results. */
+pdssm_status pdssm_scan_fwd_traced(const pdssm_dims *dims,
+                                   const int32_t *pi_dict,
+                                   int64_t pi_head_stride, const int32_t *k,
+                                   const void *d, const void *b,
+                                   const void *c, pdssm_dtype in_dtype,
+                                   const float *h0, float *y, float *h_last,
+                                   int64_t chunk, void *ws, size_t ws_bytes,
+                                   void *stream, pdssm_trace *trace);
+
+/* pdssm_scan_bwd, recording `trace` (see above).  Same results. */
+pdssm_status pdssm_scan_bwd_traced(const pdssm_dims *dims,
+                                   const int32_t *pi_dict,
+                                   int64_t pi_head_stride, const int32_t *k,
+                                   const void *d, const void *b,
+                                   const void *c, pdssm_dtype in_dtype,
+                                   const float *h0, const float *g_y,
+                                   const float *g_hlast, float *g_b,
+                                   float *g_d, float *g_c, float *g_h0,
+                                   int64_t chunk, void *ws, size_t ws_bytes,
+                                   void *stream, pdssm_trace *trace);
+
+/*
  * pdssm_scan_fwd for callers that cannot allocate device memory.  The pages
  * have no counterpart of this call: it exists for host code that owns no
  * allocator (device memory held by another framework's pool), must not call
@@ -166,8 +245,10 @@ pdssm_status pdssm_scan_bwd(const pdssm_dims *dims, const int32_t *pi_dict,
  *  * Every call on a device shares the one array and it keeps the last
  *    call's contents (each call resets what must start at zero).  Calls whose
  *    work overlaps on the GPU (different streams, no ordering) race on it.
- *  * The device status word of these calls lives in the shared array and is
- *    not exposed; check indices with pdssm_validate when in doubt.
+ *  * The device status word of these calls lives in the shared array; read
+ *    it with pdssm_noalloc_status.
+ *  * The array's address is remembered per device for the life of the
+ *    process: do not use this call on a device across cudaDeviceReset.
  */
 pdssm_status pdssm_scan_fwd_noalloc(const pdssm_dims *dims,
                                     const int32_t *pi_dict,
@@ -179,6 +260,13 @@ pdssm_status pdssm_scan_fwd_noalloc(const pdssm_dims *dims,
 
 /* Size in bytes of the static scratch array of pdssm_scan_fwd_noalloc. */
 size_t pdssm_noalloc_scratch_bytes(void);
+
+/*
+ * pdssm_ws_status for the static scratch of pdssm_scan_fwd_noalloc on the
+ * current device: synchronises the stream, returns what the kernels recorded
+ * (PDSSM_ERR_BAD_INDEX, PDSSM_ERR_TIMEOUT) and clears it.  Allocates nothing.
+ */
+pdssm_status pdssm_noalloc_status(void *stream);
 
 /*
  * Phase A alone, exposing each chunk's closed PD transfer (for tests of the
@@ -195,6 +283,32 @@ pdssm_status pdssm_chunk_transfers(const pdssm_dims *dims,
                                    int32_t *Pi_out, float *Delta_out,
                                    float *v_out, void *ws, size_t ws_bytes,
                                    void *stream);
+
+/*
+ * Test hook: copies the chunk transfers (Pi_c, Delta_c, v_c) and the carries
+ * H_c = h_{e_c} (state at the end of chunk c) that the last pdssm_scan_fwd
+ * left in `ws` (same dims, pi_head_stride and chunk), each
+ * [B][H][ceil(L/chunk)][N] on the device; Pi_out int32, the others fp32.
+ * Asynchronous on the stream.
+ */
+pdssm_status pdssm_ws_transfers(const pdssm_dims *dims, int64_t pi_head_stride,
+                                int64_t chunk, const void *ws, size_t ws_bytes,
+                                int32_t *Pi_out, float *Delta_out,
+                                float *v_out, float *H_out, void *stream);
+
+/*
+ * Self-test of the kernels' bounded waits, with a failure made on purpose
+ * but no fault: which = 0 runs the single-pass forward's look-back for a
+ * chunk whose predecessor never publishes; which = 1 waits on an mbarrier
+ * that nothing completes.  Each wait gives up after cap_ns (1 .. 2e9) of the
+ * GPU's global timer and records PDSSM_ERR_TIMEOUT in the status word of
+ * `ws` (at least pdssm_wait_selftest_ws_bytes() bytes, 256-byte aligned),
+ * which pdssm_ws_status then returns.  The kernels' own waits use a cap of
+ * 2 s.
+ */
+pdssm_status pdssm_wait_selftest(int which, int64_t cap_ns, void *ws,
+                                 size_t ws_bytes, void *stream);
+size_t pdssm_wait_selftest_ws_bytes(void);
 
 /*
  * Checks every dictionary entry lies in [0, N) and every k in [0, K) on the

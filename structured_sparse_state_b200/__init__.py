@@ -34,12 +34,24 @@ STATUS = {0: "PDSSM_OK", 1: "PDSSM_ERR_INVALID_ARG", 2: "PDSSM_ERR_UNSUPPORTED",
 EXPORTS = ("pdssm_status_str", "pdssm_last_error", "pdssm_version",
            "pdssm_workspace_bytes", "pdssm_select", "pdssm_scan_fwd",
            "pdssm_scan_bwd", "pdssm_chunk_transfers", "pdssm_validate",
-           "pdssm_ws_status", "pdssm_scan_fwd_noalloc", "pdssm_noalloc_scratch_bytes")
+           "pdssm_ws_status", "pdssm_scan_fwd_noalloc", "pdssm_noalloc_scratch_bytes",
+           "pdssm_select_with", "pdssm_select_tc_logits", "pdssm_noalloc_status",
+           "pdssm_scan_fwd_traced", "pdssm_scan_bwd_traced", "pdssm_ws_transfers",
+           "pdssm_wait_selftest", "pdssm_wait_selftest_ws_bytes")
+
+TRACE_MAX_KERNELS = 8
+
+SELECT_METHODS = {"auto": 0, "fma": 1, "tensor_core": 2}
 
 
 class Dims(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("H", ctypes.c_int64), ("L", ctypes.c_int64),
                 ("N", ctypes.c_int64), ("K", ctypes.c_int64), ("D_in", ctypes.c_int64)]
+
+
+class Trace(ctypes.Structure):
+    _fields_ = [("events", ctypes.POINTER(ctypes.c_void_p)), ("max_events", ctypes.c_int),
+                ("n_kernels", ctypes.c_int), ("names", ctypes.c_char_p * TRACE_MAX_KERNELS)]
 
 
 class PdssmError(RuntimeError):
@@ -62,6 +74,8 @@ def _load() -> ctypes.CDLL:
         "pdssm_version": (I32, []),
         "pdssm_workspace_bytes": (SZ, [D, I64, I64, I32]),
         "pdssm_select": (I32, [D, P, I32, P, P, P]),
+        "pdssm_select_with": (I32, [D, P, I32, P, P, I32, P]),
+        "pdssm_select_tc_logits": (I32, [D, P, P, P, P, P, P]),
         "pdssm_scan_fwd": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, I64, P, SZ, P]),
         "pdssm_scan_bwd": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, P, P, P, P, I64, P,
                                  SZ, P]),
@@ -70,6 +84,14 @@ def _load() -> ctypes.CDLL:
         "pdssm_ws_status": (I32, [P, SZ, P]),
         "pdssm_scan_fwd_noalloc": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, I64, P]),
         "pdssm_noalloc_scratch_bytes": (SZ, []),
+        "pdssm_noalloc_status": (I32, [P]),
+        "pdssm_ws_transfers": (I32, [D, I64, I64, P, SZ, P, P, P, P, P]),
+        "pdssm_wait_selftest": (I32, [I32, I64, P, SZ, P]),
+        "pdssm_wait_selftest_ws_bytes": (SZ, []),
+        "pdssm_scan_fwd_traced": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, I64, P, SZ, P,
+                                        ctypes.POINTER(Trace)]),
+        "pdssm_scan_bwd_traced": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, P, P, P, P, I64,
+                                        P, SZ, P, ctypes.POINTER(Trace)]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -164,9 +186,7 @@ def pdssm_workspace_bytes(B, H, L, N, K, chunk, per_head_dict=False, for_bwd=Fal
     return int(n)
 
 
-def pdssm_select(u: torch.Tensor, W_sel: torch.Tensor, k_out: Optional[torch.Tensor] = None,
-                 stream=None) -> torch.Tensor:
-    """k[b, h, t] = first argmax_k of the fp32 fma chain sum_q W_sel[h,k,q] u[b,t,q]."""
+def _select_shapes(u, W_sel, k_out):
     _cuda(u, "u", (torch.float32, torch.bfloat16))
     _cuda(W_sel, "W_sel", (torch.float32,))
     B, L, D = u.shape
@@ -176,10 +196,37 @@ def pdssm_select(u: torch.Tensor, W_sel: torch.Tensor, k_out: Optional[torch.Ten
     if k_out is None:
         k_out = torch.empty((B, H, L), dtype=torch.int32, device=u.device)
     _cuda(k_out, "k_out", (torch.int32,))
+    return B, L, D, H, K, k_out
+
+
+def pdssm_select(u: torch.Tensor, W_sel: torch.Tensor, k_out: Optional[torch.Tensor] = None,
+                 stream=None, method: str = "auto") -> torch.Tensor:
+    """k[b, h, t] = first argmax_k of the fp32 fma chain sum_q W_sel[h,k,q] u[b,t,q].
+    ``method``: "auto" (tensor cores where they apply), "fma" or "tensor_core";
+    every route gives the same k bit for bit."""
+    B, L, D, H, K, k_out = _select_shapes(u, W_sel, k_out)
     dm = dims(B, H, L, 0, K, D)
-    _check(_lib.pdssm_select(ctypes.byref(dm), _ptr(u), _dtype_code(u), _ptr(W_sel),
-                             _ptr(k_out), _stream(stream)), "pdssm_select")
+    if method == "auto":
+        _check(_lib.pdssm_select(ctypes.byref(dm), _ptr(u), _dtype_code(u), _ptr(W_sel),
+                                 _ptr(k_out), _stream(stream)), "pdssm_select")
+    else:
+        _check(_lib.pdssm_select_with(ctypes.byref(dm), _ptr(u), _dtype_code(u), _ptr(W_sel),
+                                      _ptr(k_out), SELECT_METHODS[method], _stream(stream)),
+               "pdssm_select_with")
     return k_out
+
+
+def pdssm_select_tc_logits(u: torch.Tensor, W_sel: torch.Tensor, stream=None):
+    """Test hook: the tensor-core selection's k, raw logits [B*L, H*K] and
+    per-(row, head) scale ||u_row|| * max_k ||W_hk|| (rounded up)."""
+    B, L, D, H, K, k_out = _select_shapes(u, W_sel, None)
+    logits = torch.empty((B * L, H * K), dtype=torch.float32, device=u.device)
+    scale = torch.empty((B * L, H), dtype=torch.float32, device=u.device)
+    dm = dims(B, H, L, 0, K, D)
+    _check(_lib.pdssm_select_tc_logits(ctypes.byref(dm), _ptr(u), _ptr(W_sel), _ptr(k_out),
+                                       _ptr(logits), _ptr(scale), _stream(stream)),
+           "pdssm_select_tc_logits")
+    return k_out, logits, scale
 
 
 def _scan_shapes(pi, k, d, b, c):
@@ -253,6 +300,12 @@ def pdssm_noalloc_scratch_bytes() -> int:
     return int(_lib.pdssm_noalloc_scratch_bytes())
 
 
+def pdssm_noalloc_status(stream=None) -> int:
+    """Reads and clears the status word of the no-allocation scratch
+    (synchronises)."""
+    return int(_lib.pdssm_noalloc_status(_stream(stream)))
+
+
 def pdssm_scan_bwd(pi_dict, k, d, b, c, h0, g_y, ws, chunk=128, g_hlast=None, out=None,
                    stream=None):
     """Exact adjoint; ws must be the forward's (sized with for_bwd=True).
@@ -298,6 +351,32 @@ def pdssm_chunk_transfers(pi_dict, k, d, b, chunk, ws=None, stream=None):
     return Pi, Dl, v
 
 
+def pdssm_ws_transfers(ws, B, H, L, N, K, chunk, per_head_dict=False, stream=None):
+    """Test hook: the chunk transfers (Pi, Delta, v) and carries H_c that the
+    last forward left in ws, each [B, H, C, N]."""
+    _cuda(ws, "ws", (torch.uint8,))
+    C = (L + chunk - 1) // chunk
+    dev = ws.device
+    Pi = torch.empty((B, H, C, N), dtype=torch.int32, device=dev)
+    Dl, v, Hc = (torch.empty((B, H, C, N), dtype=torch.float32, device=dev) for _ in range(3))
+    dm = dims(B, H, L, N, K)
+    _check(_lib.pdssm_ws_transfers(ctypes.byref(dm), K * N if per_head_dict else 0, int(chunk),
+                                   _ptr(ws), ws.numel(), _ptr(Pi), _ptr(Dl), _ptr(v), _ptr(Hc),
+                                   _stream(stream)), "pdssm_ws_transfers")
+    return Pi, Dl, v, Hc
+
+
+def pdssm_wait_selftest(which: int, cap_ns: int, device=None, stream=None) -> int:
+    """Runs a bounded wait that nothing completes (0: look-back flag, 1:
+    mbarrier) with the given cap; returns the status word's verdict
+    (PDSSM_ERR_TIMEOUT = 5 expected).  Synchronises."""
+    n = int(_lib.pdssm_wait_selftest_ws_bytes())
+    ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+    _check(_lib.pdssm_wait_selftest(int(which), int(cap_ns), _ptr(ws), n, _stream(stream)),
+           "pdssm_wait_selftest")
+    return pdssm_ws_status(ws, stream)
+
+
 def pdssm_validate(pi_dict, k, N, ws=None, stream=None) -> int:
     """Returns the status code (0 = all indices in range).  Synchronises."""
     _cuda(pi_dict, "pi_dict", (torch.int32,))
@@ -316,3 +395,60 @@ def pdssm_ws_status(ws, stream=None) -> int:
     """Reads and clears the workspace status word (synchronises)."""
     _cuda(ws, "ws", (torch.uint8,))
     return int(_lib.pdssm_ws_status(_ptr(ws), ws.numel(), _stream(stream)))
+
+
+# ----------------------------------------------------------------------------
+# kernel-level timing (measurement aid)
+# ----------------------------------------------------------------------------
+def make_trace_events(n: int = TRACE_MAX_KERNELS + 1, stream=None):
+    """n timing events, recorded once so that their CUDA handles exist."""
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+    s = stream or torch.cuda.current_stream()
+    for e in evs:
+        e.record(s)
+    return evs
+
+
+def _trace_struct(events):
+    arr = (ctypes.c_void_p * len(events))(*[e.cuda_event for e in events])
+    tr = Trace()
+    tr.events = ctypes.cast(arr, ctypes.POINTER(ctypes.c_void_p))
+    tr.max_events = len(events)
+    return tr, arr
+
+
+def _trace_result(tr, events):
+    """[(kernel name, ms)] of a finished traced call (synchronise first)."""
+    return [(tr.names[i].decode(), events[i].elapsed_time(events[i + 1]))
+            for i in range(tr.n_kernels)]
+
+
+def pdssm_scan_fwd_traced(pi_dict, k, d, b, c, h0, chunk, ws, y, h_last, events, stream=None):
+    """pdssm_scan_fwd recording `events` between its kernels; returns a
+    function that, after a synchronisation, gives [(kernel, ms)]."""
+    B, H, L, N, K, stride = _scan_shapes(pi_dict, k, d, b, c)
+    tr, arr = _trace_struct(events)
+    dm = dims(B, H, L, N, K)
+    _check(_lib.pdssm_scan_fwd_traced(ctypes.byref(dm), _ptr(pi_dict), stride, _ptr(k), _ptr(d),
+                                      _ptr(b), _ptr(c), _dtype_code(d), _ptr(h0), _ptr(y),
+                                      _ptr(h_last), int(chunk), _ptr(ws), ws.numel(),
+                                      _stream(stream), ctypes.byref(tr)),
+           "pdssm_scan_fwd_traced")
+    return lambda: _trace_result(tr, events)
+
+
+def pdssm_scan_bwd_traced(pi_dict, k, d, b, c, h0, g_y, ws, chunk, out, events, g_hlast=None,
+                          stream=None):
+    """pdssm_scan_bwd recording `events` between its kernels; returns a
+    function that, after a synchronisation, gives [(kernel, ms)]."""
+    B, H, L, N, K, stride = _scan_shapes(pi_dict, k, d, b, c)
+    tr, arr = _trace_struct(events)
+    g_b, g_d, g_c, g_h0 = out
+    dm = dims(B, H, L, N, K)
+    _check(_lib.pdssm_scan_bwd_traced(ctypes.byref(dm), _ptr(pi_dict), stride, _ptr(k), _ptr(d),
+                                      _ptr(b), _ptr(c), _dtype_code(d), _ptr(h0), _ptr(g_y),
+                                      _ptr(g_hlast), _ptr(g_b), _ptr(g_d), _ptr(g_c), _ptr(g_h0),
+                                      int(chunk), _ptr(ws), ws.numel(), _stream(stream),
+                                      ctypes.byref(tr)),
+           "pdssm_scan_bwd_traced")
+    return lambda: _trace_result(tr, events)

@@ -3,13 +3,15 @@
     python -m structured_sparse_state_b200.build [--force] [--verbose]
 
 nvcc compiles every csrc/*.cu for sm_100a only (no PTX fallback, no fast
-math: denormals and IEEE division stay as written) and links them into one
-shared library with the CUDA runtime linked statically.
+math: denormals and IEEE division stay as written), one object per file in
+parallel (under _build/), and links them into one shared library with the
+CUDA runtime linked statically.
 """
 import glob
 import os
 import subprocess
 import sys
+from concurrent.futures import ThreadPoolExecutor
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
@@ -20,8 +22,9 @@ NVCC_FLAGS = [
     "-O3", "-std=c++17", "-lineinfo",
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-Xcompiler", "-fPIC,-O2",
-    "-shared", "-cudart", "static",
 ]
+LINK_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a", "-shared", "-cudart", "static"]
+OBJ_DIR = os.path.join(HERE, "_build")
 
 
 def _nvcc():
@@ -45,13 +48,25 @@ def _stale():
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
+    """Compiles every csrc/*.cu to an object (in parallel), then links the
+    shared library."""
     if not force and not _stale():
         return LIB
-    cmd = [_nvcc(), *NVCC_FLAGS, "-I", INCLUDE]
-    if verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += ["-o", LIB + ".tmp", *sources()]
-    subprocess.check_call(cmd)
+    os.makedirs(OBJ_DIR, exist_ok=True)
+    nvcc = _nvcc()
+
+    def compile_one(src):
+        obj = os.path.join(OBJ_DIR, os.path.basename(src) + ".o")
+        cmd = [nvcc, *NVCC_FLAGS, "-I", INCLUDE, "-c", src, "-o", obj]
+        if verbose:
+            cmd[1:1] = ["-Xptxas", "-v"]
+        subprocess.check_call(cmd)
+        return obj
+
+    srcs = sources()
+    with ThreadPoolExecutor(max_workers=min(len(srcs), os.cpu_count() or 1)) as ex:
+        objs = list(ex.map(compile_one, srcs))
+    subprocess.check_call([nvcc, *LINK_FLAGS, "-o", LIB + ".tmp", *objs])
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

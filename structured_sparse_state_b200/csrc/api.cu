@@ -10,8 +10,10 @@
 using namespace pdssm;
 
 namespace {
-
 thread_local char g_last_error[256] = "";
+}  // namespace
+
+namespace pdssm {
 
 pdssm_status cuda_fail(cudaError_t e, const char *where) {
     snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
@@ -23,21 +25,18 @@ pdssm_status arg_fail(pdssm_status st, const char *why) {
     return st;
 }
 
-bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+}  // namespace pdssm
 
-int stage_override() {
-    static const int v = [] {
-        const char *e = getenv("PDSSM_STAGES");
-        const int n = e ? atoi(e) : 0;
-        return (n >= 2 && n <= kMaxStages) ? n : 0;
-    }();
-    return v;
-}
+namespace {
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
 
 size_t dtype_size(pdssm_dtype t) { return t == PDSSM_BF16 ? 2 : 4; }
 
+}  // namespace
+
 // Shape checks shared by the scan calls.
-pdssm_status check_scan_dims(const pdssm_dims *dm, int64_t pi_hs, int64_t chunk) {
+pdssm_status pdssm::check_scan_dims(const pdssm_dims *dm, int64_t pi_hs, int64_t chunk) {
     if (!dm) return arg_fail(PDSSM_ERR_INVALID_ARG, "dims is NULL");
     if (dm->B < 1 || dm->H < 1 || dm->L < 0 || dm->N < 1 || dm->K < 1)
         return arg_fail(PDSSM_ERR_INVALID_ARG, "need B, H, N, K >= 1 and L >= 0");
@@ -50,6 +49,8 @@ pdssm_status check_scan_dims(const pdssm_dims *dm, int64_t pi_hs, int64_t chunk)
         return arg_fail(PDSSM_ERR_UNSUPPORTED, "B*H*L too large");
     return PDSSM_OK;
 }
+
+namespace {
 
 pdssm_status check_dtype(pdssm_dtype t) {
     if (t != PDSSM_F32 && t != PDSSM_BF16)
@@ -89,28 +90,20 @@ ChunkParams make_params(const pdssm_dims *dm, const WsLayout &w, void *ws, int64
     if (w.wc) p.wc = reinterpret_cast<float *>(base + w.wc);
     if (w.lam) p.lam = reinterpret_cast<float *>(base + w.lam);
     p.status = reinterpret_cast<int *>(base + w.status);
+    p.ticket = reinterpret_cast<unsigned long long *>(base + w.look);
+    p.look = reinterpret_cast<int *>(base + w.look + kLookHeader);
+    p.wait_ns = kWaitCapNs;
     const int es = (int)dtype_size(dt);
     const int rowb = (int)dm->N * es;
     const bool vec_ok = (rowb % 16) == 0;
     const bool ptr_ok = (!d || aligned(d, 16)) && (!b || aligned(b, 16)) && (!c || aligned(c, 16));
     p.bulk = (vec_ok && ptr_ok) ? 1 : 0;
-    // double-buffered tiles (plus L2 prefetch further ahead); PDSSM_STAGES
-    // overrides the depth (2..4) for tuning
-    p.ns = stage_override() > 0 ? stage_override() : 2;
+    // double-buffered tiles (the general kernels add an L2 prefetch further ahead)
+    p.ns = kFastStages;
     return p;
 }
 
 }  // namespace
-
-// The tensor-core selection path is the default where it applies;
-// PDSSM_SELECT_FMA=1 forces the plain fma-chain kernel (for comparisons).
-bool pdssm::select_tc_enabled() {
-    static const bool on = [] {
-        const char *e = getenv("PDSSM_SELECT_FMA");
-        return !(e && atoi(e) != 0);
-    }();
-    return on;
-}
 
 extern "C" {
 
@@ -137,8 +130,9 @@ size_t pdssm_workspace_bytes(const pdssm_dims *dims, int64_t pi_head_stride, int
     return ws_layout(*dims, pi_head_stride, chunk, for_bwd != 0).total;
 }
 
-pdssm_status pdssm_select(const pdssm_dims *dims, const void *u, pdssm_dtype u_dtype,
-                          const float *W_sel, int32_t *k_out, void *stream) {
+static pdssm_status select_common(const pdssm_dims *dims, const void *u, pdssm_dtype u_dtype,
+                                  const float *W_sel, int32_t *k_out, int method,
+                                  float *logits_out, float *scale_out, void *stream) {
     if (!dims) return arg_fail(PDSSM_ERR_INVALID_ARG, "dims is NULL");
     if (check_dtype(u_dtype) != PDSSM_OK) return PDSSM_ERR_INVALID_ARG;
     if (dims->B < 1 || dims->H < 1 || dims->L < 0 || dims->K < 1 || dims->D_in < 1)
@@ -148,9 +142,39 @@ pdssm_status pdssm_select(const pdssm_dims *dims, const void *u, pdssm_dtype u_d
     if (dims->L == 0) return PDSSM_OK;
     if (!u || !W_sel || !k_out) return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL tensor pointer");
     if (!aligned(W_sel, 16)) return arg_fail(PDSSM_ERR_INVALID_ARG, "W_sel not 16-byte aligned");
-    cudaError_t e = launch_select(*dims, u, u_dtype, W_sel, k_out, (cudaStream_t)stream);
+    if (method != PDSSM_SELECT_AUTO && method != PDSSM_SELECT_FMA_CHAIN &&
+        method != PDSSM_SELECT_TENSOR_CORE)
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "unknown selection method");
+    const bool tc_ok = select_tc_supported(*dims, u_dtype, u, W_sel);
+    if (method == PDSSM_SELECT_TENSOR_CORE && !tc_ok)
+        return arg_fail(PDSSM_ERR_UNSUPPORTED,
+                        "tensor-core selection needs bf16 u, D_in a multiple of 16, K a power "
+                        "of two and H*K <= 256");
+    const bool use_tc = method == PDSSM_SELECT_TENSOR_CORE || (method == PDSSM_SELECT_AUTO && tc_ok);
+    cudaError_t e = launch_select(*dims, u, u_dtype, W_sel, k_out, use_tc, logits_out, scale_out,
+                                  (cudaStream_t)stream);
     if (e != cudaSuccess) return cuda_fail(e, "select");
     return PDSSM_OK;
+}
+
+pdssm_status pdssm_select(const pdssm_dims *dims, const void *u, pdssm_dtype u_dtype,
+                          const float *W_sel, int32_t *k_out, void *stream) {
+    return select_common(dims, u, u_dtype, W_sel, k_out, PDSSM_SELECT_AUTO, nullptr, nullptr,
+                         stream);
+}
+
+pdssm_status pdssm_select_with(const pdssm_dims *dims, const void *u, pdssm_dtype u_dtype,
+                               const float *W_sel, int32_t *k_out, int method, void *stream) {
+    return select_common(dims, u, u_dtype, W_sel, k_out, method, nullptr, nullptr, stream);
+}
+
+pdssm_status pdssm_select_tc_logits(const pdssm_dims *dims, const void *u, const float *W_sel,
+                                    int32_t *k_out, float *logits_out, float *scale_out,
+                                    void *stream) {
+    if (!logits_out || !scale_out)
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL logits or scale output");
+    return select_common(dims, u, PDSSM_BF16, W_sel, k_out, PDSSM_SELECT_TENSOR_CORE, logits_out,
+                         scale_out, stream);
 }
 
 static pdssm_status fwd_common(const pdssm_dims *dims, const int32_t *pi_dict,
@@ -178,6 +202,9 @@ static pdssm_status run_prep(const pdssm_dims *dims, const int32_t *pi_dict,
     // distance, largest fan-in)
     cudaError_t e = cudaMemsetAsync(base + w.status, 0, 16, st);
     if (e != cudaSuccess) return cuda_fail(e, "status reset");
+    // the single-pass forward's ticket counter and per-chunk flags
+    e = cudaMemsetAsync(base + w.look, 0, kLookHeader + (size_t)(dims->B * dims->H * w.C) * 4, st);
+    if (e != cudaSuccess) return cuda_fail(e, "look-back reset");
     e = launch_prep(*dims, pi_dict, pi_head_stride, reinterpret_cast<int32_t *>(base + w.dict),
                     reinterpret_cast<uint2 *>(base + w.seg),
                     reinterpret_cast<int *>(base + w.status) + 1,
@@ -188,47 +215,89 @@ static pdssm_status run_prep(const pdssm_dims *dims, const int32_t *pi_dict,
     return PDSSM_OK;
 }
 
-pdssm_status pdssm_scan_fwd(const pdssm_dims *dims, const int32_t *pi_dict,
-                            int64_t pi_head_stride, const int32_t *k, const void *d,
-                            const void *b, const void *c, pdssm_dtype in_dtype, const float *h0,
-                            float *y, float *h_last, int64_t chunk, void *ws, size_t ws_bytes,
-                            void *stream) {
+}  // extern "C"
+
+namespace {
+
+// Records the caller's events between the kernels of a traced call: mark()
+// before each kernel (with its name), finish() after the last one.
+struct Tracer {
+    pdssm_trace *t;
+    cudaStream_t s;
+    cudaError_t mark(const char *name) {
+        if (!t) return cudaSuccess;
+        if (t->n_kernels + 1 >= t->max_events || t->n_kernels >= PDSSM_TRACE_MAX_KERNELS)
+            return cudaSuccess;
+        t->names[t->n_kernels] = name;
+        return cudaEventRecord((cudaEvent_t)t->events[t->n_kernels++], s);
+    }
+    cudaError_t finish() {
+        if (!t || t->n_kernels == 0) return cudaSuccess;
+        return cudaEventRecord((cudaEvent_t)t->events[t->n_kernels], s);
+    }
+};
+
+pdssm_status scan_fwd_impl(const pdssm_dims *dims, const int32_t *pi_dict, int64_t pi_head_stride,
+                           const int32_t *k, const void *d, const void *b, const void *c,
+                           pdssm_dtype in_dtype, const float *h0, float *y, float *h_last,
+                           int64_t chunk, void *ws, size_t ws_bytes, void *stream,
+                           pdssm_trace *trace) {
     WsLayout w;
     pdssm_status st = fwd_common(dims, pi_dict, pi_head_stride, k, d, b, in_dtype, chunk, ws,
                                  ws_bytes, false, &w);
     if (st != PDSSM_OK) return st;
     if (dims->L > 0 && (!c || !y)) return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL c or y");
+    if (trace) {
+        if (!trace->events || trace->max_events < 2)
+            return arg_fail(PDSSM_ERR_INVALID_ARG, "trace needs at least two events");
+        trace->n_kernels = 0;
+    }
     cudaStream_t s = (cudaStream_t)stream;
+    Tracer tr{trace, s};
+    cudaError_t e = tr.mark("prep");
+    if (e != cudaSuccess) return cuda_fail(e, "trace event");
     st = run_prep(dims, pi_dict, pi_head_stride, w, ws, s);
     if (st != PDSSM_OK) return st;
     if (dims->L == 0) {
         if (h_last) {
             const size_t bytes = (size_t)(dims->B * dims->H * dims->N) * 4;
-            cudaError_t e = h0 ? cudaMemcpyAsync(h_last, h0, bytes, cudaMemcpyDeviceToDevice, s)
-                               : cudaMemsetAsync(h_last, 0, bytes, s);
+            e = h0 ? cudaMemcpyAsync(h_last, h0, bytes, cudaMemcpyDeviceToDevice, s)
+                   : cudaMemsetAsync(h_last, 0, bytes, s);
             if (e != cudaSuccess) return cuda_fail(e, "h_last for L = 0");
         }
-        return PDSSM_OK;
+        e = tr.finish();
+        return e == cudaSuccess ? PDSSM_OK : cuda_fail(e, "trace event");
     }
     ChunkParams p = make_params(dims, w, ws, chunk, k, d, b, c, in_dtype);
     p.h0 = h0;
     p.y = y;
     p.h_last = h_last;
-    cudaError_t e = launch_phaseA(p, in_dtype, s);
+    if (fused_path(p)) {
+        if ((e = tr.mark("single pass")) != cudaSuccess) return cuda_fail(e, "trace event");
+        e = launch_scan_fused(p, in_dtype, s);
+        if (e != cudaSuccess) return cuda_fail(e, "single-pass forward");
+        e = tr.finish();
+        return e == cudaSuccess ? PDSSM_OK : cuda_fail(e, "trace event");
+    }
+    if ((e = tr.mark("phase A")) != cudaSuccess) return cuda_fail(e, "trace event");
+    e = launch_phaseA(p, in_dtype, s);
     if (e != cudaSuccess) return cuda_fail(e, "phase A");
+    if ((e = tr.mark("phase B")) != cudaSuccess) return cuda_fail(e, "trace event");
     e = launch_phaseB(p, s);
     if (e != cudaSuccess) return cuda_fail(e, "phase B");
+    if ((e = tr.mark("phase C")) != cudaSuccess) return cuda_fail(e, "trace event");
     e = launch_phaseC(p, in_dtype, s);
     if (e != cudaSuccess) return cuda_fail(e, "phase C");
-    return PDSSM_OK;
+    e = tr.finish();
+    return e == cudaSuccess ? PDSSM_OK : cuda_fail(e, "trace event");
 }
 
-pdssm_status pdssm_scan_bwd(const pdssm_dims *dims, const int32_t *pi_dict,
-                            int64_t pi_head_stride, const int32_t *k, const void *d,
-                            const void *b, const void *c, pdssm_dtype in_dtype, const float *h0,
-                            const float *g_y, const float *g_hlast, float *g_b, float *g_d,
-                            float *g_c, float *g_h0, int64_t chunk, void *ws, size_t ws_bytes,
-                            void *stream) {
+pdssm_status scan_bwd_impl(const pdssm_dims *dims, const int32_t *pi_dict, int64_t pi_head_stride,
+                           const int32_t *k, const void *d, const void *b, const void *c,
+                           pdssm_dtype in_dtype, const float *h0, const float *g_y,
+                           const float *g_hlast, float *g_b, float *g_d, float *g_c, float *g_h0,
+                           int64_t chunk, void *ws, size_t ws_bytes, void *stream,
+                           pdssm_trace *trace) {
     WsLayout w;
     pdssm_status st = fwd_common(dims, pi_dict, pi_head_stride, k, d, b, in_dtype, chunk, ws,
                                  ws_bytes, true, &w);
@@ -237,13 +306,19 @@ pdssm_status pdssm_scan_bwd(const pdssm_dims *dims, const int32_t *pi_dict,
         return arg_fail(PDSSM_ERR_UNSUPPORTED, "backward needs chunk <= 256");
     if (dims->L > 0 && (!c || !g_y || !g_b || !g_d || !g_c))
         return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL tensor pointer");
+    if (trace) {
+        if (!trace->events || trace->max_events < 2)
+            return arg_fail(PDSSM_ERR_INVALID_ARG, "trace needs at least two events");
+        trace->n_kernels = 0;
+    }
     cudaStream_t s = (cudaStream_t)stream;
+    Tracer tr{trace, s};
+    cudaError_t e;
     if (dims->L == 0) {
         if (g_h0) {
             const size_t bytes = (size_t)(dims->B * dims->H * dims->N) * 4;
-            cudaError_t e = g_hlast
-                                ? cudaMemcpyAsync(g_h0, g_hlast, bytes, cudaMemcpyDeviceToDevice, s)
-                                : cudaMemsetAsync(g_h0, 0, bytes, s);
+            e = g_hlast ? cudaMemcpyAsync(g_h0, g_hlast, bytes, cudaMemcpyDeviceToDevice, s)
+                        : cudaMemsetAsync(g_h0, 0, bytes, s);
             if (e != cudaSuccess) return cuda_fail(e, "g_h0 for L = 0");
         }
         return PDSSM_OK;
@@ -256,13 +331,62 @@ pdssm_status pdssm_scan_bwd(const pdssm_dims *dims, const int32_t *pi_dict,
     p.g_d = g_d;
     p.g_c = g_c;
     p.g_h0 = g_h0;
-    cudaError_t e = launch_bwdA(p, in_dtype, s);
+    if ((e = tr.mark("bwd phase A")) != cudaSuccess) return cuda_fail(e, "trace event");
+    e = launch_bwdA(p, in_dtype, s);
     if (e != cudaSuccess) return cuda_fail(e, "bwd phase A");
+    if ((e = tr.mark("bwd phase B")) != cudaSuccess) return cuda_fail(e, "trace event");
     e = launch_bwdB(p, s);
     if (e != cudaSuccess) return cuda_fail(e, "bwd phase B");
+    if ((e = tr.mark("bwd phase C")) != cudaSuccess) return cuda_fail(e, "trace event");
     e = launch_bwdC(p, in_dtype, s);
     if (e != cudaSuccess) return cuda_fail(e, "bwd phase C");
-    return PDSSM_OK;
+    e = tr.finish();
+    return e == cudaSuccess ? PDSSM_OK : cuda_fail(e, "trace event");
+}
+
+}  // namespace
+
+extern "C" {
+
+pdssm_status pdssm_scan_fwd(const pdssm_dims *dims, const int32_t *pi_dict,
+                            int64_t pi_head_stride, const int32_t *k, const void *d,
+                            const void *b, const void *c, pdssm_dtype in_dtype, const float *h0,
+                            float *y, float *h_last, int64_t chunk, void *ws, size_t ws_bytes,
+                            void *stream) {
+    return scan_fwd_impl(dims, pi_dict, pi_head_stride, k, d, b, c, in_dtype, h0, y, h_last,
+                         chunk, ws, ws_bytes, stream, nullptr);
+}
+
+pdssm_status pdssm_scan_fwd_traced(const pdssm_dims *dims, const int32_t *pi_dict,
+                                   int64_t pi_head_stride, const int32_t *k, const void *d,
+                                   const void *b, const void *c, pdssm_dtype in_dtype,
+                                   const float *h0, float *y, float *h_last, int64_t chunk,
+                                   void *ws, size_t ws_bytes, void *stream, pdssm_trace *trace) {
+    if (!trace) return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL trace");
+    return scan_fwd_impl(dims, pi_dict, pi_head_stride, k, d, b, c, in_dtype, h0, y, h_last,
+                         chunk, ws, ws_bytes, stream, trace);
+}
+
+pdssm_status pdssm_scan_bwd(const pdssm_dims *dims, const int32_t *pi_dict,
+                            int64_t pi_head_stride, const int32_t *k, const void *d,
+                            const void *b, const void *c, pdssm_dtype in_dtype, const float *h0,
+                            const float *g_y, const float *g_hlast, float *g_b, float *g_d,
+                            float *g_c, float *g_h0, int64_t chunk, void *ws, size_t ws_bytes,
+                            void *stream) {
+    return scan_bwd_impl(dims, pi_dict, pi_head_stride, k, d, b, c, in_dtype, h0, g_y, g_hlast,
+                         g_b, g_d, g_c, g_h0, chunk, ws, ws_bytes, stream, nullptr);
+}
+
+pdssm_status pdssm_scan_bwd_traced(const pdssm_dims *dims, const int32_t *pi_dict,
+                                   int64_t pi_head_stride, const int32_t *k, const void *d,
+                                   const void *b, const void *c, pdssm_dtype in_dtype,
+                                   const float *h0, const float *g_y, const float *g_hlast,
+                                   float *g_b, float *g_d, float *g_c, float *g_h0,
+                                   int64_t chunk, void *ws, size_t ws_bytes, void *stream,
+                                   pdssm_trace *trace) {
+    if (!trace) return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL trace");
+    return scan_bwd_impl(dims, pi_dict, pi_head_stride, k, d, b, c, in_dtype, h0, g_y, g_hlast,
+                         g_b, g_d, g_c, g_h0, chunk, ws, ws_bytes, stream, trace);
 }
 
 pdssm_status pdssm_chunk_transfers(const pdssm_dims *dims, const int32_t *pi_dict,
@@ -288,6 +412,54 @@ pdssm_status pdssm_chunk_transfers(const pdssm_dims *dims, const int32_t *pi_dic
     cudaError_t e = launch_phaseA(p, in_dtype, s);
     if (e != cudaSuccess) return cuda_fail(e, "phase A");
     return PDSSM_OK;
+}
+
+pdssm_status pdssm_ws_transfers(const pdssm_dims *dims, int64_t pi_head_stride, int64_t chunk,
+                                const void *ws, size_t ws_bytes, int32_t *Pi_out,
+                                float *Delta_out, float *v_out, float *H_out, void *stream) {
+    pdssm_status st = check_scan_dims(dims, pi_head_stride, chunk);
+    if (st != PDSSM_OK) return st;
+    if (!ws || !Pi_out || !Delta_out || !v_out || !H_out)
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL pointer");
+    const WsLayout w = ws_layout(*dims, pi_head_stride, chunk, false);
+    if (ws_bytes < w.total) return arg_fail(PDSSM_ERR_WORKSPACE, "workspace too small");
+    const size_t bytes = (size_t)(dims->B * dims->H * w.C * dims->N) * 4;
+    if (bytes == 0) return PDSSM_OK;
+    const unsigned char *base = reinterpret_cast<const unsigned char *>(ws);
+    cudaStream_t s = (cudaStream_t)stream;
+    void *dst[4] = {Pi_out, Delta_out, v_out, H_out};
+    const size_t src[4] = {w.Pi, w.Dl, w.v, w.Hc};
+    for (int i = 0; i < 4; ++i) {
+        cudaError_t e = cudaMemcpyAsync(dst[i], base + src[i], bytes, cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return cuda_fail(e, "transfer copy");
+    }
+    return PDSSM_OK;
+}
+
+pdssm_status pdssm_wait_selftest(int which, int64_t cap_ns, void *ws, size_t ws_bytes,
+                                 void *stream) {
+    if (which != 0 && which != 1) return arg_fail(PDSSM_ERR_INVALID_ARG, "which must be 0 or 1");
+    if (cap_ns < 1 || cap_ns > (int64_t)kWaitCapNs)
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "cap_ns must lie in [1, 2e9]");
+    // a one-sequence, two-chunk layout whose flags are all zero
+    const pdssm_dims dm = {1, 1, 2, 32, 1, 0};
+    const WsLayout w = ws_layout(dm, 0, 1, false);
+    if (!ws || ws_bytes < w.total || !aligned(ws, 256))
+        return arg_fail(PDSSM_ERR_WORKSPACE, "workspace too small or not 256-byte aligned");
+    cudaStream_t s = (cudaStream_t)stream;
+    unsigned char *base = reinterpret_cast<unsigned char *>(ws);
+    cudaError_t e = cudaMemsetAsync(base, 0, w.total, s);
+    if (e != cudaSuccess) return cuda_fail(e, "self-test reset");
+    ChunkParams p = make_params(&dm, w, ws, 1, nullptr, nullptr, nullptr, nullptr, PDSSM_F32);
+    p.wait_ns = (uint64_t)cap_ns;
+    e = launch_wait_selftest(p, which, s);
+    if (e != cudaSuccess) return cuda_fail(e, "wait self-test");
+    return PDSSM_OK;
+}
+
+size_t pdssm_wait_selftest_ws_bytes(void) {
+    const pdssm_dims dm = {1, 1, 2, 32, 1, 0};
+    return ws_layout(dm, 0, 1, false).total;
 }
 
 pdssm_status pdssm_validate(const pdssm_dims *dims, const int32_t *pi_dict,

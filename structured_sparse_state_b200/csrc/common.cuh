@@ -5,9 +5,9 @@
 // r < NPL, NPL = ceil(N / 32) in {1, 2}.  Chunk data (rows of d, b, c) are
 // contiguous in HBM, so each warp streams its chunk through shared memory in
 // tiles of kTS steps with 1-D bulk copies (cp.async.bulk, the TMA engine's
-// non-tensor path) completed on per-warp mbarriers: a compile-time two-stage
-// ring in the fast kernels (N = 32 / 64), a ring of p.ns stages with L2
-// prefetch ahead of it in the general kernels.
+// non-tensor path) completed on per-warp mbarriers: a two-stage ring (fixed
+// at compile time in the fast kernels for N = 32 / 64; the general kernels
+// add an L2 prefetch ahead of it).
 #pragma once
 
 #include <cuda_bf16.h>
@@ -25,7 +25,7 @@ namespace pdssm {
 constexpr int kTS = 8;         // steps per staged tile = steps per readout group
 constexpr int kMaxWPC = 8;     // most warps (units) per CTA in the chunk kernels
 constexpr int kMaxN = 64;
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 2;
 constexpr int kBwdMaxChunk = 256;   // checkpoints of one chunk kept in shared memory (general bwd C)
 constexpr int kDcap = 8;            // sources per target held in the slot table
 constexpr int kPrefetchTiles = 4;   // tiles prefetched into L2 ahead of the staged ones (general kernels)
@@ -40,9 +40,13 @@ enum : int { kStBadIndex = 1, kStTimeout = 2 };
 // workspace layout (all offsets 256-byte aligned)
 // ---------------------------------------------------------------------------
 struct WsLayout {
-    size_t status, dict, tab, fan, seg, Pi, Dl, v, Hc, wc, lam, total;
+    size_t status, dict, tab, fan, seg, look, Pi, Dl, v, Hc, wc, lam, total;
     int64_t C, Hd;
 };
+
+// Look-back region of the single-pass forward: a 64-bit chunk ticket counter
+// (first 8 bytes of a 256-byte header), then one flag word per chunk.
+constexpr size_t kLookHeader = 256;
 
 inline size_t align256(size_t x) { return (x + 255) / 256 * 256; }
 
@@ -61,6 +65,7 @@ inline WsLayout ws_layout(const pdssm_dims &dm, int64_t pi_hs, int64_t chunk,
     w.tab = o;    o = align256(o + (size_t)(w.Hd * dm.K * kDcap * 64));
     w.fan = o;    o = align256(o + (size_t)(w.Hd * dm.K) * 4);
     w.seg = o;    o = align256(o + (size_t)(w.Hd * dm.K) * 32 * 8);
+    w.look = o;   o = align256(o + kLookHeader + units * 4);
     w.Pi = o;     o = align256(o + vecs);
     w.Dl = o;     o = align256(o + vecs);
     w.v = o;      o = align256(o + vecs);
@@ -96,6 +101,9 @@ struct ChunkParams {
     float *g_b, *g_d, *g_c, *g_h0;
     float *h_last;
     int *status;
+    int *look;                // single-pass forward: per-chunk flags (0, kFlagAgg, kFlagIncl)
+    unsigned long long *ticket;   // single-pass forward: next chunk ticket
+    uint64_t wait_ns;         // cap of every bounded wait, in ns of the global timer
     int ns;                   // pipeline stages
     int wpc;                  // warps (units) per CTA
     int bulk;                 // 1: bulk-copy staging; 0: cooperative copies
@@ -174,15 +182,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Bounded wait: gives up after ~2 s of wall time or 2^26 polls.
-static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+// Cap of every bounded wait (global-timer ns) unless a caller passes another.
+constexpr uint64_t kWaitCapNs = 2000000000ull;
+
+// Bounded wait: gives up after cap_ns of wall time or 2^26 polls.
+static __device__ __noinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                      uint64_t cap_ns = kWaitCapNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_ns();
     for (uint32_t it = 0; it < (1u << 26); ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 1023u) == 1023u && global_ns() - t0 > 2000000000ull) break;
+        if ((it & 1023u) == 1023u && global_ns() - t0 > cap_ns) break;
     }
     return false;
+}
+
+// Flag words shared between CTAs of one grid (single-pass forward): the
+// writer stores its data, fences, and publishes the flag with a release
+// store; the reader polls with acquire loads and reads the data through L2.
+__device__ __forceinline__ int ld_acquire_gpu(const int *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_gpu(int *p, int v) {
+    asm volatile("st.release.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_shared() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 // ---------------------------------------------------------------------------
@@ -702,6 +729,25 @@ __device__ __forceinline__ void copy_slot(unsigned char *dst, const ChunkParams 
     }
 }
 
+// View of one staged dictionary slot.
+__device__ __forceinline__ SmemDict dict_view(const ChunkParams &p, const unsigned char *mine) {
+    const int K = (int)p.K, N = (int)p.N;
+    const int c = dict_parts(p.dict_content);
+    SmemDict sd;
+    sd.map = reinterpret_cast<const int *>(mine);
+    int off = dict_map_bytes(K, N, c);
+    sd.tab = nullptr;
+    sd.fan = nullptr;
+    sd.seg = nullptr;
+    if (c & kDictTab) {
+        sd.tab = mine + off;
+        sd.fan = reinterpret_cast<const int *>(mine + off + K * kDcap * 64);
+        off += dict_tab_bytes(K);
+    }
+    if (c & kDictSeg) sd.seg = reinterpret_cast<const uint2 *>(mine + (off + 7) / 8 * 8);
+    return sd;
+}
+
 // Loads the dictionary used by this CTA's warps into shared memory and
 // returns this warp's view.  Must be reached by every thread of the CTA.
 // scale = 4 stores map entries as byte offsets into int32 rows.
@@ -961,14 +1007,21 @@ inline cudaError_t launch_units(KernT kern, ChunkParams p, int per_warp, cudaStr
 }
 
 // ---------------------------------------------------------------------------
+// host-side argument checks and error text (api.cu)
+// ---------------------------------------------------------------------------
+pdssm_status check_scan_dims(const pdssm_dims *dm, int64_t pi_hs, int64_t chunk);
+pdssm_status cuda_fail(cudaError_t e, const char *where);   // sets the last-error text
+pdssm_status arg_fail(pdssm_status st, const char *why);    // sets the last-error text
+
+// ---------------------------------------------------------------------------
 // host launchers (one per kernel family)
 // ---------------------------------------------------------------------------
 cudaError_t launch_select(const pdssm_dims &dm, const void *u, pdssm_dtype ut, const float *W,
-                          int32_t *k_out, cudaStream_t st);
+                          int32_t *k_out, bool use_tc, float *logits_out, float *scale_out,
+                          cudaStream_t st);
 bool select_tc_supported(const pdssm_dims &dm, pdssm_dtype ut, const void *u, const float *W);
-bool select_tc_enabled();
 cudaError_t launch_select_tc(const pdssm_dims &dm, const void *u, const float *W, int32_t *k_out,
-                             cudaStream_t st);
+                             float *logits_out, float *scale_out, cudaStream_t st);
 cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
                         uint2 *seg, int *dict_stats,
                         uint8_t *tab, int32_t *fan, int64_t Hd, int *status, cudaStream_t st);
@@ -978,6 +1031,9 @@ cudaError_t launch_phaseA(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st)
 bool fast_path(const ChunkParams &p);
 cudaError_t launch_phaseA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
 cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
+cudaError_t launch_scan_fused(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
+bool fused_path(const ChunkParams &p);
+cudaError_t launch_wait_selftest(const ChunkParams &p, int which, cudaStream_t st);
 cudaError_t launch_bwdA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
 cudaError_t launch_bwdC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
 cudaError_t launch_phaseB(const ChunkParams &p, cudaStream_t st);

@@ -10,21 +10,34 @@
 //   * readout partials go to the per-warp transpose buffer.
 // The general kernels in fwd.cu serve every other N and unaligned rows.
 #include "common.cuh"
+#include "transfer_ops.cuh"
 
 namespace pdssm {
 
-// Phase A of one chunk (this warp's unit); LV selects the PD step (0: the
-// permutation step, else the segment-table step with LV shuffle levels).
+// The closed PD transfer of a segment, as the lanes hold it at the end of
+// phase A: column e = lane * NPL + r moves to pos[r] / sizeof(T) with factor
+// Dl[r]; v[r] is the segment's state (started from zero) at element e.
+template <int NPL>
+struct SegTransfer {
+    int pos[NPL];
+    float Dl[NPL];
+    float v[NPL];
+};
+
+// Phase A over the segment of `len` steps starting at global row `row0`
+// (one sequence): the local readout (when p.y is set) and the segment's
+// closed transfer.  LV selects the PD step (0: the permutation step, else the
+// segment-table step with LV shuffle levels).  Initialises this warp's ring
+// barriers; uses tiles 0 .. ceil(len / kTS) - 1 of the ring.  Returns false
+// if a staging wait gave up (status flagged, transfer undefined).
 template <typename T, int NPL, int LV>
-__device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const SmemDict &sd,
-                                                 unsigned char *wbase, int64_t unit, int lane) {
+__device__ __forceinline__ bool phaseA_segment(const ChunkParams &p, const SmemDict &sd,
+                                               unsigned char *wbase, int64_t row0, int len,
+                                               int lane, SegTransfer<NPL> &out) {
     constexpr int N = 32 * NPL;
     constexpr int ROWB = N * (int)sizeof(T);
     constexpr int TENS = kTS * ROWB;
     const int K = (int)p.K;
-    const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
-    const int64_t s = cidx * p.chunk;
-    const int len = (int)imin64(p.chunk, p.L - s);
     const bool with_y = p.y != nullptr;
     const int nt = with_y ? 3 : 2;
 
@@ -36,7 +49,6 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
     ring.bar0 = smem_u32(ybuf + kYbufFloats);
     ring.len = len;
     ring.nt = nt;
-    const int64_t row0 = bh * p.L + s;
     ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + row0 * ROWB;
     ring.src[1] = reinterpret_cast<const unsigned char *>(p.b) + row0 * ROWB;
     ring.src[2] = with_y ? reinterpret_cast<const unsigned char *>(p.c) + row0 * ROWB
@@ -68,7 +80,7 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
     for (int i = 0; i < ntiles; ++i) {
         if (!ring.wait(i)) {
             ring.abort(i, ntiles, p.status, lane);
-            return;
+            return false;
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
@@ -159,13 +171,33 @@ __device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const Sme
         if (i + kFastStages < ntiles) ring.issue(i + kFastStages, lane);
         kreg = clamp_k(knext, K, p.status);
     }
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        out.pos[r] = posb[r];
+        out.Dl[r] = Dl[r];
+        out.v[r] = h[r];
+    }
+    return true;
+}
+
+// Phase A of one chunk (this warp's unit) for the three-phase forward: the
+// transfer goes to the workspace.
+template <typename T, int NPL, int LV>
+__device__ __forceinline__ void phaseA_fast_unit(const ChunkParams &p, const SmemDict &sd,
+                                                 unsigned char *wbase, int64_t unit, int lane) {
+    const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
+    const int64_t s = cidx * p.chunk;
+    const int len = (int)imin64(p.chunk, p.L - s);
+    SegTransfer<NPL> tr;
+    if (!phaseA_segment<T, NPL, LV>(p, sd, wbase, bh * p.L + s, len, lane, tr)) return;
+    constexpr int ES = (int)sizeof(T);
     const int64_t o = unit * p.N;
 #pragma unroll
     for (int r = 0; r < NPL; ++r) {
         const int e2 = lane * NPL + r;
-        p.Pi[o + e2] = posb[r] / ES;
-        p.Dl[o + e2] = Dl[r];
-        p.v[o + e2] = h[r];
+        p.Pi[o + e2] = tr.pos[r] / ES;
+        p.Dl[o + e2] = tr.Dl[r];
+        p.v[o + e2] = tr.v[r];
     }
 }
 
@@ -190,66 +222,58 @@ __global__ void __launch_bounds__(kMaxWPC * 32, (sizeof(T) == 4 && NPL == 2) ? 2
     }
 }
 
-template <typename T, int NPL>
-__global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams p) {
-    extern __shared__ __align__(128) unsigned char sm_c_raw[];
-    unsigned char *sm_c = smem_base256(sm_c_raw);
-    pdl_trigger();
-    pdl_wait();   // the carries come from the preceding kernel
+// Carry correction (phase C) over the segment of `len` steps starting at
+// global row `row0`, in path form: column e = lane * NPL + r of the carry
+// starts with weight w[r] and follows the selected maps; y gains
+// sum_e c_t[pos_t(e)] w_t(e) at every step.  The ring has NT tensors per
+// stage; d goes to tensor 0 and c to tensor CQ.  Tile i of the segment uses
+// ring slot tbase + i (so a warp can continue the barrier phases of an
+// earlier pass over the same ring).  Returns false if a staging wait gave up.
+template <typename T, int NPL, int NT, int CQ>
+__device__ __forceinline__ bool phaseC_segment(const ChunkParams &p, const SmemDict &sd,
+                                               uint32_t ring_s, uint32_t bar0, float *ybuf,
+                                               int64_t row0, int len, float (&w)[NPL],
+                                               int tbase, int lane) {
     constexpr int N = 32 * NPL;
     constexpr int ROWB = N * (int)sizeof(T);
     constexpr int TENS = kTS * ROWB;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const SmemDict sd = stage_dict(p, sm_c, warp, lane, (int)sizeof(T));
-    const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
-    if (unit >= p.units) return;
     const int K = (int)p.K;
-    const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
-    if (cidx == 0 && p.h0 == nullptr) return;   // zero initial state: nothing to correct
-    const int64_t s = cidx * p.chunk;
-    const int len = (int)imin64(p.chunk, p.L - s);
-
-    unsigned char *wbase = sm_c + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
-    using RingT = FastRing<2, ROWB>;
-    float *ybuf = reinterpret_cast<float *>(wbase + kFastStages * RingT::STAGEB);   // [kTS][33]
+    using RingT = FastRing<NT, ROWB>;
     RingT ring;
-    ring.ring_s = smem_u32(wbase);
-    ring.bar0 = smem_u32(ybuf + kYbufFloats);
+    ring.ring_s = ring_s;
+    ring.bar0 = bar0;
     ring.len = len;
-    ring.nt = 2;
-    const int64_t seq_row0 = bh * p.L;
-    const int64_t row0 = seq_row0 + s;
+    ring.nt = NT;
+#pragma unroll
+    for (int q = 0; q < NT; ++q) ring.src[q] = reinterpret_cast<const unsigned char *>(p.d);
     ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + row0 * ROWB;
-    ring.src[1] = reinterpret_cast<const unsigned char *>(p.c) + row0 * ROWB;
-    ring_init_bars(ring.bar0, kFastStages, lane);
+    ring.src[CQ] = reinterpret_cast<const unsigned char *>(p.c) + row0 * ROWB;
+    constexpr unsigned kMask = 1u | (1u << CQ);
 
     const int ntiles = (len + kTS - 1) / kTS;
-    for (int i = 0; i < kFastStages && i < ntiles; ++i) ring.issue(i, lane);
+    for (int i = 0; i < kFastStages && i < ntiles; ++i) ring.issue_tile(tbase + i, i, kMask, lane);
 
     const uint32_t map_s = smem_u32(sd.map), yb_lane = smem_u32(ybuf) + lane * 4;
     constexpr int ES = (int)sizeof(T);
-    float w[NPL];
     int posb[NPL];   // column positions as byte offsets into a staged row
 #pragma unroll
-    for (int r = 0; r < NPL; ++r) {
-        const int e = lane * NPL + r;
-        posb[r] = e * ES;
-        w[r] = cidx == 0 ? p.h0[bh * p.N + e] : p.Hc[(unit - 1) * p.N + e];
-    }
+    for (int r = 0; r < NPL; ++r) posb[r] = (lane * NPL + r) * ES;
     const int32_t *kp = p.k + row0;
     float *yp = p.y + row0;
     int kreg = load_k(kp, lane, lane < kTS && lane < len, K, p.status);
 
     for (int i = 0; i < ntiles; ++i) {
-        if (!ring.wait(i)) {
-            ring.abort(i, ntiles, p.status, lane);
-            return;
+        if (!ring.wait(tbase + i)) {
+            if (lane == 0) flag_status(p.status, kStTimeout);
+            for (int j = i; j < ntiles && j < i + kFastStages; ++j) ring.wait(tbase + j);
+            __syncwarp();
+            return false;
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
         const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
         const float yold = ((lane & 3) == 0 && (lane >> 2) < n) ? yp[t0 + (lane >> 2)] : 0.f;
-        const uint32_t row0s = ring.tile(i);
+        const uint32_t row0s = ring.tile(tbase + i);
         if (n == kTS) {
             // full tile: steps unrolled, row and readout offsets immediate
             for_each_q(
@@ -262,7 +286,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
                     for (int r = 0; r < NPL; ++r) {
                         w[r] *= lds_elem_at<T, Q * ROWB>(row0s + posb[r]);
                         posb[r] = lds_next_pos<T>(pk + posb[r]);
-                        acc = fmaf(lds_elem_at<T, Q * ROWB + TENS>(row0s + posb[r]), w[r], acc);
+                        acc = fmaf(lds_elem_at<T, Q * ROWB + CQ * TENS>(row0s + posb[r]), w[r], acc);
                     }
                     sts_f32_at<Q * 33 * 4>(yb_lane, acc);
                 },
@@ -278,7 +302,7 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
                 for (int r = 0; r < NPL; ++r) {
                     w[r] *= lds_elem_at<T, 0>(row + posb[r]);
                     posb[r] = lds_next_pos<T>(pk + posb[r]);
-                    acc = fmaf(lds_elem_at<T, TENS>(row + posb[r]), w[r], acc);
+                    acc = fmaf(lds_elem_at<T, CQ * TENS>(row + posb[r]), w[r], acc);
                 }
                 sts_f32(yb, acc);
             }
@@ -287,8 +311,354 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
         const float ys = ybuf_quad_sum(ybuf, lane);
         if ((lane & 3) == 0 && (lane >> 2) < n) yp[t0 + (lane >> 2)] = yold + ys;
         warp_barrier();
-        if (i + kFastStages < ntiles) ring.issue(i + kFastStages, lane);
+        if (i + kFastStages < ntiles) ring.issue_tile(tbase + i + kFastStages, i + kFastStages, kMask, lane);
         kreg = clamp_k(knext, K, p.status);
+    }
+    return true;
+}
+
+template <typename T, int NPL>
+__global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams p) {
+    extern __shared__ __align__(128) unsigned char sm_c_raw[];
+    unsigned char *sm_c = smem_base256(sm_c_raw);
+    pdl_trigger();
+    pdl_wait();   // the carries come from the preceding kernel
+    constexpr int N = 32 * NPL;
+    constexpr int ROWB = N * (int)sizeof(T);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const SmemDict sd = stage_dict(p, sm_c, warp, lane, (int)sizeof(T));
+    const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
+    if (unit >= p.units) return;
+    const int64_t bh = unit / p.C, cidx = unit - bh * p.C;
+    if (cidx == 0 && p.h0 == nullptr) return;   // zero initial state: nothing to correct
+    const int64_t s = cidx * p.chunk;
+    const int len = (int)imin64(p.chunk, p.L - s);
+
+    unsigned char *wbase = sm_c + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
+    using RingT = FastRing<2, ROWB>;
+    float *ybuf = reinterpret_cast<float *>(wbase + kFastStages * RingT::STAGEB);   // [kTS][33]
+    const uint32_t bar0 = smem_u32(ybuf + kYbufFloats);
+    ring_init_bars(bar0, kFastStages, lane);
+    float w[NPL];
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        const int e = lane * NPL + r;
+        w[r] = cidx == 0 ? p.h0[bh * p.N + e] : p.Hc[(unit - 1) * p.N + e];
+    }
+    phaseC_segment<T, NPL, 2, 1>(p, sd, smem_u32(wbase), bar0, ybuf, bh * p.L + s, len, w, 0,
+                                 lane);
+}
+
+// ---------------------------------------------------------------------------
+// Single-pass forward (phases A, B and C in one kernel).
+//
+// One CTA per chunk; chunks are taken in the order of a ticket counter,
+// chunk-major (ticket t: chunk t / (B H) of sequence t % (B H)), so every
+// predecessor of a chunk in its sequence holds a smaller ticket and is
+// already running or done.  The chunk is cut into kFusedWarps sub-chunks,
+// one per warp:
+//   1. each warp runs phase A on its sub-chunk (local readout into y, the
+//      sub-chunk's closed transfer);
+//   2. an inclusive Hillis-Steele scan over the warps composes the
+//      sub-chunk transfers (log2 kFusedWarps rounds in shared memory): warp
+//      w holds T_w o ... o T_0, the last warp the chunk's transfer A_c;
+//   3. the last warp publishes A_c (flag kFlagAgg); warp 0 finds the carry
+//      H_{c-1} by decoupled look-back: the nearest predecessor with a
+//      published carry (kFlagIncl; the sequence start counts, with h0),
+//      then the aggregates of the predecessors after it applied in order;
+//      it publishes H_c = A_c(H_{c-1}) (kFlagIncl) and h_last;
+//   4. each warp takes its sub-chunk's carry (the exclusive prefix of the
+//      scan applied to H_{c-1}) and runs phase C on its sub-chunk; d and c
+//      were read a few microseconds before and are re-read from L2.
+// The workspace ends up holding the same chunk transfers (Pi_c, Delta_c,
+// v_c) and carries H_c as after the three-phase kernels, so the backward
+// pass reads either.  Every flag wait is bounded: a chunk whose wait gives
+// up flags PDSSM_ERR_TIMEOUT, takes a zero carry and still publishes, so no
+// successor waits on it.
+// ---------------------------------------------------------------------------
+constexpr int kFusedWarps = 8;
+enum : int { kFlagAgg = 1, kFlagIncl = 2 };
+
+// Transfer of chunk `unit` (as published by another CTA of this grid) in the
+// layout of transfer_ops.cuh; read through L2 (__ldcg), never the
+// non-coherent read-only path.
+__device__ __forceinline__ void load_published(const ChunkParams &p, int64_t unit, int lane,
+                                               int (&P)[2], float (&D)[2], float (&V)[2]) {
+    const int64_t o = unit * p.N;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int e = lane + 32 * r;
+        if (e < p.N) {
+            P[r] = __ldcg(p.Pi + o + e);
+            D[r] = __ldcg(p.Dl + o + e);
+            V[r] = __ldcg(p.v + o + e);
+        } else {
+            P[r] = kPadIdx;
+            D[r] = 0.f;
+            V[r] = 0.f;
+        }
+    }
+}
+
+// Carry H_{c-1} into chunk cidx of sequence bh (warp-collective; layout of
+// transfer_ops.cuh).  Each lane polls one predecessor flag; the window of 32
+// moves back while every flag in it is kFlagAgg.  Returns false if the wait
+// ran past p.wait_ns (x is then zero).
+__device__ __noinline__ bool lookback_carry(const ChunkParams &p, int64_t bh, int64_t cidx,
+                                            bool perm, ScatterScratch &sc, int lane,
+                                            float (&x)[2]) {
+    const int64_t u0 = bh * p.C;
+    int64_t top = cidx - 1;
+    int64_t base = -1;
+    bool ok = true;
+    const uint64_t t0 = global_ns();
+    for (;;) {
+        const int64_t j = top - lane;
+        // the sequence start counts as a published carry (h0)
+        const int f = j >= 0 ? ld_acquire_gpu(p.look + u0 + j) : kFlagIncl;
+        const unsigned incl = __ballot_sync(kFull, f >= kFlagIncl);
+        const unsigned none = __ballot_sync(kFull, f < kFlagAgg);
+        if (incl) {
+            const int i = __ffs(incl) - 1;
+            if ((none & ((1u << i) - 1u)) == 0) {
+                base = top - i;
+                break;
+            }
+        } else if (none == 0) {
+            top -= 32;   // all 32 hold aggregates only: look further back
+            continue;
+        }
+        if (global_ns() - t0 > p.wait_ns) {
+            ok = false;
+            break;
+        }
+        __nanosleep(100);
+    }
+    __syncwarp();
+    __threadfence();
+    if (!ok) {
+        if (lane == 0) flag_status(p.status, kStTimeout);
+        x[0] = x[1] = 0.f;
+        return false;
+    }
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        const int e = lane + 32 * r;
+        if (e >= p.N)
+            x[r] = 0.f;
+        else if (base >= 0)
+            x[r] = __ldcg(p.Hc + (u0 + base) * p.N + e);
+        else
+            x[r] = p.h0 ? p.h0[bh * p.N + e] : 0.f;
+    }
+    for (int64_t j = base + 1; j < cidx; ++j) {
+        int P[2];
+        float D[2], V[2], z[2];
+        load_published(p, u0 + j, lane, P, D, V);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) z[r] = D[r] * x[r];
+        warp_scatter(P, z, V, x, sc, lane, perm);
+    }
+    return true;
+}
+
+// Per-warp scratch of steps 2-4, inside the warp's staging ring (idle
+// between phase A and phase C): scan buffers [2][64] of P, D and V, the
+// scatter scratch, and one vector for the layout change of the carry.
+struct FusedScratch {
+    int P[2][64];
+    float D[2][64];
+    float V[2][64];
+    ScatterScratch sc;
+    float xs[64];
+};
+
+template <typename T, int NPL>
+__global__ void __launch_bounds__(kFusedWarps * 32, 3) k_scan_fused(const ChunkParams p) {
+    extern __shared__ __align__(128) unsigned char sm_f_raw[];
+    unsigned char *sm = smem_base256(sm_f_raw);
+    pdl_trigger();
+    pdl_wait();   // dictionary tables and cleared flags come from the preceding work
+    constexpr int N = 32 * NPL;
+    constexpr int ROWB = N * (int)sizeof(T);
+    constexpr int ES = (int)sizeof(T);
+    using RingT = FastRing<3, ROWB>;
+    static_assert(kFastStages * RingT::STAGEB >= (int)sizeof(FusedScratch),
+                  "scan scratch must fit the staging ring");
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    unsigned long long *s_ticket = reinterpret_cast<unsigned long long *>(sm);
+    float *s_carry = reinterpret_cast<float *>(sm + 64);            // [64]
+    unsigned char *dict_s = sm + 512;
+    if (threadIdx.x == 0) *s_ticket = atomicAdd(p.ticket, 1ull);
+    __syncthreads();
+    const int64_t tk = (int64_t)*s_ticket;
+    const int64_t BH = p.B * p.H;
+    const int64_t cidx = tk / BH, bh = tk - cidx * BH;
+    const int64_t unit = bh * p.C + cidx;
+    copy_slot(dict_s, p, p.dict_hs ? (bh % p.H) : 0, threadIdx.x, blockDim.x, ES);
+    __syncthreads();
+    const SmemDict sd = dict_view(p, dict_s);
+    const bool perm = __ldg(p.dict_stats + 1) <= 1;   // every map a permutation
+
+    // 1. phase A of this warp's sub-chunk
+    const int64_t s0 = cidx * p.chunk;
+    const int len = (int)imin64(p.chunk, p.L - s0);
+    const int S = (len + kFusedWarps - 1) / kFusedWarps;
+    const int ws0 = min(warp * S, len);
+    const int wlen = min(S, len - ws0);
+    const int64_t row0 = bh * p.L + s0 + ws0;
+    unsigned char *wbase =
+        dict_s + dict_slot_bytes((int)p.K, (int)p.N, p.dict_content) + (size_t)warp * p.smem_per_warp;
+    SegTransfer<NPL> tr;
+    bool ok;
+    switch (step_variant(p.dict_stats)) {
+        case 0: ok = phaseA_segment<T, NPL, 0>(p, sd, wbase, row0, wlen, lane, tr); break;
+        case 1: ok = phaseA_segment<T, NPL, 1>(p, sd, wbase, row0, wlen, lane, tr); break;
+        case 2: ok = phaseA_segment<T, NPL, 2>(p, sd, wbase, row0, wlen, lane, tr); break;
+        case 3: ok = phaseA_segment<T, NPL, 3>(p, sd, wbase, row0, wlen, lane, tr); break;
+        default: ok = phaseA_segment<T, NPL, 5>(p, sd, wbase, row0, wlen, lane, tr); break;
+    }
+    const int ntA = (wlen + kTS - 1) / kTS;
+    FusedScratch &fs = *reinterpret_cast<FusedScratch *>(wbase);
+    FusedScratch &last = *reinterpret_cast<FusedScratch *>(
+        dict_s + dict_slot_bytes((int)p.K, (int)p.N, p.dict_content) +
+        (size_t)(kFusedWarps - 1) * p.smem_per_warp);
+
+    // 2. the sub-chunk transfer into the scan layout, then the in-CTA scan
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) {
+        const int e = lane * NPL + r;
+        fs.P[0][e] = ok ? tr.pos[r] / ES : e;
+        fs.D[0][e] = ok ? tr.Dl[r] : 1.f;
+        fs.V[0][e] = ok ? tr.v[r] : 0.f;
+    }
+    if (NPL == 1) {   // padding elements 32 .. 63
+        fs.P[0][32 + lane] = kPadIdx;
+        fs.D[0][32 + lane] = 0.f;
+        fs.V[0][32 + lane] = 0.f;
+    }
+    __syncwarp();
+    Agg a;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+        a.P[r] = fs.P[0][lane + 32 * r];
+        a.D[r] = fs.D[0][lane + 32 * r];
+        a.V[r] = fs.V[0][lane + 32 * r];
+    }
+    __syncthreads();
+    int cur = 0;
+#pragma unroll
+    for (int dd = 1; dd < kFusedWarps; dd <<= 1) {
+        if (warp >= dd) {
+            // this warp's aggregate goes after warp (warp - dd)'s
+            const FusedScratch &src = *reinterpret_cast<const FusedScratch *>(
+                wbase - (size_t)dd * p.smem_per_warp);
+            Agg lo;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                lo.P[r] = src.P[cur][lane + 32 * r];
+                lo.D[r] = src.D[cur][lane + 32 * r];
+                lo.V[r] = src.V[cur][lane + 32 * r];
+            }
+            compose_after(lo, fs.P[cur], fs.D[cur], a.P, a.D, a.V, fs.sc, lane, perm);
+            a = lo;
+        }
+        const int nxt = cur ^ 1;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            fs.P[nxt][lane + 32 * r] = a.P[r];
+            fs.D[nxt][lane + 32 * r] = a.D[r];
+            fs.V[nxt][lane + 32 * r] = a.V[r];
+        }
+        cur = nxt;
+        __syncthreads();
+    }
+
+    // 3. publish the chunk's transfer; find and publish its carry
+    if (warp == kFusedWarps - 1) {
+        const int64_t o = unit * p.N;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int e = lane + 32 * r;
+            if (e < p.N) {
+                p.Pi[o + e] = a.P[r];
+                p.Dl[o + e] = a.D[r];
+                p.v[o + e] = a.V[r];
+            }
+        }
+        if (cidx > 0) {
+            __threadfence();
+            __syncwarp();
+            if (lane == 0) st_release_gpu(p.look + unit, kFlagAgg);
+        }
+    }
+    if (warp == 0) {
+        float x[2];
+        if (cidx == 0) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int e = lane + 32 * r;
+                x[r] = (p.h0 && e < p.N) ? p.h0[bh * p.N + e] : 0.f;
+            }
+        } else {
+            lookback_carry(p, bh, cidx, perm, fs.sc, lane, x);
+        }
+        // H_c = A_c(H_{c-1}) with A_c from the last warp's scan buffer
+        int P[2];
+        float z[2], hc[2], V[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            P[r] = last.P[cur][lane + 32 * r];
+            z[r] = last.D[cur][lane + 32 * r] * x[r];
+            V[r] = last.V[cur][lane + 32 * r];
+        }
+        warp_scatter(P, z, V, hc, fs.sc, lane, perm);
+        const int64_t o = unit * p.N;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int e = lane + 32 * r;
+            if (e < p.N) {
+                p.Hc[o + e] = hc[r];
+                if (cidx == p.C - 1 && p.h_last) p.h_last[bh * p.N + e] = hc[r];
+            }
+            s_carry[lane + 32 * r] = e < p.N ? x[r] : 0.f;
+        }
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) st_release_gpu(p.look + unit, kFlagIncl);
+    }
+    __syncthreads();
+
+    // 4. this sub-chunk's carry, then its carry correction
+    float xw[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) xw[r] = s_carry[lane + 32 * r];
+    if (warp > 0) {
+        const FusedScratch &prev = *reinterpret_cast<const FusedScratch *>(wbase - p.smem_per_warp);
+        int P[2];
+        float z[2], V[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            P[r] = prev.P[cur][lane + 32 * r];
+            z[r] = prev.D[cur][lane + 32 * r] * xw[r];
+            V[r] = prev.V[cur][lane + 32 * r];
+        }
+        warp_scatter(P, z, V, xw, fs.sc, lane, perm);
+    }
+    fs.xs[lane] = xw[0];
+    fs.xs[lane + 32] = xw[1];
+    __syncwarp();
+    float w[NPL];
+#pragma unroll
+    for (int r = 0; r < NPL; ++r) w[r] = fs.xs[lane * NPL + r];
+    // every warp is done with the scratch before copies land in the rings
+    fence_proxy_async_shared();
+    __syncthreads();
+    if (ok && wlen > 0 && !(cidx == 0 && warp == 0 && p.h0 == nullptr)) {
+        float *ybuf = reinterpret_cast<float *>(wbase + kFastStages * RingT::STAGEB) + 2 * kPbStride;
+        phaseC_segment<T, NPL, 3, 2>(p, sd, smem_u32(wbase), smem_u32(ybuf + kYbufFloats), ybuf,
+                                     row0, wlen, w, ntA, lane);
     }
 }
 
@@ -312,6 +682,56 @@ cudaError_t launch_phaseA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
                          : launch_fast(k_phaseA_fast<__nv_bfloat16, 1>, p, smem, st);
     return p.N == 64 ? launch_fast(k_phaseA_fast<float, 2>, p, smem, st)
                      : launch_fast(k_phaseA_fast<float, 1>, p, smem, st);
+}
+
+// Self-test of the bounded waits (a failure made on purpose, without a
+// fault): which = 0 runs the look-back of chunk 1 of a sequence whose chunk 0
+// never publishes; which = 1 waits on an mbarrier that nothing completes.
+// Either gives up after p.wait_ns and flags PDSSM_ERR_TIMEOUT.  One warp.
+__global__ void k_wait_selftest(const ChunkParams p, int which) {
+    __shared__ __align__(16) ScatterScratch sc;
+    __shared__ __align__(8) uint64_t bar;
+    const int lane = threadIdx.x & 31;
+    if (which == 0) {
+        float x[2];
+        lookback_carry(p, 0, 1, true, sc, lane, x);
+    } else {
+        if (lane == 0) {
+            mbar_init(smem_u32(&bar), 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
+        const bool done = mbar_wait_bounded(smem_u32(&bar), 0, p.wait_ns);
+        if (!done && lane == 0) flag_status(p.status, kStTimeout);
+    }
+}
+
+cudaError_t launch_wait_selftest(const ChunkParams &p, int which, cudaStream_t st) {
+    k_wait_selftest<<<1, 32, 0, st>>>(p, which);
+    return cudaGetLastError();
+}
+
+// The single-pass forward serves the fast-path shapes (one CTA per chunk:
+// the grid must fit the launch limit).
+bool fused_path(const ChunkParams &p) { return fast_path(p) && p.units <= 0x7fffffff; }
+
+// The single-pass forward: one CTA of kFusedWarps warps per chunk.
+cudaError_t launch_scan_fused(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
+    const int es = dt == PDSSM_BF16 ? 2 : 4;
+    p.dict_content = (dt == PDSSM_BF16 ? kDictMap16 : kDictMap) | kDictSeg;
+    p.smem_per_warp = warp_smem_bytes(kFastStages, 3, (int)p.N * es);
+    p.wpc = kFusedWarps;
+    const size_t smem = 512 + (size_t)dict_slot_bytes((int)p.K, (int)p.N, p.dict_content) +
+                        (size_t)kFusedWarps * p.smem_per_warp + 256;
+    auto go = [&](auto kern) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(kern, dim3((unsigned)p.units), dim3(kFusedWarps * 32), smem, st, p);
+    };
+    if (dt == PDSSM_BF16)
+        return p.N == 64 ? go(k_scan_fused<__nv_bfloat16, 2>) : go(k_scan_fused<__nv_bfloat16, 1>);
+    return p.N == 64 ? go(k_scan_fused<float, 2>) : go(k_scan_fused<float, 1>);
 }
 
 cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {

@@ -9,6 +9,7 @@
 // kStaticScratchBytes of device memory that every GPU which loads the
 // library holds until the process exits.
 #include <mutex>
+#include <stdio.h>
 
 #include "common.cuh"
 
@@ -24,7 +25,9 @@ std::mutex g_scratch_mu;
 
 // Device address of the static scratch array on `dev` (the current device).
 // In host code the array's name is only a host-side stand-in, so the device
-// address is looked up once per device and remembered.
+// address is looked up once per device and remembered for the process: the
+// library must not be used on a device across cudaDeviceReset (the array of
+// the new context would live elsewhere).
 cudaError_t scratch_address(int dev, void **out) {
     std::lock_guard<std::mutex> lock(g_scratch_mu);
     if (dev >= 0 && dev < kMaxDevices && g_scratch_ptr[dev]) {
@@ -39,6 +42,16 @@ cudaError_t scratch_address(int dev, void **out) {
     return cudaSuccess;
 }
 
+// The scratch of the current device, or a status (with its last-error text).
+pdssm_status current_scratch(void **ws) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return pdssm::cuda_fail(e, "cudaGetDevice");
+    e = scratch_address(dev, ws);
+    if (e != cudaSuccess) return pdssm::cuda_fail(e, "cudaGetSymbolAddress of the static scratch");
+    return PDSSM_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -50,17 +63,30 @@ pdssm_status pdssm_scan_fwd_noalloc(const pdssm_dims *dims, const int32_t *pi_di
                                     const void *b, const void *c, pdssm_dtype in_dtype,
                                     const float *h0, float *y, float *h_last, int64_t chunk,
                                     void *stream) {
+    // the same shape checks (and statuses) as pdssm_scan_fwd
+    pdssm_status st = pdssm::check_scan_dims(dims, pi_head_stride, chunk);
+    if (st != PDSSM_OK) return st;
     const size_t need = pdssm_workspace_bytes(dims, pi_head_stride, chunk, 0);
-    if (need == 0) return PDSSM_ERR_INVALID_ARG;
-    if (need > kStaticScratchBytes) return PDSSM_ERR_UNSUPPORTED;
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return PDSSM_ERR_CUDA;
+    if (need > kStaticScratchBytes) {
+        char why[160];
+        snprintf(why, sizeof(why), "workspace of %zu bytes exceeds the static scratch of %zu bytes",
+                 need, kStaticScratchBytes);
+        return pdssm::arg_fail(PDSSM_ERR_UNSUPPORTED, why);
+    }
     void *ws = nullptr;
-    if (scratch_address(dev, &ws) != cudaSuccess) return PDSSM_ERR_CUDA;
+    st = current_scratch(&ws);
+    if (st != PDSSM_OK) return st;
     // pdssm_scan_fwd clears the status word and overwrites every other part
     // of the workspace it reads, so what an earlier call left there is moot.
     return pdssm_scan_fwd(dims, pi_dict, pi_head_stride, k, d, b, c, in_dtype, h0, y, h_last,
                           chunk, ws, kStaticScratchBytes, stream);
+}
+
+pdssm_status pdssm_noalloc_status(void *stream) {
+    void *ws = nullptr;
+    const pdssm_status st = current_scratch(&ws);
+    if (st != PDSSM_OK) return st;
+    return pdssm_ws_status(ws, kStaticScratchBytes, stream);
 }
 
 }  // extern "C"

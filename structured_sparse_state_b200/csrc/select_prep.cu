@@ -109,10 +109,10 @@ static cudaError_t select_k(const pdssm_dims &dm, const void *u, const float *W,
 }
 
 cudaError_t launch_select(const pdssm_dims &dm, const void *u, pdssm_dtype ut, const float *W,
-                          int32_t *k_out, cudaStream_t st) {
+                          int32_t *k_out, bool use_tc, float *logits_out, float *scale_out,
+                          cudaStream_t st) {
     if (dm.B * dm.L == 0) return cudaSuccess;
-    if (select_tc_enabled() && select_tc_supported(dm, ut, u, W))
-        return launch_select_tc(dm, u, W, k_out, st);
+    if (use_tc) return launch_select_tc(dm, u, W, k_out, logits_out, scale_out, st);
     return ut == PDSSM_BF16 ? select_k<__nv_bfloat16>(dm, u, W, k_out, st)
                             : select_k<float>(dm, u, W, k_out, st);
 }

@@ -125,6 +125,8 @@ struct TcSelectParams {
     const float *W;          // [H][K][D] fp32
     const __nv_bfloat16 *u;  // [rows][D]
     int32_t *k_out;          // [B][H][L]
+    float *logits_out;       // test hook: raw tensor-core logits [rows][H*K], or NULL
+    float *scale_out;        // test hook: ||u_row|| * max_k ||W_hk|| (rounded up) [rows][H]
     int64_t rows, L;
     int D, H, K, NP;         // NP = H*K rounded up to 16
     int ntiles;
@@ -447,7 +449,13 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 float b1 = lg[0];
 #pragma unroll
                 for (int kk = 1; kk < KT; ++kk) b1 = fmaxf(b1, lg[kk]);
-                const float thr = b1 - 2.0f * __fmul_ru(__fmul_ru(unorm, Wn[h]), ceps);
+                const float S = __fmul_ru(unorm, Wn[h]);
+                const float thr = b1 - 2.0f * __fmul_ru(S, ceps);
+                if (p.logits_out) {
+#pragma unroll
+                    for (int kk = 0; kk < KT; ++kk) p.logits_out[row * (H * KT) + h * KT + kk] = lg[kk];
+                    p.scale_out[row * H + h] = S;
+                }
                 unsigned cand = 0;
 #pragma unroll
                 for (int kk = 0; kk < KT; ++kk) cand |= (lg[kk] >= thr ? 1u : 0u) << kk;
@@ -535,7 +543,7 @@ bool select_tc_supported(const pdssm_dims &dm, pdssm_dtype ut, const void *u, co
 }
 
 cudaError_t launch_select_tc(const pdssm_dims &dm, const void *u, const float *W, int32_t *k_out,
-                             cudaStream_t st) {
+                             float *logits_out, float *scale_out, cudaStream_t st) {
     const int64_t rows = dm.B * dm.L;
     const int D = (int)dm.D_in;
     const int NP = (int)((dm.H * dm.K + 15) / 16 * 16);
@@ -557,6 +565,8 @@ cudaError_t launch_select_tc(const pdssm_dims &dm, const void *u, const float *W
     p.W = W;
     p.u = reinterpret_cast<const __nv_bfloat16 *>(u);
     p.k_out = k_out;
+    p.logits_out = logits_out;
+    p.scale_out = scale_out;
     p.rows = rows;
     p.L = dm.L;
     p.D = D;

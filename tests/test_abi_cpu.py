@@ -106,3 +106,25 @@ def test_binding_refuses_cpu_tensors():
     W = torch.zeros(1, 2, 8)
     with pytest.raises(ValueError):
         pd.pdssm_select(u, W)
+
+
+def test_select_with_rejects_an_unknown_method():
+    dm = pd.dims(1, 1, 10, 0, 4, 16)
+    P = ctypes.c_void_p(256)
+    st = pd.lib().pdssm_select_with(ctypes.byref(dm), P, 0, P, P, 7, None)
+    assert st == 1 and "unknown selection method" in pd.last_error()
+
+
+def test_traced_calls_need_a_trace_with_two_events():
+    dm = pd.dims(1, 1, 10, 8, 4)
+    P = ctypes.c_void_p(256)
+    lib = pd.lib()
+    assert lib.pdssm_scan_fwd_traced(ctypes.byref(dm), P, 0, P, P, P, P, 0, None, P, None, 4,
+                                     P, 1 << 20, None, None) == 1
+    ev = (ctypes.c_void_p * 1)(None)
+    tr = pd.Trace()
+    tr.events = ctypes.cast(ev, ctypes.POINTER(ctypes.c_void_p))
+    tr.max_events = 1
+    assert lib.pdssm_scan_fwd_traced(ctypes.byref(dm), P, 0, P, P, P, P, 0, None, P, None, 4,
+                                     P, 1 << 20, None, ctypes.byref(tr)) == 1
+    assert "two events" in pd.last_error()

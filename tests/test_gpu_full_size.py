@@ -79,6 +79,10 @@ def test_full_size_bf16_selection_and_forward():
     t = to_device(inp)
     k, y, h_last, _ = _run_steps(inp, t, cfg["chunk"], select=True, grad=False)
     assert torch.isfinite(y).all() and torch.isfinite(h_last).all()
+    # deterministic: a second run gives the same bits
+    k2, y2, h2, _ = _run_steps(inp, t, cfg["chunk"], select=True, grad=False, steps=1)
+    assert torch.equal(k, k2) and torch.equal(y, y2) and torch.equal(h_last, h2)
+    del k2, y2, h2
     tol = tol_for(inp)
     for b, h in _rows(cfg["B"], cfg["H"], 4, seed=2):
         k_ref = oracle.select(inp.u[b:b + 1], inp.W[h:h + 1])          # [1, 1, L]
@@ -109,6 +113,9 @@ def test_full_size_stiff_impulse_forward():
     t = to_device(inp)
     _, y, h_last, _ = _run_steps(inp, t, cfg["chunk"], select=False, grad=False)
     assert torch.isfinite(y).all() and torch.isfinite(h_last).all()
+    _, y2, h2, _ = _run_steps(inp, t, cfg["chunk"], select=False, grad=False, steps=1)
+    assert torch.equal(y, y2) and torch.equal(h_last, h2)
+    del y2, h2
     n_big = 0
     for b, h in _rows(cfg["B"], cfg["H"], 5, seed=3):
         y_ref, hl_ref = oracle.scan_fwd(inp.pi, _slice(inp.k, b, h), _slice(inp.d, b, h),
@@ -125,6 +132,11 @@ def test_full_size_fp32_forward_and_adjoint():
     _, y, h_last, g = _run_steps(inp, t, cfg["chunk"], select=False, grad=True)
     for x in (y, h_last) + g:
         assert torch.isfinite(x).all()
+    _, y2, h2, g2 = _run_steps(inp, t, cfg["chunk"], select=False, grad=True, steps=1)
+    assert torch.equal(y, y2) and torch.equal(h_last, h2)
+    for a, a2 in zip(g, g2):
+        assert torch.equal(a, a2)
+    del y2, h2, g2
     for b, h in _rows(cfg["B"], cfg["H"], 6, seed=4):
         args = (inp.pi, _slice(inp.k, b, h), _slice(inp.d, b, h), _slice(inp.b, b, h),
                 _slice(inp.c, b, h), _slice(inp.h0, b, h))

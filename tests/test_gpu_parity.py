@@ -104,34 +104,95 @@ def test_select_near_ties_take_the_exact_path():
     assert not (kr == 5).any() or (kr == 3).any()
 
 
-def test_select_full_size_tensor_core_equals_fma_kernel(tmp_path):
-    """The full bf16 selection workload: the tensor-core kernel and the plain
-    fma-chain kernel (forced in a child process) agree on every index, and a
-    sample of rows matches the oracle."""
-    import subprocess
-    import sys
+def test_select_full_size_tensor_core_equals_fma_kernel():
+    """The full bf16 selection workload: the tensor-core route and the plain
+    fma-chain route agree on every index, and a sample of rows matches the
+    oracle."""
     inp = gen.generate(gen.workload(2))
     u = dev(inp.u, bf16=True)
     W = dev(inp.W)
-    k_tc = pd.pdssm_select(u, W).cpu().numpy()
-    np.save(tmp_path / "u.npy", inp.u)
-    np.save(tmp_path / "W.npy", inp.W)
-    code = (
-        "import sys, numpy as np, torch; sys.path.insert(0, %r);"
-        "import structured_sparse_state_b200 as pd;"
-        "u = torch.from_numpy(np.load(%r)).to(torch.bfloat16).cuda();"
-        "W = torch.from_numpy(np.load(%r)).cuda();"
-        "np.save(%r, pd.pdssm_select(u, W).cpu().numpy())"
-    ) % (str(__import__('pathlib').Path(__file__).resolve().parents[1]), str(tmp_path / "u.npy"),
-         str(tmp_path / "W.npy"), str(tmp_path / "k.npy"))
-    env = dict(__import__('os').environ, PDSSM_SELECT_FMA="1")
-    subprocess.run([sys.executable, "-c", code], check=True, env=env, timeout=600)
-    k_fma = np.load(tmp_path / "k.npy")
+    k_tc = pd.pdssm_select(u, W, method="tensor_core").cpu().numpy()
+    k_fma = pd.pdssm_select(u, W, method="fma").cpu().numpy()
     assert (k_tc == k_fma).all()
+    assert (pd.pdssm_select(u, W).cpu().numpy() == k_tc).all()
     rows = [0, 1, 7, 4095, 9999, 16383]
     for b in (0, 5):
         kr = oracle.select(inp.u[b:b + 1, rows], inp.W)
         assert (k_tc[b][:, rows] == kr[0]).all()
+
+
+def _exact_logits(u, W):
+    """Exact (fp64) sums u . W for bf16-valued u and fp32 W: every product is
+    exact in fp64 and D <= 256 sums of them lose far less than the bounds
+    checked here."""
+    B, L, D = u.shape
+    H, K, _ = W.shape
+    return u.reshape(B * L, D).astype(np.float64) @ W.reshape(H * K, D).astype(np.float64).T
+
+
+TC_ACC_BOUND = lambda D: D * 2.0 ** -21 + 2.0 ** -16   # noqa: E731
+
+
+@pytest.mark.parametrize("H,K,D", [(16, 16, 128), (4, 8, 64), (2, 32, 256), (8, 4, 48)])
+def test_select_tensor_core_logits_within_certified_bound(H, K, D):
+    """The certification assumes |tensor-core logit - exact sum| <=
+    (D 2^-21 + 2^-16) * ||u|| * max_k ||W_hk||.  Check it on raw logits
+    read through the test hook, against exact sums."""
+    rng = np.random.default_rng(4242 + D)
+    B, L = 2, 1000
+    u = gen.round_bf16(rng.standard_normal((B, L, D)).astype(np.float32))
+    u[0, :10] *= 1e3                       # a few large rows
+    u[1, :10] *= 1e-3                      # and a few small ones
+    u = gen.round_bf16(u)
+    W = (rng.standard_normal((H, K, D)) / np.sqrt(D)).astype(np.float32)
+    k, lg, sc = pd.pdssm_select_tc_logits(dev(u, bf16=True), dev(W))
+    lg = lg.cpu().numpy().astype(np.float64)
+    sc = np.repeat(sc.cpu().numpy().astype(np.float64), K, axis=1)
+    exact = _exact_logits(u, W)
+    # the scale is ||u|| max ||W_hk||, rounded up
+    un = np.sqrt((u.reshape(B * L, D).astype(np.float64) ** 2).sum(1))
+    wn = np.sqrt((W.astype(np.float64) ** 2).sum(2)).max(1)
+    assert (sc >= np.repeat(un[:, None] * wn[None, :], K, axis=1) * (1 - 1e-12)).all()
+    ratio = np.abs(lg - exact) / (TC_ACC_BOUND(D) * sc)
+    assert ratio.max() <= 1.0, f"tensor-core error {ratio.max():.3f} x the assumed bound"
+    assert (k.cpu().numpy() == oracle.select(u, W)).all()
+
+
+def test_select_gaps_just_above_the_certification_threshold():
+    """Rows whose top-2 gap lies in [2.2, 3.8] x eps (eps = the certification
+    half-width) are decided by the single-candidate branch; they must still
+    match the fma-chain contract bit for bit.  The two leading weights differ
+    only in the coefficient of u_0, so the gap is u_0 times it; the other
+    candidates sit far below through u_1."""
+    H, K, D, B, L = 4, 16, 128, 2, 2048
+    rng = np.random.default_rng(909)
+    W = (rng.standard_normal((H, 1, D)) / np.sqrt(D)).astype(np.float32).repeat(K, 1)
+    W[:, 1, 0] -= 1.0                          # l_0 - l_1 = u_0
+    W[:, 2:, 1] -= 0.5                         # l_k = l_0 - 0.5 u_1 for k >= 2
+    u = gen.round_bf16(rng.standard_normal((B, L, D)).astype(np.float32))
+    u[:, :, 1] = 4.0
+    ceps = 1.01 * (D * 2.0 ** -21 + 2.0 ** -16 + D * 2.0 ** -24)
+    wn = np.sqrt((W.astype(np.float64) ** 2).sum(2)).max()
+    target = rng.uniform(2.4, 3.6, (B, L)) * np.where(rng.random((B, L)) < 0.5, 1.0, -1.0)
+    for _ in range(3):                         # u_0 enters ||u|| slightly
+        un = np.sqrt((u.astype(np.float64) ** 2).sum(2))
+        u[:, :, 0] = target * ceps * un * wn * 1.002
+        u = gen.round_bf16(u)
+    ud, Wd = dev(u, bf16=True), dev(W)
+    k, lg, sc = pd.pdssm_select_tc_logits(ud, Wd)
+    kr = oracle.select(u, W)
+    assert (k.cpu().numpy() == kr).all()
+    assert set(np.unique(kr)) == {0, 1}
+    exact = _exact_logits(u, W).reshape(B * L, H, K)
+    gap = np.abs(exact[:, :, 0] - exact[:, :, 1])
+    eps = ceps * sc.cpu().numpy().astype(np.float64)
+    rel = gap / eps
+    assert ((rel > 2.0) & (rel < 4.0)).mean() > 0.95
+    lgn = lg.cpu().numpy().reshape(B * L, H, K).astype(np.float64)
+    thr = lgn.max(2) - 2 * eps
+    single = ((lgn >= thr[:, :, None]).sum(2) == 1)
+    assert single.sum() >= 0.9 * B * L * H, "most decisions take the certified branch"
+    assert (pd.pdssm_select(ud, Wd, method="fma").cpu().numpy() == kr).all()
 
 
 # ----------------------------------------------------------------------------
@@ -150,6 +211,68 @@ def test_chunk_transfers(idx, over, chunk):
     tol = tol_for(inp)
     assert floored_relerr(Dl.cpu().numpy(), Dl_r) <= tol
     assert floored_relerr(v.cpu().numpy(), v_r) <= tol
+
+
+# ----------------------------------------------------------------------------
+# single-pass forward (N = 32 / 64, aligned rows): look-back and in-CTA scan
+# ----------------------------------------------------------------------------
+def _prefix_states(inp, k_np, chunk):
+    """Oracle state at the end of every chunk: h_last of each prefix."""
+    L = inp.d.shape[2]
+    out = []
+    for e in range(chunk, L + chunk, chunk):
+        e = min(e, L)
+        _, h = oracle.scan_fwd(inp.pi, k_np[:, :, :e], inp.d[:, :, :e], inp.b[:, :, :e],
+                               inp.c[:, :, :e], inp.h0)
+        out.append(h)
+    return np.stack(out, axis=2)
+
+
+@pytest.mark.parametrize("kind", ["maps", "perm"])
+@pytest.mark.parametrize("N,dtype", [(32, "f32"), (64, "f32"), (32, "bf16"), (64, "bf16")])
+def test_single_pass_transfers_and_carries(N, dtype, kind):
+    """After the single-pass forward the workspace holds every chunk's
+    composed transfer (maps bit-exact against the oracle's step-by-step
+    composition) and the carry at every chunk end (the oracle's state)."""
+    inp = small(N + len(kind), 2, 3, 1000, N, 6, kind=kind, dtype=dtype)
+    chunk = 64
+    t = to_device(inp)
+    y, hl, ws = pd.pdssm_scan_fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=chunk)
+    Pi, Dl, v, Hc = pd.pdssm_ws_transfers(ws, 2, 3, 1000, N, 6, chunk)
+    torch.cuda.synchronize()
+    assert pd.pdssm_ws_status(ws) == 0
+    Pi_r, Dl_r, v_r = oracle.chunk_transfers(inp.pi, inp.k, inp.d, inp.b, chunk)
+    assert (Pi.cpu().numpy() == Pi_r).all()
+    tol = tol_for(inp)
+    assert floored_relerr(Dl.cpu().numpy(), Dl_r) <= tol
+    assert floored_relerr(v.cpu().numpy(), v_r) <= tol
+    assert floored_relerr(Hc.cpu().numpy(), _prefix_states(inp, inp.k, chunk)) <= tol
+
+
+@pytest.mark.parametrize("chunk", [1, 3, 7, 8, 9, 15, 17, 63, 65, 300])
+@pytest.mark.parametrize("N", [32, 64])
+def test_single_pass_chunk_sizes(chunk, N):
+    """Chunks shorter than the CTA's eight sub-chunks leave warps with empty
+    sub-chunks; ragged chunks and tails throughout."""
+    check_fwd(small(chunk + N, 1, 3, 777, N, 5), chunk=chunk)
+
+
+@pytest.mark.parametrize("N,kind", [(32, "perm"), (64, "maps")])
+def test_single_pass_long_look_back(N, kind):
+    """One sequence of 60000 steps in chunks of 8: hundreds of chunks of the
+    same sequence run at once, so look-backs walk back over whole windows of
+    published aggregates."""
+    check_fwd(small(5, 1, 1, 60000, N, 8, kind=kind), chunk=8)
+
+
+@pytest.mark.parametrize("which", [0, 1])
+def test_bounded_waits_time_out_and_report(which):
+    """A wait that nothing completes (a look-back flag no chunk publishes; an
+    mbarrier no copy completes) gives up after its cap and the host reads
+    PDSSM_ERR_TIMEOUT from the status word; the context stays usable."""
+    assert pd.pdssm_wait_selftest(which, 1_000_000) == 5
+    inp = small(3, 1, 1, 100, 32, 3)
+    check_fwd(inp, chunk=16)
 
 
 # ----------------------------------------------------------------------------
@@ -337,6 +460,29 @@ def test_forward_deterministic():
     y1, h1, _ = pd.pdssm_scan_fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=128)
     y2, h2, _ = pd.pdssm_scan_fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=128)
     assert torch.equal(y1, y2) and torch.equal(h1, h2)
+
+
+@pytest.mark.parametrize("idx,over,chunk", [(4, dict(B=1, H=4, L=4096), 128),
+                                             (1, dict(B=2, H=3, L=1500), 64),
+                                             (3, dict(H=4, L=3000), 256)])
+def test_backward_deterministic(idx, over, chunk):
+    """The adjoint's sums follow fixed trees: two runs give the same bits."""
+    inp = gen.generate(gen.workload(idx, **over))
+    if inp.k is None:
+        inp.k = oracle_k(inp)
+    if inp.g_y is None:
+        inp.g_y = np.random.default_rng(8).standard_normal(inp.d.shape[:3]).astype(np.float32)
+    t = to_device(inp)
+    kk = dev(inp.k, torch.int32)
+    gy = dev(inp.g_y)
+    outs = []
+    for _ in range(2):
+        y, hl, ws = pd.pdssm_scan_fwd(t["pi"], kk, t["d"], t["b"], t["c"], t["h0"], chunk=chunk,
+                                      for_bwd=True)
+        g = pd.pdssm_scan_bwd(t["pi"], kk, t["d"], t["b"], t["c"], t["h0"], gy, ws, chunk=chunk)
+        outs.append((y, hl) + tuple(g))
+    for a, b in zip(*outs):
+        assert torch.equal(a, b)
 
 
 # ----------------------------------------------------------------------------
