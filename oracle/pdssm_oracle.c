@@ -379,24 +379,29 @@ void oracle_scan_fwd_maps(int64_t B, int64_t H, int64_t L, int64_t N, const int3
  *
  * Flash PD-SSM technical summary, Methodology §2: the forward uses the hard
  * selection (argmax) and the hard dictionary (column hardmax); the backward
- * replaces both by tempered softmaxes so that gradients reach the selection
- * weights and the dense dictionary matrices (Proposition 2's surrogate
- * gradients, exact as tau -> 0; its expressions are not on the pages).
- * Reading taken here: the transition of step t is relaxed to
- *     T_t = sum_k s_{t,k} Q_k,   s_t = softmax(l_t * inv_tau_s),
- *     Q_k[:, j] = softmax(A_k[:, j] * inv_tau_a)   (column softmax),
- * and the loss gradient with respect to T_t is taken on the hard trajectory:
- *     dl/dT_t = lambda_t z_t^T,  z_t = d_t (.) h_{t-1},
- * lambda_t = dl/dh_t of the hard model (oracle_scan_bwd's g_b).  Then
- *     g_s[t,k] = lambda_t^T Q_k z_t
+ * replaces the discrete choices by tempered softmaxes so that gradients reach
+ * the selection weights and the dense dictionary matrices (Proposition 2's
+ * surrogate gradients, exact as tau -> 0; its expressions are not on the
+ * pages).  Reading taken here: each discrete choice is relaxed on its own,
+ * the other one held at its hard value, around the hard trajectory
+ * (lambda_t = dl/dh_t of the hard model, oracle_scan_bwd's g_b, and
+ * z_t = d_t (.) h_{t-1}):
+ *   selection:  T_t = sum_k s_{t,k} P_k,  s_t = softmax(l_t * inv_tau_s),
+ *               P_k the hard dictionary (column hardmax of A_k):
+ *     g_s[t,k] = lambda_t^T P_k z_t = sum_j lambda_t[pi_k(j)] z_t[j]
  *     g_l[t,k] = inv_tau_s s_{t,k} (g_s[t,k] - sum_k' s_{t,k'} g_s[t,k'])
  *     g_W[h,k,:] = sum_{b,t} g_l[b,h,t,k] u[b,t,:]
- *     g_Q[k] = sum_{b,h,t} s_{t,k} lambda_t z_t^T      (per head if a_hs != 0)
- *     g_A[k][:,j] = inv_tau_a Q_k[:,j] (.) (g_Q[k][:,j] - <Q_k[:,j], g_Q[k][:,j]>).
+ *   dictionary: T_t = Q_{k_t},  Q_k[:, j] = softmax(A_k[:, j] * inv_tau_a)
+ *               (column softmax), k_t the hard selection:
+ *     G_k = sum_{b,h,t : k_t = k} lambda_t z_t^T        (per head if a_hs != 0)
+ *     g_A[k][:,j] = inv_tau_a Q_k[:,j] (.) (G_k[:,j] - <Q_k[:,j], G_k[:,j]>).
  * These are exactly the gradients, at fixed lambda and z, of the linearised
- * loss G(W, A) = sum_t lambda_t^T T_t(W, A) z_t.  All in fp64 except the
- * logits (the fp32 fmaf chain of oracle_select, which also gives k_t) and
- * the hard dictionary (oracle_dict_hardmax of A).
+ * losses G_sel(W) = sum_t lambda_t^T (sum_k s_{t,k} P_k) z_t and
+ * G_dict(A) = sum_t lambda_t^T Q_{k_t} z_t.  Both keep the backward sparse:
+ * O(N K) per step for the selection, one O(N^2) outer product per step for
+ * the dictionary.  fp64 throughout except the logits (the fp32 fmaf chain of
+ * oracle_select, which also gives k_t) and the hard dictionary
+ * (oracle_dict_hardmax of A).
  * Loss: sum_t g_y[t] y_t + <g_hlast, h_{L-1}> (g_hlast may be NULL).
  * Outputs: g_l double [B][H][L][K], g_W double [H][K][D],
  * g_A double [Hd][K][N][N] with Hd = H if a_hs else 1.
@@ -410,7 +415,7 @@ void oracle_surrogate_grad(int64_t B, int64_t H, int64_t L, int64_t N, int64_t K
 {
     const int64_t Hd = a_hs ? H : 1;
     const int64_t NN = N * N;
-    /* hard dictionary and the column softmaxes */
+    /* hard dictionary, and the column softmaxes of the dictionary matrices */
     int32_t *pi = (int32_t *)malloc(sizeof(int32_t) * (size_t)(Hd * K * N));
     oracle_dict_hardmax(Hd * K, N, A, pi);
     double *Q = (double *)malloc(sizeof(double) * (size_t)(Hd * K * NN));
@@ -429,7 +434,7 @@ void oracle_surrogate_grad(int64_t B, int64_t H, int64_t L, int64_t N, int64_t K
             for (int64_t i = 0; i < N; ++i)
                 Q[m * NN + IDX2(i, j, N)] /= Z;
         }
-    /* hard selection and the hard trajectory with its adjoint */
+    /* hard selection, the hard trajectory and its adjoint */
     int32_t *k = (int32_t *)malloc(sizeof(int32_t) * (size_t)(B * H * L));
     oracle_select(B, L, D, H, K, u, W, k);
     double *g_b = (double *)malloc(sizeof(double) * (size_t)(B * H * L * N));
@@ -443,7 +448,7 @@ void oracle_surrogate_grad(int64_t B, int64_t H, int64_t L, int64_t N, int64_t K
     double *s = (double *)malloc(sizeof(double) * (size_t)K);
     double *gs = (double *)malloc(sizeof(double) * (size_t)K);
     double *z = (double *)malloc(sizeof(double) * (size_t)N);
-    double *gQ = (double *)calloc((size_t)(Hd * K * NN), sizeof(double));
+    double *G = (double *)calloc((size_t)(Hd * K * NN), sizeof(double));
     for (int64_t i = 0; i < H * K * D; ++i)
         g_W[i] = 0.0;
     for (int64_t bb = 0; bb < B; ++bb)
@@ -461,7 +466,9 @@ void oracle_surrogate_grad(int64_t B, int64_t H, int64_t L, int64_t N, int64_t K
                 const int64_t row = (bh * L + t) * N;
                 const double *lam = g_b + row;
                 const float *ur = u + (bb * L + t) * D;
-                /* logits in the fp32 contract, softmax in fp64 */
+                for (int64_t j = 0; j < N; ++j)
+                    z[j] = d[row + j] * hs[t * N + j];
+                /* selection: logits in the fp32 contract, softmax in fp64 */
                 double mx = 0.0;
                 for (int64_t kk = 0; kk < K; ++kk) {
                     const float *wr = W + (hh * K + kk) * D;
@@ -479,21 +486,14 @@ void oracle_surrogate_grad(int64_t B, int64_t H, int64_t L, int64_t N, int64_t K
                 }
                 for (int64_t kk = 0; kk < K; ++kk)
                     s[kk] /= Z;
-                for (int64_t j = 0; j < N; ++j)
-                    z[j] = d[row + j] * hs[t * N + j];
                 double sg = 0.0;
                 for (int64_t kk = 0; kk < K; ++kk) {
-                    const double *Qk = Q + (hd * K + kk) * NN;
+                    const int32_t *pq = pi + hd * K * N + kk * N;
                     double acc = 0.0;
-                    for (int64_t i = 0; i < N; ++i)
-                        for (int64_t j = 0; j < N; ++j)
-                            acc += lam[i] * Qk[IDX2(i, j, N)] * z[j];
+                    for (int64_t j = 0; j < N; ++j)
+                        acc += lam[pq[j]] * z[j];
                     gs[kk] = acc;
                     sg += s[kk] * acc;
-                    double *gQk = gQ + (hd * K + kk) * NN;
-                    for (int64_t i = 0; i < N; ++i)
-                        for (int64_t j = 0; j < N; ++j)
-                            gQk[IDX2(i, j, N)] += s[kk] * lam[i] * z[j];
                 }
                 for (int64_t kk = 0; kk < K; ++kk) {
                     const double gl = inv_tau_s * s[kk] * (gs[kk] - sg);
@@ -501,16 +501,21 @@ void oracle_surrogate_grad(int64_t B, int64_t H, int64_t L, int64_t N, int64_t K
                     for (int64_t q = 0; q < D; ++q)
                         g_W[(hh * K + kk) * D + q] += gl * (double)ur[q];
                 }
+                /* dictionary: the outer product joins the selected matrix's sum */
+                double *Gk = G + (hd * K + k[bh * L + t]) * NN;
+                for (int64_t i = 0; i < N; ++i)
+                    for (int64_t j = 0; j < N; ++j)
+                        Gk[IDX2(i, j, N)] += lam[i] * z[j];
             }
         }
     for (int64_t m = 0; m < Hd * K; ++m)
         for (int64_t j = 0; j < N; ++j) {
             double dotq = 0.0;
             for (int64_t i = 0; i < N; ++i)
-                dotq += Q[m * NN + IDX2(i, j, N)] * gQ[m * NN + IDX2(i, j, N)];
+                dotq += Q[m * NN + IDX2(i, j, N)] * G[m * NN + IDX2(i, j, N)];
             for (int64_t i = 0; i < N; ++i)
                 g_A[m * NN + IDX2(i, j, N)] =
-                    inv_tau_a * Q[m * NN + IDX2(i, j, N)] * (gQ[m * NN + IDX2(i, j, N)] - dotq);
+                    inv_tau_a * Q[m * NN + IDX2(i, j, N)] * (G[m * NN + IDX2(i, j, N)] - dotq);
         }
     free(pi);
     free(Q);
@@ -524,7 +529,7 @@ void oracle_surrogate_grad(int64_t B, int64_t H, int64_t L, int64_t N, int64_t K
     free(s);
     free(gs);
     free(z);
-    free(gQ);
+    free(G);
 }
 
 /* oracle_soft_exp over an array (for the tests). */

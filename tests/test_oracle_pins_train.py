@@ -222,22 +222,39 @@ def _softmax(x, axis):
     return e / e.sum(axis=axis, keepdims=True)
 
 
-def _linearised_loss(u, W, A, inv_s, inv_a, lam, z):
-    """G(W, A) = sum_t lambda_t^T (sum_k s_{t,k} Q_k) z_t in fp64 (dense)."""
+def _sel_loss(u, W, pi, inv_s, lam, z):
+    """G_sel(W) = sum_t lambda_t^T (sum_k s_{t,k} P_k) z_t, with dense P_k."""
     lg = np.einsum("hkd,bld->bhlk", W, u.astype(np.float64))
     s = _softmax(lg * inv_s, axis=-1)
+    N = pi.shape[-1]
+    P = np.zeros(pi.shape[:-1] + (N, N))
+    np.put_along_axis(P, pi[..., None, :], 1.0, axis=-2)
+    if P.ndim == 3:
+        return float(np.einsum("bhlk,bhli,kij,bhlj->", s, lam, P, z))
+    return float(np.einsum("bhlk,bhli,hkij,bhlj->", s, lam, P, z))
+
+
+def _dict_loss(A, k, inv_a, lam, z):
+    """G_dict(A) = sum_t lambda_t^T Q_{k_t} z_t, Q the column softmaxes."""
     Q = _softmax(A * inv_a, axis=-2)
-    if Q.ndim == 3:
-        return float(np.einsum("bhlk,bhli,kij,bhlj->", s, lam, Q, z))
-    return float(np.einsum("bhlk,bhli,hkij,bhlj->", s, lam, Q, z))
+    B, H, L = k.shape
+    total = 0.0
+    for bb in range(B):
+        for hh in range(H):
+            for t in range(L):
+                Qk = Q[k[bb, hh, t]] if Q.ndim == 3 else Q[hh, k[bb, hh, t]]
+                total += lam[bb, hh, t] @ Qk @ z[bb, hh, t]
+    return total
 
 
 @pytest.mark.parametrize("per_head", [False, True])
-def test_surrogate_gradients_match_finite_differences_of_the_linearised_loss(per_head):
+def test_surrogate_gradients_match_finite_differences_of_the_linearised_losses(per_head):
     u, W, A, d, b, c, h0, g_y = _train_case(11, per_head=per_head)
     inv_s, inv_a = 1.7, 2.3
     g_l, g_W, g_A = oracle.surrogate_grad(u, W, A, inv_s, inv_a, d, b, c, h0, g_y)
     lam, z = _hard_trajectory(u, W, A, d, b, c, h0, g_y)
+    pi = oracle.dict_hardmax(A)
+    k = oracle.select(u, W)
     W64, A64 = W.astype(np.float64), A.astype(np.float64)
     eps = 1e-6
     rng = np.random.default_rng(0)
@@ -246,23 +263,36 @@ def test_surrogate_gradients_match_finite_differences_of_the_linearised_loss(per
         Wp, Wm = W64.copy(), W64.copy()
         Wp[idx] += eps
         Wm[idx] -= eps
-        fd = (_linearised_loss(u, Wp, A64, inv_s, inv_a, lam, z) -
-              _linearised_loss(u, Wm, A64, inv_s, inv_a, lam, z)) / (2 * eps)
+        fd = (_sel_loss(u, Wp, pi, inv_s, lam, z) - _sel_loss(u, Wm, pi, inv_s, lam, z)) / (2 * eps)
         assert abs(fd - g_W[idx]) <= 1e-5 * max(1.0, abs(fd)), (idx, fd, g_W[idx])
     for _ in range(12):
         idx = tuple(int(rng.integers(0, n)) for n in A.shape)
         Ap, Am = A64.copy(), A64.copy()
         Ap[idx] += eps
         Am[idx] -= eps
-        fd = (_linearised_loss(u, W64, Ap, inv_s, inv_a, lam, z) -
-              _linearised_loss(u, W64, Am, inv_s, inv_a, lam, z)) / (2 * eps)
+        fd = (_dict_loss(Ap, k, inv_a, lam, z) - _dict_loss(Am, k, inv_a, lam, z)) / (2 * eps)
         assert abs(fd - g_A[idx]) <= 1e-5 * max(1.0, abs(fd)), (idx, fd, g_A[idx])
+    # the logit gradients are the same derivative taken at the logits
+    lg = np.einsum("hkd,bld->bhlk", W64, u.astype(np.float64))
+    for _ in range(6):
+        bb, hh, t, kk = (int(rng.integers(0, n)) for n in g_l.shape)
+        P = np.zeros(pi.shape[:-1] + (pi.shape[-1],) * 2)
+        np.put_along_axis(P, pi[..., None, :], 1.0, axis=-2)
+        Pk = P if P.ndim == 3 else P[hh]
+
+        def at(delta):
+            x = lg[bb, hh, t].copy()
+            x[kk] += delta
+            s = _softmax(x * inv_s, axis=-1)
+            return float(np.einsum("k,i,kij,j->", s, lam[bb, hh, t], Pk, z[bb, hh, t]))
+        fd = (at(eps) - at(-eps)) / (2 * eps)
+        assert abs(fd - g_l[bb, hh, t, kk]) <= 1e-5 * max(1.0, abs(fd))
 
 
 def test_surrogate_logit_gradients_sum_to_zero_and_vanish_for_equal_matrices():
     """softmax is invariant to a common shift of the logits, so each step's
-    logit gradients sum to zero; with all A_k equal the relaxed transition
-    does not depend on the weights at all."""
+    logit gradients sum to zero; with all A_k equal every selector is the
+    same, so the relaxed transition does not depend on the weights at all."""
     u, W, A, d, b, c, h0, g_y = _train_case(12)
     g_l, g_W, g_A = oracle.surrogate_grad(u, W, A, 1.3, 1.0, d, b, c, h0, g_y)
     assert np.max(np.abs(g_l.sum(-1))) <= 1e-12 * max(1.0, np.max(np.abs(g_l)))
