@@ -229,6 +229,96 @@ pdssm_status pdssm_scan_bwd_traced(const pdssm_dims *dims,
                                    void *stream, pdssm_trace *trace);
 
 /*
+ * Dictionary from dense matrices (Flash PD-SSM technical summary,
+ * Methodology §1: the dictionary holds column one-hot selectors, the column
+ * hardmax of dense matrices):
+ *     pi_out[m][j] = first i maximising A[m][i][j]   (strict >, ascending i)
+ * for the n_mats matrices A [n_mats][N][N] (fp32, device); pi_out int32
+ * [n_mats][N] (device) is then a dictionary for pdssm_scan_fwd (n_mats = K,
+ * or H*K with pi_head_stride = K*N).  1 <= N <= 64.
+ */
+pdssm_status pdssm_dict_hardmax(int64_t n_mats, int64_t N, const float *A,
+                                int32_t *pi_out, void *stream);
+
+/*
+ * The original PD-SSM's input-dependent transitions (Methodology §1: a
+ * convex combination of dense dictionary matrices, sparsified by a column
+ * hardmax), as a dense comparison path for the hard selection.  For every
+ * (b, h, t), in this fixed fp32 arithmetic:
+ *   l_k  = the fma chain of pdssm_select (W_sel[h][k] . u[b][t], ascending q),
+ *   m    = max_k l_k,  e_k = exp_soft((l_k - m) * inv_tau),  Z = sum_k e_k
+ *          (ascending k),  s_k = e_k / Z,
+ *   M[i][j] = fmaf chain over ascending k of s_k * A_k[i][j] (from 0),
+ *   maps_out[b][h][t][j] = first i maximising M[i][j],
+ * where exp_soft(x) (x <= 0) is Cody-Waite reduction x = n ln2 + r (ln2 as
+ * 0.693145751953125 + 1.42860677e-06), the degree-7 Taylor polynomial of e^r
+ * in Horner form with fmaf, times 2^n; 0 for x < -86.  Dictionary matrix
+ * (h, k) at A + h*a_head_stride + k*N*N (a_head_stride = 0: shared by the
+ * heads).  u [B][L][D_in] (fp32 or bf16), W_sel [H][K][D_in] fp32, A fp32,
+ * maps_out int32 [B][H][L][N], all device.  Costs O(N^2 K) per step.
+ */
+pdssm_status pdssm_soft_maps(const pdssm_dims *dims, const void *u,
+                             pdssm_dtype u_dtype, const float *W_sel,
+                             const float *A, int64_t a_head_stride,
+                             float inv_tau, int32_t *maps_out, void *stream);
+
+/*
+ * Forward scan with one column-selector map per step (the transitions of
+ * pdssm_soft_maps): as pdssm_scan_fwd with pi_{k_t} replaced by
+ * maps[b][h][t] (int32 [B][H][L][N], entries in [0, N)).  Sequential in t,
+ * one warp per (b, h); needs no workspace.  y [B][H][L] and h_last [B][H][N]
+ * (may be NULL) fp32; h0 may be NULL.
+ */
+pdssm_status pdssm_scan_fwd_maps(const pdssm_dims *dims, const int32_t *maps,
+                                 const void *d, const void *b, const void *c,
+                                 pdssm_dtype in_dtype, const float *h0,
+                                 float *y, float *h_last, void *stream);
+
+/*
+ * Straight-through surrogate gradients of the hard selection and of the
+ * column-hardmax dictionary (Flash PD-SSM technical summary, Methodology
+ * §2: hard forward; in the backward the discrete choices are replaced by
+ * tempered softmaxes so that gradients reach the selection weights W_sel
+ * and the dense dictionary matrices A; the pages do not print Proposition
+ * 2's expressions).  Reading: each choice is relaxed on its own around the
+ * hard trajectory, with lambda_t = dl/dh_t (pdssm_scan_bwd's g_b) and
+ * z_t = d_t (.) h_{t-1}:
+ *   selection  (softmax over the hard selectors P_k, weights
+ *               s_t = softmax(l_t * inv_tau_s), l_t the logits of pdssm_select):
+ *     g_s[t,k]    = sum_j lambda_t[pi_k(j)] z_t[j]
+ *     g_logits[b][h][t][k] = inv_tau_s s_k (g_s[t,k] - sum_k' s_k' g_s[t,k'])
+ *     g_W[h][k][:] = sum_{b,t} g_logits[b][h][t][k] u[b][t][:]
+ *   dictionary (column softmax Q_k of A_k * inv_tau_a for the selected k_t):
+ *     G_k = sum_{b,h,t : k_t = k} lambda_t z_t^T
+ *     g_A[k][:,j] = inv_tau_a Q_k[:,j] (.) (G_k[:,j] - <Q_k[:,j], G_k[:,j]>)
+ * The costs stay those of the hard model: O(N K) per step for the selection,
+ * one N x N outer product per step for the dictionary.
+ * Preconditions (same dims, chunk, dictionary): pi_dict = pdssm_dict_hardmax
+ * of A ([Hd][K][N], Hd = H when a_head_stride = K*N*N, else 1); k = the hard
+ * selection; pdssm_scan_fwd ran with workspace `ws` (its carries are read)
+ * and pi_head_stride = K*N when A is per head; lambda = g_b of
+ * pdssm_scan_bwd.  u [B][L][D_in] (fp32 / bf16), W_sel [H][K][D_in] fp32,
+ * A fp32 (matrix (h, k) at A + h*a_head_stride + k*N*N), d, b of in_dtype,
+ * h0 fp32 or NULL.  Outputs fp32: g_logits [B][H][L][K], g_W [H][K][D_in],
+ * g_A like A.  scratch: pdssm_surrogate_scratch_bytes(dims, a_head_stride)
+ * bytes, 256-byte aligned.  Deterministic (every sum in a fixed order).
+ */
+size_t pdssm_surrogate_scratch_bytes(const pdssm_dims *dims,
+                                     int64_t a_head_stride);
+pdssm_status pdssm_surrogate_bwd(const pdssm_dims *dims, const void *u,
+                                 pdssm_dtype u_dtype, const float *W_sel,
+                                 const float *A, int64_t a_head_stride,
+                                 const int32_t *pi_dict, const int32_t *k,
+                                 const void *d, const void *b,
+                                 pdssm_dtype in_dtype, const float *h0,
+                                 const float *lambda, int64_t chunk,
+                                 const void *ws, size_t ws_bytes,
+                                 float inv_tau_s, float inv_tau_a,
+                                 void *scratch, size_t scratch_bytes,
+                                 float *g_logits, float *g_W, float *g_A,
+                                 void *stream);
+
+/*
  * pdssm_scan_fwd for callers that cannot allocate device memory.  The pages
  * have no counterpart of this call: it exists for host code that owns no
  * allocator (device memory held by another framework's pool), must not call

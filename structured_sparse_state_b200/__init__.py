@@ -37,7 +37,9 @@ EXPORTS = ("pdssm_status_str", "pdssm_last_error", "pdssm_version",
            "pdssm_ws_status", "pdssm_scan_fwd_noalloc", "pdssm_noalloc_scratch_bytes",
            "pdssm_select_with", "pdssm_select_tc_logits", "pdssm_noalloc_status",
            "pdssm_scan_fwd_traced", "pdssm_scan_bwd_traced", "pdssm_ws_transfers",
-           "pdssm_wait_selftest", "pdssm_wait_selftest_ws_bytes")
+           "pdssm_wait_selftest", "pdssm_wait_selftest_ws_bytes", "pdssm_dict_hardmax",
+           "pdssm_soft_maps", "pdssm_scan_fwd_maps", "pdssm_surrogate_scratch_bytes",
+           "pdssm_surrogate_bwd")
 
 TRACE_MAX_KERNELS = 8
 
@@ -88,6 +90,12 @@ def _load() -> ctypes.CDLL:
         "pdssm_ws_transfers": (I32, [D, I64, I64, P, SZ, P, P, P, P, P]),
         "pdssm_wait_selftest": (I32, [I32, I64, P, SZ, P]),
         "pdssm_wait_selftest_ws_bytes": (SZ, []),
+        "pdssm_dict_hardmax": (I32, [I64, I64, P, P, P]),
+        "pdssm_soft_maps": (I32, [D, P, I32, P, P, I64, ctypes.c_float, P, P]),
+        "pdssm_scan_fwd_maps": (I32, [D, P, P, P, P, I32, P, P, P, P]),
+        "pdssm_surrogate_scratch_bytes": (SZ, [D, I64]),
+        "pdssm_surrogate_bwd": (I32, [D, P, I32, P, P, I64, P, P, P, P, I32, P, P, I64, P, SZ,
+                                      ctypes.c_float, ctypes.c_float, P, SZ, P, P, P, P]),
         "pdssm_scan_fwd_traced": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, I64, P, SZ, P,
                                         ctypes.POINTER(Trace)]),
         "pdssm_scan_bwd_traced": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, P, P, P, P, I64,
@@ -452,3 +460,107 @@ def pdssm_scan_bwd_traced(pi_dict, k, d, b, c, h0, g_y, ws, chunk, out, events, 
                                       ctypes.byref(tr)),
            "pdssm_scan_bwd_traced")
     return lambda: _trace_result(tr, events)
+
+
+# ----------------------------------------------------------------------------
+# dictionary from dense matrices; the original soft selection (comparison)
+# ----------------------------------------------------------------------------
+def pdssm_dict_hardmax(A: torch.Tensor, stream=None) -> torch.Tensor:
+    """pi[..., j] = first argmax_i A[..., i, j] for dense [..., N, N] fp32 A."""
+    _cuda(A, "A", (torch.float32,))
+    N = A.shape[-1]
+    if A.shape[-2] != N:
+        raise ValueError("A must be [..., N, N]")
+    pi = torch.empty(A.shape[:-1], dtype=torch.int32, device=A.device)
+    n = A.numel() // (N * N)
+    _check(_lib.pdssm_dict_hardmax(n, N, _ptr(A), _ptr(pi), _stream(stream)),
+           "pdssm_dict_hardmax")
+    return pi
+
+
+def pdssm_soft_maps(u, W_sel, A, inv_tau, maps_out=None, stream=None):
+    """Per-step column-hardmax maps of the soft-selection mixture (the
+    original PD-SSM's transitions); returns int32 [B, H, L, N]."""
+    _cuda(u, "u", (torch.float32, torch.bfloat16))
+    _cuda(W_sel, "W_sel", (torch.float32,))
+    B, L, D = u.shape
+    H, K, D2 = W_sel.shape
+    if D != D2:
+        raise ValueError("u and W_sel disagree on D_in")
+    _cuda(A, "A", (torch.float32,))
+    N = A.shape[-1]
+    if A.dim() == 3:
+        a_hs = 0
+        if tuple(A.shape) != (K, N, N):
+            raise ValueError("A must be [K, N, N] or [H, K, N, N]")
+    else:
+        a_hs = K * N * N
+        if tuple(A.shape) != (H, K, N, N):
+            raise ValueError("A must be [K, N, N] or [H, K, N, N]")
+    if maps_out is None:
+        maps_out = torch.empty((B, H, L, N), dtype=torch.int32, device=u.device)
+    _cuda(maps_out, "maps_out", (torch.int32,))
+    dm = dims(B, H, L, N, K, D)
+    _check(_lib.pdssm_soft_maps(ctypes.byref(dm), _ptr(u), _dtype_code(u), _ptr(W_sel),
+                                _ptr(A), a_hs, float(inv_tau), _ptr(maps_out), _stream(stream)),
+           "pdssm_soft_maps")
+    return maps_out
+
+
+def pdssm_scan_fwd_maps(maps, d, b, c, h0=None, y=None, h_last=None, stream=None):
+    """Forward scan with one map per step; returns (y, h_last)."""
+    _cuda(maps, "maps", (torch.int32,))
+    _cuda(d, "d", (torch.float32, torch.bfloat16))
+    B, H, L, N = d.shape
+    if tuple(maps.shape) != (B, H, L, N):
+        raise ValueError("maps must be [B, H, L, N]")
+    for name, t in (("b", b), ("c", c)):
+        _cuda(t, name, (d.dtype,))
+        if t.shape != d.shape:
+            raise ValueError(f"{name} shape differs from d")
+    if h0 is not None:
+        _cuda(h0, "h0", (torch.float32,))
+    if y is None:
+        y = torch.empty((B, H, L), dtype=torch.float32, device=d.device)
+    if h_last is None:
+        h_last = torch.empty((B, H, N), dtype=torch.float32, device=d.device)
+    dm = dims(B, H, L, N, 1)
+    _check(_lib.pdssm_scan_fwd_maps(ctypes.byref(dm), _ptr(maps), _ptr(d), _ptr(b), _ptr(c),
+                                    _dtype_code(d), _ptr(h0), _ptr(y), _ptr(h_last),
+                                    _stream(stream)), "pdssm_scan_fwd_maps")
+    return y, h_last
+
+
+# ----------------------------------------------------------------------------
+# straight-through surrogate gradients
+# ----------------------------------------------------------------------------
+def pdssm_surrogate_bwd(u, W_sel, A, pi_dict, k, d, b, h0, lam, ws, chunk, inv_tau_s,
+                        inv_tau_a, stream=None):
+    """Surrogate gradients (g_logits [B,H,L,K], g_W like W_sel, g_A like A)
+    of the hard model; pi_dict = pdssm_dict_hardmax(A), ws = the forward's
+    workspace, lam = g_b of pdssm_scan_bwd.  Allocates its scratch."""
+    _cuda(u, "u", (torch.float32, torch.bfloat16))
+    _cuda(W_sel, "W_sel", (torch.float32,))
+    _cuda(A, "A", (torch.float32,))
+    _cuda(lam, "lambda", (torch.float32,))
+    _cuda(ws, "ws", (torch.uint8,))
+    B, H, L, N, K, _ = _scan_shapes(pi_dict, k, d, b, None)
+    D = u.shape[-1]
+    a_hs = K * N * N if A.dim() == 4 else 0
+    if h0 is not None:
+        _cuda(h0, "h0", (torch.float32,))
+    dm = dims(B, H, L, N, K, D)
+    nbytes = int(_lib.pdssm_surrogate_scratch_bytes(ctypes.byref(dm), a_hs))
+    if nbytes == 0:
+        raise PdssmError(1, "pdssm_surrogate_scratch_bytes")
+    scratch = torch.empty(nbytes, dtype=torch.uint8, device=d.device)
+    g_l = torch.empty((B, H, L, K), dtype=torch.float32, device=d.device)
+    g_W = torch.empty_like(W_sel)
+    g_A = torch.empty_like(A)
+    _check(_lib.pdssm_surrogate_bwd(ctypes.byref(dm), _ptr(u), _dtype_code(u), _ptr(W_sel),
+                                    _ptr(A), a_hs, _ptr(pi_dict), _ptr(k), _ptr(d), _ptr(b),
+                                    _dtype_code(d), _ptr(h0), _ptr(lam), int(chunk), _ptr(ws),
+                                    ws.numel(), float(inv_tau_s), float(inv_tau_a),
+                                    _ptr(scratch), nbytes, _ptr(g_l), _ptr(g_W), _ptr(g_A),
+                                    _stream(stream)), "pdssm_surrogate_bwd")
+    return g_l, g_W, g_A

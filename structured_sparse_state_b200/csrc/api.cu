@@ -436,6 +436,108 @@ pdssm_status pdssm_ws_transfers(const pdssm_dims *dims, int64_t pi_head_stride, 
     return PDSSM_OK;
 }
 
+pdssm_status pdssm_dict_hardmax(int64_t n_mats, int64_t N, const float *A, int32_t *pi_out,
+                                void *stream) {
+    if (n_mats < 0 || N < 1 || N > kMaxN)
+        return arg_fail(N > kMaxN ? PDSSM_ERR_UNSUPPORTED : PDSSM_ERR_INVALID_ARG,
+                        "need n_mats >= 0 and 1 <= N <= 64");
+    if (n_mats == 0) return PDSSM_OK;
+    if (!A || !pi_out) return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL pointer");
+    cudaError_t e = launch_dict_hardmax(n_mats, (int)N, A, pi_out, (cudaStream_t)stream);
+    return e == cudaSuccess ? PDSSM_OK : cuda_fail(e, "dictionary hardmax");
+}
+
+pdssm_status pdssm_soft_maps(const pdssm_dims *dims, const void *u, pdssm_dtype u_dtype,
+                             const float *W_sel, const float *A, int64_t a_head_stride,
+                             float inv_tau, int32_t *maps_out, void *stream) {
+    if (!dims) return arg_fail(PDSSM_ERR_INVALID_ARG, "dims is NULL");
+    if (check_dtype(u_dtype) != PDSSM_OK) return PDSSM_ERR_INVALID_ARG;
+    if (dims->B < 1 || dims->H < 1 || dims->L < 0 || dims->N < 1 || dims->K < 1 ||
+        dims->D_in < 1)
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "need B, H, N, K, D_in >= 1 and L >= 0");
+    if (dims->N > kMaxN || dims->K > 32 || dims->D_in > 256)
+        return arg_fail(PDSSM_ERR_UNSUPPORTED, "N > 64, K > 32 or D_in > 256");
+    if (a_head_stride != 0 && a_head_stride < dims->K * dims->N * dims->N)
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "a_head_stride must be 0 or >= K*N*N");
+    if (!(inv_tau > 0.f) || inv_tau > 3.0e38f)
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "inv_tau must be positive and finite");
+    if (dims->L == 0) return PDSSM_OK;
+    if (!u || !W_sel || !A || !maps_out) return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL pointer");
+    cudaError_t e = launch_soft_maps(*dims, u, u_dtype, W_sel, A, a_head_stride, inv_tau,
+                                     maps_out, (cudaStream_t)stream);
+    return e == cudaSuccess ? PDSSM_OK : cuda_fail(e, "soft maps");
+}
+
+pdssm_status pdssm_scan_fwd_maps(const pdssm_dims *dims, const int32_t *maps, const void *d,
+                                 const void *b, const void *c, pdssm_dtype in_dtype,
+                                 const float *h0, float *y, float *h_last, void *stream) {
+    pdssm_status st = check_scan_dims(dims, 0, 1);
+    if (st != PDSSM_OK) return st;
+    if (check_dtype(in_dtype) != PDSSM_OK) return PDSSM_ERR_INVALID_ARG;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (dims->L == 0) {
+        if (h_last) {
+            const size_t bytes = (size_t)(dims->B * dims->H * dims->N) * 4;
+            cudaError_t e = h0 ? cudaMemcpyAsync(h_last, h0, bytes, cudaMemcpyDeviceToDevice, s)
+                               : cudaMemsetAsync(h_last, 0, bytes, s);
+            if (e != cudaSuccess) return cuda_fail(e, "h_last for L = 0");
+        }
+        return PDSSM_OK;
+    }
+    if (!maps || !d || !b || !c || !y) return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL pointer");
+    cudaError_t e = launch_scan_maps(*dims, maps, d, b, c, in_dtype, h0, y, h_last, s);
+    return e == cudaSuccess ? PDSSM_OK : cuda_fail(e, "scan with per-step maps");
+}
+
+static pdssm_status check_surrogate_dims(const pdssm_dims *dims, int64_t a_hs) {
+    if (!dims) return arg_fail(PDSSM_ERR_INVALID_ARG, "dims is NULL");
+    if (dims->B < 1 || dims->H < 1 || dims->L < 0 || dims->N < 1 || dims->K < 1 ||
+        dims->D_in < 1)
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "need B, H, N, K, D_in >= 1 and L >= 0");
+    if (dims->N > kMaxN || dims->K > 32 || dims->D_in > 256)
+        return arg_fail(PDSSM_ERR_UNSUPPORTED, "N > 64, K > 32 or D_in > 256");
+    if (a_hs != 0 && a_hs < dims->K * dims->N * dims->N)
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "a_head_stride must be 0 or >= K*N*N");
+    return PDSSM_OK;
+}
+
+size_t pdssm_surrogate_scratch_bytes(const pdssm_dims *dims, int64_t a_head_stride) {
+    if (check_surrogate_dims(dims, a_head_stride) != PDSSM_OK) return 0;
+    return surrogate_scratch_bytes(*dims, a_head_stride);
+}
+
+pdssm_status pdssm_surrogate_bwd(const pdssm_dims *dims, const void *u, pdssm_dtype u_dtype,
+                                 const float *W_sel, const float *A, int64_t a_head_stride,
+                                 const int32_t *pi_dict, const int32_t *k, const void *d,
+                                 const void *b, pdssm_dtype in_dtype, const float *h0,
+                                 const float *lambda, int64_t chunk, const void *ws,
+                                 size_t ws_bytes, float inv_tau_s, float inv_tau_a,
+                                 void *scratch, size_t scratch_bytes, float *g_logits,
+                                 float *g_W, float *g_A, void *stream) {
+    pdssm_status st = check_surrogate_dims(dims, a_head_stride);
+    if (st != PDSSM_OK) return st;
+    if (check_dtype(u_dtype) != PDSSM_OK || check_dtype(in_dtype) != PDSSM_OK)
+        return PDSSM_ERR_INVALID_ARG;
+    if (chunk < 1) return arg_fail(PDSSM_ERR_INVALID_ARG, "chunk must be >= 1");
+    if (!(inv_tau_s > 0.f) || !(inv_tau_a > 0.f) || inv_tau_s > 3.0e38f || inv_tau_a > 3.0e38f)
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "inverse temperatures must be positive and finite");
+    if (!W_sel || !A || !pi_dict || !g_W || !g_A || !ws || !scratch)
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL pointer");
+    if (dims->L > 0 && (!u || !k || !d || !b || !lambda || !g_logits))
+        return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL tensor pointer");
+    const int64_t pi_hs = a_head_stride ? dims->K * dims->N : 0;
+    const WsLayout w = ws_layout(*dims, pi_hs, chunk, false);
+    if (ws_bytes < w.total) return arg_fail(PDSSM_ERR_WORKSPACE, "forward workspace too small");
+    if (scratch_bytes < surrogate_scratch_bytes(*dims, a_head_stride))
+        return arg_fail(PDSSM_ERR_WORKSPACE, "surrogate scratch too small");
+    if (!aligned(scratch, 256)) return arg_fail(PDSSM_ERR_INVALID_ARG, "scratch not 256-byte aligned");
+    const float *Hc = reinterpret_cast<const float *>(reinterpret_cast<const unsigned char *>(ws) + w.Hc);
+    cudaError_t e = launch_surrogate(*dims, u, u_dtype, W_sel, A, a_head_stride, pi_dict, k, d, b,
+                                     in_dtype, h0, Hc, chunk, lambda, inv_tau_s, inv_tau_a,
+                                     scratch, g_logits, g_W, g_A, (cudaStream_t)stream);
+    return e == cudaSuccess ? PDSSM_OK : cuda_fail(e, "surrogate backward");
+}
+
 pdssm_status pdssm_wait_selftest(int which, int64_t cap_ns, void *ws, size_t ws_bytes,
                                  void *stream) {
     if (which != 0 && which != 1) return arg_fail(PDSSM_ERR_INVALID_ARG, "which must be 0 or 1");

@@ -1034,6 +1034,21 @@ cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
 cudaError_t launch_scan_fused(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
 bool fused_path(const ChunkParams &p);
 cudaError_t launch_wait_selftest(const ChunkParams &p, int which, cudaStream_t st);
+cudaError_t launch_dict_hardmax(int64_t n_mats, int N, const float *A, int32_t *pi,
+                                cudaStream_t st);
+cudaError_t launch_soft_maps(const pdssm_dims &dm, const void *u, pdssm_dtype ut,
+                             const float *W, const float *A, int64_t a_hs, float inv_tau,
+                             int32_t *maps, cudaStream_t st);
+size_t surrogate_scratch_bytes(const pdssm_dims &dm, int64_t a_hs);
+cudaError_t launch_surrogate(const pdssm_dims &dm, const void *u, pdssm_dtype ut, const float *W,
+                             const float *A, int64_t a_hs, const int32_t *pi, const int32_t *k,
+                             const void *d, const void *b, pdssm_dtype dt, const float *h0,
+                             const float *Hc, int64_t chunk, const float *lam, float inv_tau_s,
+                             float inv_tau_a, void *scratch, float *g_l, float *g_W, float *g_A,
+                             cudaStream_t st);
+cudaError_t launch_scan_maps(const pdssm_dims &dm, const int32_t *maps, const void *d,
+                             const void *b, const void *c, pdssm_dtype dt, const float *h0,
+                             float *y, float *h_last, cudaStream_t st);
 cudaError_t launch_bwdA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
 cudaError_t launch_bwdC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
 cudaError_t launch_phaseB(const ChunkParams &p, cudaStream_t st);
