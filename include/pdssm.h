@@ -216,6 +216,30 @@ pdssm_status pdssm_scan_fwd_traced(const pdssm_dims *dims,
                                    int64_t chunk, void *ws, size_t ws_bytes,
                                    void *stream, pdssm_trace *trace);
 
+/*
+ * Hard selection inside the forward scan (Flash PD-SSM technical summary,
+ * Methodology §1 and §4: the selection of step t is the argmax of K linear
+ * scores of u_t): the results of pdssm_select followed by pdssm_scan_fwd,
+ * in one single-pass kernel whose CTAs select their own chunk's steps, so
+ * the indices never travel through device memory (k_out, when not NULL,
+ * receives a copy for a later backward).  The selection follows the
+ * contract of pdssm_select bit for bit: logits of a warp-level bf16 tensor-
+ * core product against W_sel's hi / lo bf16 parts, a certified argmax, and
+ * the exact fp32 fma chains for near ties.  Needs bf16 u, D_in a multiple of
+ * 16 (<= 256), K <= 16, N = 32 or 64 with 16-byte aligned rows, chunk <=
+ * 1024 and L >= 1; otherwise PDSSM_ERR_UNSUPPORTED (use the two calls).
+ * Other arguments as pdssm_scan_fwd (dims->D_in is u's width).
+ */
+pdssm_status pdssm_select_scan_fwd(const pdssm_dims *dims, const void *u,
+                                   pdssm_dtype u_dtype, const float *W_sel,
+                                   const int32_t *pi_dict,
+                                   int64_t pi_head_stride, const void *d,
+                                   const void *b, const void *c,
+                                   pdssm_dtype in_dtype, const float *h0,
+                                   float *y, float *h_last, int32_t *k_out,
+                                   int64_t chunk, void *ws, size_t ws_bytes,
+                                   void *stream);
+
 /* pdssm_scan_bwd, recording `trace` (see above).  Same results. */
 pdssm_status pdssm_scan_bwd_traced(const pdssm_dims *dims,
                                    const int32_t *pi_dict,

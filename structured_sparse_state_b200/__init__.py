@@ -39,7 +39,7 @@ EXPORTS = ("pdssm_status_str", "pdssm_last_error", "pdssm_version",
            "pdssm_scan_fwd_traced", "pdssm_scan_bwd_traced", "pdssm_ws_transfers",
            "pdssm_wait_selftest", "pdssm_wait_selftest_ws_bytes", "pdssm_dict_hardmax",
            "pdssm_soft_maps", "pdssm_scan_fwd_maps", "pdssm_surrogate_scratch_bytes",
-           "pdssm_surrogate_bwd")
+           "pdssm_surrogate_bwd", "pdssm_select_scan_fwd")
 
 TRACE_MAX_KERNELS = 8
 
@@ -94,6 +94,8 @@ def _load() -> ctypes.CDLL:
         "pdssm_soft_maps": (I32, [D, P, I32, P, P, I64, ctypes.c_float, P, P]),
         "pdssm_scan_fwd_maps": (I32, [D, P, P, P, P, I32, P, P, P, P]),
         "pdssm_surrogate_scratch_bytes": (SZ, [D, I64]),
+        "pdssm_select_scan_fwd": (I32, [D, P, I32, P, P, I64, P, P, P, I32, P, P, P, P, I64, P,
+                                        SZ, P]),
         "pdssm_surrogate_bwd": (I32, [D, P, I32, P, P, I64, P, P, P, P, I32, P, P, I64, P, SZ,
                                       ctypes.c_float, ctypes.c_float, P, SZ, P, P, P, P]),
         "pdssm_scan_fwd_traced": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, I64, P, SZ, P,
@@ -302,6 +304,42 @@ def pdssm_scan_fwd_noalloc(pi_dict, k, d, b, c, h0=None, chunk=128, y=None, h_la
                                        _ptr(y), _ptr(h_last), int(chunk), _stream(stream)),
            "pdssm_scan_fwd_noalloc")
     return y, h_last
+
+
+def pdssm_select_scan_fwd(u, W_sel, pi_dict, d, b, c, h0=None, chunk=128, ws=None, y=None,
+                          h_last=None, k_out=None, stream=None):
+    """Selection inside the single-pass forward (indices stay in shared
+    memory; k_out, if given, receives a copy).  Returns (y, h_last, ws)."""
+    _cuda(u, "u", (torch.bfloat16, torch.float32))
+    _cuda(W_sel, "W_sel", (torch.float32,))
+    _cuda(d, "d", (torch.float32, torch.bfloat16))
+    B, H, L, N = d.shape
+    Bu, Lu, D = u.shape
+    H2, K, D2 = W_sel.shape
+    if (Bu, Lu, H2, D2) != (B, L, H, D):
+        raise ValueError("u [B, L, D_in] and W_sel [H, K, D_in] disagree with d")
+    for name, t in (("b", b), ("c", c)):
+        _cuda(t, name, (d.dtype,))
+    _cuda(pi_dict, "pi_dict", (torch.int32,))
+    stride = _dict_stride(pi_dict, H, K, N)
+    dev = d.device
+    if ws is None:
+        ws = make_workspace(B, H, L, N, K, chunk, dev, stride != 0, False)
+    if y is None:
+        y = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    if h_last is None:
+        h_last = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    if k_out is not None:
+        _cuda(k_out, "k_out", (torch.int32,))
+    if h0 is not None:
+        _cuda(h0, "h0", (torch.float32,))
+    dm = dims(B, H, L, N, K, D)
+    _check(_lib.pdssm_select_scan_fwd(ctypes.byref(dm), _ptr(u), _dtype_code(u), _ptr(W_sel),
+                                      _ptr(pi_dict), stride, _ptr(d), _ptr(b), _ptr(c),
+                                      _dtype_code(d), _ptr(h0), _ptr(y), _ptr(h_last),
+                                      _ptr(k_out), int(chunk), _ptr(ws), ws.numel(),
+                                      _stream(stream)), "pdssm_select_scan_fwd")
+    return y, h_last, ws
 
 
 def pdssm_noalloc_scratch_bytes() -> int:

@@ -180,12 +180,13 @@ pdssm_status pdssm_select_tc_logits(const pdssm_dims *dims, const void *u, const
 static pdssm_status fwd_common(const pdssm_dims *dims, const int32_t *pi_dict,
                                int64_t pi_head_stride, const int32_t *k, const void *d,
                                const void *b, pdssm_dtype in_dtype, int64_t chunk, void *ws,
-                               size_t ws_bytes, bool for_bwd, WsLayout *wout) {
+                               size_t ws_bytes, bool for_bwd, WsLayout *wout,
+                               bool k_given = true) {
     pdssm_status st = check_scan_dims(dims, pi_head_stride, chunk);
     if (st != PDSSM_OK) return st;
     if (check_dtype(in_dtype) != PDSSM_OK) return PDSSM_ERR_INVALID_ARG;
     if (!pi_dict || !ws) return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL dictionary or workspace");
-    if (dims->L > 0 && (!k || !d || !b))
+    if (dims->L > 0 && ((k_given && !k) || !d || !b))
         return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL tensor pointer");
     if (!aligned(ws, 256)) return arg_fail(PDSSM_ERR_INVALID_ARG, "ws not 256-byte aligned");
     const WsLayout w = ws_layout(*dims, pi_head_stride, chunk, for_bwd);
@@ -274,7 +275,7 @@ pdssm_status scan_fwd_impl(const pdssm_dims *dims, const int32_t *pi_dict, int64
     p.h_last = h_last;
     if (fused_path(p)) {
         if ((e = tr.mark("single pass")) != cudaSuccess) return cuda_fail(e, "trace event");
-        e = launch_scan_fused(p, in_dtype, s);
+        e = launch_scan_fused(p, in_dtype, s, false);
         if (e != cudaSuccess) return cuda_fail(e, "single-pass forward");
         e = tr.finish();
         return e == cudaSuccess ? PDSSM_OK : cuda_fail(e, "trace event");
@@ -365,6 +366,40 @@ pdssm_status pdssm_scan_fwd_traced(const pdssm_dims *dims, const int32_t *pi_dic
     if (!trace) return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL trace");
     return scan_fwd_impl(dims, pi_dict, pi_head_stride, k, d, b, c, in_dtype, h0, y, h_last,
                          chunk, ws, ws_bytes, stream, trace);
+}
+
+pdssm_status pdssm_select_scan_fwd(const pdssm_dims *dims, const void *u, pdssm_dtype u_dtype,
+                                   const float *W_sel, const int32_t *pi_dict,
+                                   int64_t pi_head_stride, const void *d, const void *b,
+                                   const void *c, pdssm_dtype in_dtype, const float *h0, float *y,
+                                   float *h_last, int32_t *k_out, int64_t chunk, void *ws,
+                                   size_t ws_bytes, void *stream) {
+    if (!dims) return arg_fail(PDSSM_ERR_INVALID_ARG, "dims is NULL");
+    if (dims->L < 1) return arg_fail(PDSSM_ERR_INVALID_ARG, "need L >= 1");
+    if (!u || !W_sel) return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL u or W_sel");
+    WsLayout w;
+    pdssm_status st = fwd_common(dims, pi_dict, pi_head_stride, nullptr, d, b, in_dtype, chunk,
+                                 ws, ws_bytes, false, &w, false);
+    if (st != PDSSM_OK) return st;
+    if (!c || !y) return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL c or y");
+    ChunkParams p = make_params(dims, w, ws, chunk, nullptr, d, b, c, in_dtype);
+    p.u = u;
+    p.W_sel = W_sel;
+    p.D_in = (int)dims->D_in;
+    p.k_out = k_out;
+    if (u_dtype != PDSSM_BF16 || !fused_select_ok(p, u, W_sel))
+        return arg_fail(PDSSM_ERR_UNSUPPORTED,
+                        "the selection runs inside the forward for bf16 u, D_in a multiple of 16 "
+                        "(<= 256), K <= 16, N = 32 or 64 with 16-byte aligned rows and chunk <= "
+                        "1024; use pdssm_select and pdssm_scan_fwd otherwise");
+    cudaStream_t s = (cudaStream_t)stream;
+    st = run_prep(dims, pi_dict, pi_head_stride, w, ws, s);
+    if (st != PDSSM_OK) return st;
+    p.h0 = h0;
+    p.y = y;
+    p.h_last = h_last;
+    cudaError_t e = launch_scan_fused(p, in_dtype, s, true);
+    return e == cudaSuccess ? PDSSM_OK : cuda_fail(e, "selection + single-pass forward");
 }
 
 pdssm_status pdssm_scan_bwd(const pdssm_dims *dims, const int32_t *pi_dict,

@@ -104,6 +104,11 @@ struct ChunkParams {
     int *look;                // single-pass forward: per-chunk flags (0, kFlagAgg, kFlagIncl)
     unsigned long long *ticket;   // single-pass forward: next chunk ticket
     uint64_t wait_ns;         // cap of every bounded wait, in ns of the global timer
+    // selection inside the single-pass forward (k never leaves the CTA)
+    const void *u;            // bf16 [B][L][D_in]
+    const float *W_sel;       // [H][K][D_in]
+    int D_in;
+    int32_t *k_out;           // optional copy of the selection [B][H][L]
     int ns;                   // pipeline stages
     int wpc;                  // warps (units) per CTA
     int bulk;                 // 1: bulk-copy staging; 0: cooperative copies
@@ -1031,8 +1036,9 @@ cudaError_t launch_phaseA(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st)
 bool fast_path(const ChunkParams &p);
 cudaError_t launch_phaseA_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
 cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
-cudaError_t launch_scan_fused(ChunkParams p, pdssm_dtype dt, cudaStream_t st);
+cudaError_t launch_scan_fused(ChunkParams p, pdssm_dtype dt, cudaStream_t st, bool select);
 bool fused_path(const ChunkParams &p);
+bool fused_select_ok(const ChunkParams &p, const void *u, const float *W);
 cudaError_t launch_wait_selftest(const ChunkParams &p, int which, cudaStream_t st);
 cudaError_t launch_dict_hardmax(int64_t n_mats, int N, const float *A, int32_t *pi,
                                 cudaStream_t st);

@@ -33,7 +33,8 @@ struct SegTransfer {
 template <typename T, int NPL, int LV>
 __device__ __forceinline__ bool phaseA_segment(const ChunkParams &p, const SmemDict &sd,
                                                unsigned char *wbase, int64_t row0, int len,
-                                               int lane, SegTransfer<NPL> &out) {
+                                               int lane, SegTransfer<NPL> &out,
+                                               const int32_t *ks = nullptr) {
     constexpr int N = 32 * NPL;
     constexpr int ROWB = N * (int)sizeof(T);
     constexpr int TENS = kTS * ROWB;
@@ -73,9 +74,13 @@ __device__ __forceinline__ bool phaseA_segment(const ChunkParams &p, const SmemD
         Dl[r] = 1.f;
         posb[r] = (lane * NPL + r) * ES;
     }
-    const int32_t *kp = p.k + row0;
+    // selection indices: from global memory, or (ks) from this CTA's shared memory
+    const int32_t *kp = ks ? ks : p.k + row0;
+    auto kload = [&](int idx, bool valid) {
+        return valid ? (ks ? kp[idx] : __ldg(kp + idx)) : 0;
+    };
     float *yp = with_y ? p.y + row0 : nullptr;
-    int kreg = load_k(kp, lane, lane < kTS && lane < len, K, p.status);
+    int kreg = clamp_k(kload(lane, lane < kTS && lane < len), K, p.status);
 
     for (int i = 0; i < ntiles; ++i) {
         if (!ring.wait(i)) {
@@ -84,7 +89,7 @@ __device__ __forceinline__ bool phaseA_segment(const ChunkParams &p, const SmemD
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
-        const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
+        const int knext = kload(t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
         const uint32_t row0s = ring.tile(i);
         // values of step q that do not depend on the state, loaded one step
         // ahead so their latency overlaps the previous step's work
@@ -233,7 +238,8 @@ template <typename T, int NPL, int NT, int CQ>
 __device__ __forceinline__ bool phaseC_segment(const ChunkParams &p, const SmemDict &sd,
                                                uint32_t ring_s, uint32_t bar0, float *ybuf,
                                                int64_t row0, int len, float (&w)[NPL],
-                                               int tbase, int lane) {
+                                               int tbase, int lane,
+                                               const int32_t *ks = nullptr) {
     constexpr int N = 32 * NPL;
     constexpr int ROWB = N * (int)sizeof(T);
     constexpr int TENS = kTS * ROWB;
@@ -258,9 +264,12 @@ __device__ __forceinline__ bool phaseC_segment(const ChunkParams &p, const SmemD
     int posb[NPL];   // column positions as byte offsets into a staged row
 #pragma unroll
     for (int r = 0; r < NPL; ++r) posb[r] = (lane * NPL + r) * ES;
-    const int32_t *kp = p.k + row0;
+    const int32_t *kp = ks ? ks : p.k + row0;
+    auto kload = [&](int idx, bool valid) {
+        return valid ? (ks ? kp[idx] : __ldg(kp + idx)) : 0;
+    };
     float *yp = p.y + row0;
-    int kreg = load_k(kp, lane, lane < kTS && lane < len, K, p.status);
+    int kreg = clamp_k(kload(lane, lane < kTS && lane < len), K, p.status);
 
     for (int i = 0; i < ntiles; ++i) {
         if (!ring.wait(tbase + i)) {
@@ -271,7 +280,7 @@ __device__ __forceinline__ bool phaseC_segment(const ChunkParams &p, const SmemD
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
-        const int knext = load_k_raw(kp, t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
+        const int knext = kload(t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
         const float yold = ((lane & 3) == 0 && (lane >> 2) < n) ? yp[t0 + (lane >> 2)] : 0.f;
         const uint32_t row0s = ring.tile(tbase + i);
         if (n == kTS) {
@@ -462,6 +471,135 @@ __device__ __noinline__ bool lookback_carry(const ChunkParams &p, int64_t bh, in
     return true;
 }
 
+// ---------------------------------------------------------------------------
+// Hard selection inside the single-pass forward (k stays in shared memory).
+// The logits of 16 rows x 16 maps per warp-level bf16 tensor-core product
+// (mma m16n8k16, fp32 accumulation) against W split into W_hi = bf16(W) and
+// W_lo = bf16(W - W_hi), so every product is exact and |W - W_hi - W_lo| <=
+// 2^-16 |W|.  The argmax is certified as in the standalone tensor-core
+// selection: with S = ||u_row|| max_k ||W_hk|| (rounded up), the product
+// logit lies within (D 2^-21 + 2^-16) S of the exact sum and the contract's
+// fp32 fma chain within D 2^-24 S, so the contract's first argmax is among
+// the logits within twice their sum of the top one; a single candidate is
+// the answer, several are decided by their exact fp32 fma chains.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Sum of squares of the two bf16 values packed in w, added to s.
+__device__ __forceinline__ float sq2(uint32_t w, float s) {
+    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xffff0000u);
+    return fmaf(hi, hi, fmaf(lo, lo, s));
+}
+
+// The contract's fp32 fma chains of the candidate maps of one row (first
+// maximum in ascending k).
+__device__ __noinline__ int resolve_row(const ChunkParams &p, int64_t h, int64_t urow,
+                                        unsigned cand) {
+    const int D = p.D_in;
+    const __nv_bfloat16 *ur = reinterpret_cast<const __nv_bfloat16 *>(p.u) + urow * D;
+    float bv = 0.f;
+    int best = -1;
+    while (cand) {
+        const int kk = __ffs(cand) - 1;
+        cand &= cand - 1;
+        const float *wr = p.W_sel + (h * p.K + kk) * D;
+        float acc = 0.f;
+        for (int q = 0; q < D; ++q) acc = __fmaf_rn(__ldg(wr + q), __bfloat162float(ur[q]), acc);
+        if (best < 0 || acc > bv) {
+            bv = acc;
+            best = kk;
+        }
+    }
+    return best;
+}
+
+// Selection of rows [0, n) starting at u row urow0 (b * L + t0) for head h:
+// writes k of each row into ks[row].  Whi / Wlo: [16][D/2] packed bf16
+// pairs of this head's W (rows >= K zero); Wn = max_k ||W_hk|| rounded up.
+__device__ void select_rows_mma(const ChunkParams &p, const uint32_t *Whi, const uint32_t *Wlo,
+                                float Wn, int64_t h, int64_t urow0, int n, int32_t *ks, int lane) {
+    const int D = p.D_in, K = (int)p.K, D2 = D / 2;
+    const int g = lane >> 2, q = lane & 3;
+    const float ceps = 1.01f * ((float)D * 4.76837158203125e-07f + 1.52587890625e-05f +
+                                (float)D * 5.9604644775390625e-08f);
+    const int ntl = K > 8 ? 2 : 1;
+    for (int m0 = 0; m0 < n; m0 += 16) {
+        const bool v0 = m0 + g < n, v1 = m0 + g + 8 < n;
+        const uint32_t *u0 = reinterpret_cast<const uint32_t *>(
+            reinterpret_cast<const __nv_bfloat16 *>(p.u) + (urow0 + m0 + g) * D);
+        const uint32_t *u1 = u0 + 4 * D;   // row g + 8 (8 rows of D bf16 = 4 D words)
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        float s0 = 0.f, s1 = 0.f;
+        for (int kb = 0; kb < D2; kb += 8) {
+            const uint32_t a0 = v0 ? __ldg(u0 + kb + q) : 0u;
+            const uint32_t a1 = v1 ? __ldg(u1 + kb + q) : 0u;
+            const uint32_t a2 = v0 ? __ldg(u0 + kb + q + 4) : 0u;
+            const uint32_t a3 = v1 ? __ldg(u1 + kb + q + 4) : 0u;
+            s0 = sq2(a2, sq2(a0, s0));
+            s1 = sq2(a3, sq2(a1, s1));
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+                if (nt >= ntl) break;
+                const int wrow = (nt * 8 + g) * D2 + kb + q;
+                mma_bf16_16816(acc[nt], a0, a1, a2, a3, Whi[wrow], Whi[wrow + 4]);
+                mma_bf16_16816(acc[nt], a0, a1, a2, a3, Wlo[wrow], Wlo[wrow + 4]);
+            }
+        }
+        // row norms: the four lanes of a quad share rows g and g + 8
+        s0 += __shfl_xor_sync(kFull, s0, 1);
+        s0 += __shfl_xor_sync(kFull, s0, 2);
+        s1 += __shfl_xor_sync(kFull, s1, 1);
+        s1 += __shfl_xor_sync(kFull, s1, 2);
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+            // this lane's logits of the row: maps nt * 8 + 2 q + {0, 1}
+            float lg[4];
+            int kk[4];
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    kk[nt * 2 + e] = nt * 8 + 2 * q + e;
+                    lg[nt * 2 + e] = acc[nt][half * 2 + e];
+                }
+            float b1 = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (kk[e] < K) b1 = fmaxf(b1, lg[e]);
+            b1 = fmaxf(b1, __shfl_xor_sync(kFull, b1, 1));
+            b1 = fmaxf(b1, __shfl_xor_sync(kFull, b1, 2));
+            const float unorm = __fmul_ru(__fsqrt_ru(half ? s1 : s0), 1.0009765625f);
+            const float thr = b1 - 2.0f * __fmul_ru(__fmul_ru(unorm, Wn), ceps);
+            unsigned cand = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                if (kk[e] < K && lg[e] >= thr) cand |= 1u << kk[e];
+            cand |= __shfl_xor_sync(kFull, cand, 1);
+            cand |= __shfl_xor_sync(kFull, cand, 2);
+            const int row = m0 + g + 8 * half;
+            if (q == 0 && row < n) {
+                int kv;
+                if (__popc(cand) == 1) {
+                    kv = __ffs(cand) - 1;
+                } else {
+                    // near tie, or no finite logit: the exact chains decide
+                    if (cand == 0) cand = (1u << K) - 1u;
+                    kv = resolve_row(p, h, urow0 + row, cand);
+                }
+                ks[row] = kv;
+            }
+        }
+    }
+}
+
 // Per-warp scratch of steps 2-4, inside the warp's staging ring (idle
 // between phase A and phase C): scan buffers [2][64] of P, D and V, the
 // scatter scratch, and one vector for the layout change of the carry.
@@ -473,7 +611,7 @@ struct FusedScratch {
     float xs[64];
 };
 
-template <typename T, int NPL>
+template <typename T, int NPL, bool SEL>
 __global__ void __launch_bounds__(kFusedWarps * 32, 3) k_scan_fused(const ChunkParams p) {
     extern __shared__ __align__(128) unsigned char sm_f_raw[];
     unsigned char *sm = smem_base256(sm_f_raw);
@@ -500,23 +638,75 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 3) k_scan_fused(const ChunkP
     const SmemDict sd = dict_view(p, dict_s);
     const bool perm = __ldg(p.dict_stats + 1) <= 1;   // every map a permutation
 
-    // 1. phase A of this warp's sub-chunk
     const int64_t s0 = cidx * p.chunk;
     const int len = (int)imin64(p.chunk, p.L - s0);
     const int S = (len + kFusedWarps - 1) / kFusedWarps;
     const int ws0 = min(warp * S, len);
     const int wlen = min(S, len - ws0);
     const int64_t row0 = bh * p.L + s0 + ws0;
-    unsigned char *wbase =
-        dict_s + dict_slot_bytes((int)p.K, (int)p.N, p.dict_content) + (size_t)warp * p.smem_per_warp;
+    unsigned char *wregions = dict_s + dict_slot_bytes((int)p.K, (int)p.N, p.dict_content);
+    unsigned char *wbase = wregions + (size_t)warp * p.smem_per_warp;
+    const int32_t *ks = nullptr;
+
+    // 0. (SEL) the selection of this warp's sub-chunk, into shared memory
+    if constexpr (SEL) {
+        const int Smax = (int)((p.chunk + kFusedWarps - 1) / kFusedWarps);
+        int32_t *ksw = reinterpret_cast<int32_t *>(wregions + (size_t)kFusedWarps * p.smem_per_warp) +
+                       warp * Smax;
+        const int D = p.D_in, D2 = D / 2;
+        const int64_t hh = bh % p.H, bb = bh / p.H;
+        // W of this head split into bf16 hi / lo parts (rows >= K zero), in
+        // the warp regions (idle until phase A), and max_k ||W_hk|| rounded up
+        uint32_t *Whi = reinterpret_cast<uint32_t *>(wregions);
+        uint32_t *Wlo = Whi + 16 * D2;
+        int *wn_bits = reinterpret_cast<int *>(sm + 8);
+        if (threadIdx.x == 0) *wn_bits = 0;
+        __syncthreads();
+        for (int rr = warp; rr < 16; rr += kFusedWarps) {
+            float ss = 0.f;
+            for (int d2 = lane; d2 < D2; d2 += 32) {
+                float w0 = 0.f, w1 = 0.f;
+                if (rr < (int)p.K) {
+                    const float2 wv = *reinterpret_cast<const float2 *>(
+                        p.W_sel + (hh * p.K + rr) * D + 2 * d2);
+                    w0 = wv.x;
+                    w1 = wv.y;
+                }
+                const __nv_bfloat16 h0b = __float2bfloat16_rn(w0), h1b = __float2bfloat16_rn(w1);
+                const __nv_bfloat16 l0b = __float2bfloat16_rn(w0 - __bfloat162float(h0b));
+                const __nv_bfloat16 l1b = __float2bfloat16_rn(w1 - __bfloat162float(h1b));
+                Whi[rr * D2 + d2] = (uint32_t)__bfloat16_as_ushort(h0b) |
+                                    ((uint32_t)__bfloat16_as_ushort(h1b) << 16);
+                Wlo[rr * D2 + d2] = (uint32_t)__bfloat16_as_ushort(l0b) |
+                                    ((uint32_t)__bfloat16_as_ushort(l1b) << 16);
+                ss = __fmaf_ru(w0, w0, ss);
+                ss = __fmaf_ru(w1, w1, ss);
+            }
+#pragma unroll
+            for (int o = 16; o; o >>= 1) ss = __fadd_ru(ss, __shfl_xor_sync(kFull, ss, o));
+            if (lane == 0) atomicMax(wn_bits, __float_as_int(ss));   // non-negative: bits order
+        }
+        __syncthreads();
+        const float Wn = __fmul_ru(__fsqrt_ru(__int_as_float(*wn_bits)), 1.0009765625f);
+        select_rows_mma(p, Whi, Wlo, Wn, hh, bb * p.L + s0 + ws0, wlen, ksw, lane);
+        __syncwarp();
+        if (p.k_out)
+            for (int i = lane; i < wlen; i += 32) p.k_out[row0 + i] = ksw[i];
+        ks = ksw;
+        // every warp is done with W before phase A's copies land in the regions
+        fence_proxy_async_shared();
+        __syncthreads();
+    }
+
+    // 1. phase A of this warp's sub-chunk
     SegTransfer<NPL> tr;
     bool ok;
     switch (step_variant(p.dict_stats)) {
-        case 0: ok = phaseA_segment<T, NPL, 0>(p, sd, wbase, row0, wlen, lane, tr); break;
-        case 1: ok = phaseA_segment<T, NPL, 1>(p, sd, wbase, row0, wlen, lane, tr); break;
-        case 2: ok = phaseA_segment<T, NPL, 2>(p, sd, wbase, row0, wlen, lane, tr); break;
-        case 3: ok = phaseA_segment<T, NPL, 3>(p, sd, wbase, row0, wlen, lane, tr); break;
-        default: ok = phaseA_segment<T, NPL, 5>(p, sd, wbase, row0, wlen, lane, tr); break;
+        case 0: ok = phaseA_segment<T, NPL, 0>(p, sd, wbase, row0, wlen, lane, tr, ks); break;
+        case 1: ok = phaseA_segment<T, NPL, 1>(p, sd, wbase, row0, wlen, lane, tr, ks); break;
+        case 2: ok = phaseA_segment<T, NPL, 2>(p, sd, wbase, row0, wlen, lane, tr, ks); break;
+        case 3: ok = phaseA_segment<T, NPL, 3>(p, sd, wbase, row0, wlen, lane, tr, ks); break;
+        default: ok = phaseA_segment<T, NPL, 5>(p, sd, wbase, row0, wlen, lane, tr, ks); break;
     }
     const int ntA = (wlen + kTS - 1) / kTS;
     FusedScratch &fs = *reinterpret_cast<FusedScratch *>(wbase);
@@ -658,7 +848,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 3) k_scan_fused(const ChunkP
     if (ok && wlen > 0 && !(cidx == 0 && warp == 0 && p.h0 == nullptr)) {
         float *ybuf = reinterpret_cast<float *>(wbase + kFastStages * RingT::STAGEB) + 2 * kPbStride;
         phaseC_segment<T, NPL, 3, 2>(p, sd, smem_u32(wbase), smem_u32(ybuf + kYbufFloats), ybuf,
-                                     row0, wlen, w, ntA, lane);
+                                     row0, wlen, w, ntA, lane, ks);
     }
 }
 
@@ -715,23 +905,45 @@ cudaError_t launch_wait_selftest(const ChunkParams &p, int which, cudaStream_t s
 // the grid must fit the launch limit).
 bool fused_path(const ChunkParams &p) { return fast_path(p) && p.units <= 0x7fffffff; }
 
-// The single-pass forward: one CTA of kFusedWarps warps per chunk.
-cudaError_t launch_scan_fused(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
+// The selection runs inside the single-pass forward for bf16 u with D_in a
+// multiple of 16 (at most 256), K <= 16, and chunks of at most 1024 steps
+// (their indices stay in shared memory).
+bool fused_select_ok(const ChunkParams &p, const void *u, const float *W) {
+    return fused_path(p) && p.D_in % 16 == 0 && p.D_in >= 16 && p.D_in <= 256 && p.K <= 16 &&
+           p.chunk <= 1024 && ((uintptr_t)u % 16) == 0 && ((uintptr_t)W % 16) == 0;
+}
+
+// The single-pass forward: one CTA of kFusedWarps warps per chunk; with
+// `select`, the CTA also takes its chunk's selection (p.u, p.W_sel).
+cudaError_t launch_scan_fused(ChunkParams p, pdssm_dtype dt, cudaStream_t st, bool select) {
     const int es = dt == PDSSM_BF16 ? 2 : 4;
     p.dict_content = (dt == PDSSM_BF16 ? kDictMap16 : kDictMap) | kDictSeg;
     p.smem_per_warp = warp_smem_bytes(kFastStages, 3, (int)p.N * es);
     p.wpc = kFusedWarps;
-    const size_t smem = 512 + (size_t)dict_slot_bytes((int)p.K, (int)p.N, p.dict_content) +
-                        (size_t)kFusedWarps * p.smem_per_warp + 256;
+    size_t smem = 512 + (size_t)dict_slot_bytes((int)p.K, (int)p.N, p.dict_content) +
+                  (size_t)kFusedWarps * p.smem_per_warp + 256;
+    if (select) {
+        // the sub-chunks' indices after the warp regions; W's hi / lo parts
+        // (64 D_in bytes) fit inside the regions
+        smem += (size_t)kFusedWarps * ((p.chunk + kFusedWarps - 1) / kFusedWarps) * 4;
+        if ((size_t)64 * p.D_in > (size_t)kFusedWarps * p.smem_per_warp) return cudaErrorInvalidValue;
+    }
     auto go = [&](auto kern) {
         cudaError_t e =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
         return launch_pdl(kern, dim3((unsigned)p.units), dim3(kFusedWarps * 32), smem, st, p);
     };
+    if (select) {
+        if (dt == PDSSM_BF16)
+            return p.N == 64 ? go(k_scan_fused<__nv_bfloat16, 2, true>)
+                             : go(k_scan_fused<__nv_bfloat16, 1, true>);
+        return p.N == 64 ? go(k_scan_fused<float, 2, true>) : go(k_scan_fused<float, 1, true>);
+    }
     if (dt == PDSSM_BF16)
-        return p.N == 64 ? go(k_scan_fused<__nv_bfloat16, 2>) : go(k_scan_fused<__nv_bfloat16, 1>);
-    return p.N == 64 ? go(k_scan_fused<float, 2>) : go(k_scan_fused<float, 1>);
+        return p.N == 64 ? go(k_scan_fused<__nv_bfloat16, 2, false>)
+                         : go(k_scan_fused<__nv_bfloat16, 1, false>);
+    return p.N == 64 ? go(k_scan_fused<float, 2, false>) : go(k_scan_fused<float, 1, false>);
 }
 
 cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
