@@ -301,12 +301,127 @@ def run_ours(args, cfg):
             keep = ("value", "unit", "ms_per_step", "steps", "warmup", "dtype", "config",
                     "roofline", "phases_ms", "clocks", "gpu_launches", "cpu_baseline")
             out["extra"][xcfg["name"]] = {k: x[k] for k in keep if k in x}
+        torch.cuda.empty_cache()
+        out["extra"]["comparisons"] = measure_comparisons(args, torch, pd, dev)
     if world > 1:
         dist.destroy_process_group()
     return out
 
 
 EXTRA_WORKLOADS = (3, 4)
+
+
+def _event_ms(torch, fn, reps, warm=2):
+    """Mean device time of fn() over reps calls (CUDA events on the current
+    stream, after warm-up)."""
+    for _ in range(warm):
+        fn()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    s.record()
+    for _ in range(reps):
+        fn()
+    e.record()
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / reps
+
+
+def measure_comparisons(args, torch, pd, dev):
+    """Timings of the paths around the headline one (device time, inputs
+    resident):
+      * the single-pass forward vs the three-kernel forward, and selection
+        inside the single-pass forward vs the two calls, on the full bf16
+        selection workload;
+      * the original PD-SSM's soft selection (per-step dense mixture and
+        column hardmax, then the per-step-map scan) vs the hard path, on the
+        same workload at B = 1 (context for the pages' figure that PD-SSM
+        ran about 40x slower than Mamba2; here both sides are this
+        library's kernels);
+      * the straight-through surrogate backward on the same workload at
+        B = 2, next to the hard forward + exact adjoint."""
+    out = {}
+    cfg = gen.workload(DEFAULT_WORKLOAD)
+    inp = gen.generate(cfg)
+    B, H, L, N, K = cfg["B"], cfg["H"], cfg["L"], cfg["N"], cfg["K"]
+    chunk = cfg["chunk"]
+
+    def bf(x):
+        return torch.from_numpy(np.ascontiguousarray(x)).to(torch.bfloat16).to(dev)
+
+    u, d, b, c = bf(inp.u), bf(inp.d), bf(inp.b), bf(inp.c)
+    W = torch.from_numpy(inp.W).to(dev)
+    pi = torch.from_numpy(inp.pi).to(dev)
+    k = torch.empty((B, H, L), dtype=torch.int32, device=dev)
+    y = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    hl = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    ws = pd.make_workspace(B, H, L, N, K, chunk, dev)
+    reps = max(5, args.steps // 10)
+    t_two = _event_ms(torch, lambda: (pd.pdssm_select(u, W, k_out=k),
+                                      pd.pdssm_scan_fwd(pi, k, d, b, c, None, chunk=chunk,
+                                                        ws=ws, y=y, h_last=hl)), reps)
+    t_fused = _event_ms(torch, lambda: pd.pdssm_select_scan_fwd(u, W, pi, d, b, c, None,
+                                                                chunk=chunk, ws=ws, y=y,
+                                                                h_last=hl), reps)
+    pd.pdssm_select(u, W, k_out=k)
+    t_3k = _event_ms(torch, lambda: pd.pdssm_scan_fwd(pi, k, d, b, c, None, chunk=chunk, ws=ws,
+                                                      y=y, h_last=hl), reps)
+    t_1k = _event_ms(torch, lambda: pd.pdssm_scan_fwd_single_pass(pi, k, d, b, c, None,
+                                                                  chunk=chunk, ws=ws, y=y,
+                                                                  h_last=hl), reps)
+    upd = updates(cfg)
+    out["single_pass_forward"] = {
+        "workload": cfg["name"], "three_kernels_ms": round(t_3k, 5),
+        "single_pass_ms": round(t_1k, 5)}
+    out["fused_selection"] = {
+        "workload": cfg["name"], "select_then_scan_ms": round(t_two, 5),
+        "select_inside_scan_ms": round(t_fused, 5),
+        "select_inside_scan_updates_per_s": upd / (t_fused * 1e-3)}
+    # soft selection vs hard selection at B = 1
+    rng = np.random.default_rng(7)
+    A = torch.from_numpy(rng.standard_normal((K, N, N)).astype(np.float32)).to(dev)
+    u1, d1, b1, c1 = u[:1].contiguous(), d[:1].contiguous(), b[:1].contiguous(), c[:1].contiguous()
+    k1 = k[:1].contiguous()
+    y1, hl1 = y[:1].contiguous(), hl[:1].contiguous()
+    ws1 = pd.make_workspace(1, H, L, N, K, chunk, dev)
+    pi_A = pd.pdssm_dict_hardmax(A)
+    maps = torch.empty((1, H, L, N), dtype=torch.int32, device=dev)
+    t_hard = _event_ms(torch, lambda: (pd.pdssm_select(u1, W, k_out=k1),
+                                       pd.pdssm_scan_fwd(pi_A, k1, d1, b1, c1, None,
+                                                         chunk=chunk, ws=ws1, y=y1,
+                                                         h_last=hl1)), reps)
+    t_maps = _event_ms(torch, lambda: pd.pdssm_soft_maps(u1, W, A, 1.0, maps_out=maps), 3, 1)
+    t_scan_maps = _event_ms(torch, lambda: pd.pdssm_scan_fwd_maps(maps, d1, b1, c1, None, y1,
+                                                                  hl1), 3, 1)
+    out["soft_selection_dense"] = {
+        "workload": cfg["name"] + " at B=1", "hard_select_scan_ms": round(t_hard, 5),
+        "soft_maps_ms": round(t_maps, 3), "per_step_map_scan_ms": round(t_scan_maps, 3),
+        "soft_over_hard": round((t_maps + t_scan_maps) / t_hard, 1)}
+    del maps, ws1
+    # surrogate backward at B = 2
+    B2 = 2
+    u2, d2, b2, c2 = (x[:B2].contiguous() for x in (u, d, b, c))
+    g_y = torch.randn((B2, H, L), device=dev)
+    k2 = torch.empty((B2, H, L), dtype=torch.int32, device=dev)
+    pd.pdssm_select(u2, W, k_out=k2)
+    ws2 = pd.make_workspace(B2, H, L, N, K, chunk, dev, False, True)
+    y2 = torch.empty((B2, H, L), dtype=torch.float32, device=dev)
+    hl2 = torch.empty((B2, H, N), dtype=torch.float32, device=dev)
+    gouts = tuple(torch.empty((B2, H, L, N), device=dev) for _ in range(3)) + (
+        torch.empty((B2, H, N), device=dev),)
+
+    def fwd_bwd():
+        pd.pdssm_scan_fwd(pi_A, k2, d2, b2, c2, None, chunk=chunk, ws=ws2, y=y2, h_last=hl2,
+                          for_bwd=True)
+        pd.pdssm_scan_bwd(pi_A, k2, d2, b2, c2, None, g_y, ws2, chunk=chunk, out=gouts)
+    t_fb = _event_ms(torch, fwd_bwd, reps)
+    t_sur = _event_ms(torch, lambda: pd.pdssm_surrogate_bwd(u2, W, A, pi_A, k2, d2, b2, None,
+                                                            gouts[0], ws2, chunk, 1.0, 1.0), 3, 1)
+    out["surrogate_bwd"] = {
+        "workload": cfg["name"] + " at B=2", "hard_fwd_plus_adjoint_ms": round(t_fb, 5),
+        "surrogate_ms": round(t_sur, 5),
+        "surrogate_updates_per_s": B2 * H * L * N / (t_sur * 1e-3)}
+    return out
 
 
 def measure(args, cfg, torch, pd, dev, world, rank, dist, K_steps, with_e2e, with_cpu,

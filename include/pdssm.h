@@ -151,11 +151,7 @@ pdssm_status pdssm_select_tc_logits(const pdssm_dims *dims, const void *u,
  * Chunked forward scan (Methodology §3).  Runs phase A0 (sanitised copy of
  * the dictionary), A (per chunk: local readout of the state started from zero,
  * closed PD transfer Pi_c, Delta_c, v_c), B (carry prefix scan H_c, h_last)
- * and C (carry correction of the readout y).  For N = 32 or 64 with 16-byte
- * aligned rows the three phases run as one kernel (one CTA per chunk, in
- * chunk order: phase A on sub-chunks, their transfers composed in the CTA,
- * the carry taken from the predecessors by decoupled look-back, then phase
- * C); other shapes run them as three kernels.  Writes y [B][H][L] and, when
+ * and C (carry correction of the readout y), as three kernels.  Writes y [B][H][L] and, when
  * non-NULL, h_last [B][H][N] = h_{L-1} (h0 when L = 0).  h0 may be NULL
  * (zero initial state).  ws must hold pdssm_workspace_bytes(dims,
  * pi_head_stride, chunk, 0) bytes, 256-byte aligned; its contents are
@@ -239,6 +235,30 @@ pdssm_status pdssm_select_scan_fwd(const pdssm_dims *dims, const void *u,
                                    float *y, float *h_last, int32_t *k_out,
                                    int64_t chunk, void *ws, size_t ws_bytes,
                                    void *stream);
+
+/*
+ * The forward scan as ONE kernel (Methodology §3 with the three phases
+ * fused): persistent CTAs take chunks in chunk order; a team of warps runs
+ * phase A on the chunk's sub-chunks, composes their transfers, publishes
+ * the chunk's transfer, takes its carry from the predecessors' published
+ * transfers and carries (decoupled look-back, every wait bounded), publishes
+ * its own carry, and runs phase C on data phase A read shortly before.
+ * Same arguments, results and workspace contents as pdssm_scan_fwd (so
+ * pdssm_scan_bwd may follow it); needs N = 32 or 64 with 16-byte aligned
+ * rows, else PDSSM_ERR_UNSUPPORTED.  It moves close to the algorithmic bytes
+ * (no phase C re-read from DRAM for most chunks) but, with thousands of
+ * chunks in flight over few sequences, spends more time on the look-back
+ * chain than the carry scan of the three-kernel form, which stays the
+ * default.
+ */
+pdssm_status pdssm_scan_fwd_single_pass(const pdssm_dims *dims,
+                                        const int32_t *pi_dict,
+                                        int64_t pi_head_stride,
+                                        const int32_t *k, const void *d,
+                                        const void *b, const void *c,
+                                        pdssm_dtype in_dtype, const float *h0,
+                                        float *y, float *h_last, int64_t chunk,
+                                        void *ws, size_t ws_bytes, void *stream);
 
 /* pdssm_scan_bwd, recording `trace` (see above).  Same results. */
 pdssm_status pdssm_scan_bwd_traced(const pdssm_dims *dims,

@@ -39,7 +39,7 @@ EXPORTS = ("pdssm_status_str", "pdssm_last_error", "pdssm_version",
            "pdssm_scan_fwd_traced", "pdssm_scan_bwd_traced", "pdssm_ws_transfers",
            "pdssm_wait_selftest", "pdssm_wait_selftest_ws_bytes", "pdssm_dict_hardmax",
            "pdssm_soft_maps", "pdssm_scan_fwd_maps", "pdssm_surrogate_scratch_bytes",
-           "pdssm_surrogate_bwd", "pdssm_select_scan_fwd")
+           "pdssm_surrogate_bwd", "pdssm_select_scan_fwd", "pdssm_scan_fwd_single_pass")
 
 TRACE_MAX_KERNELS = 8
 
@@ -94,6 +94,8 @@ def _load() -> ctypes.CDLL:
         "pdssm_soft_maps": (I32, [D, P, I32, P, P, I64, ctypes.c_float, P, P]),
         "pdssm_scan_fwd_maps": (I32, [D, P, P, P, P, I32, P, P, P, P]),
         "pdssm_surrogate_scratch_bytes": (SZ, [D, I64]),
+        "pdssm_scan_fwd_single_pass": (I32, [D, P, I64, P, P, P, P, I32, P, P, P, I64, P, SZ,
+                                             P]),
         "pdssm_select_scan_fwd": (I32, [D, P, I32, P, P, I64, P, P, P, I32, P, P, P, P, I64, P,
                                         SZ, P]),
         "pdssm_surrogate_bwd": (I32, [D, P, I32, P, P, I64, P, P, P, P, I32, P, P, I64, P, SZ,
@@ -281,6 +283,30 @@ def pdssm_scan_fwd(pi_dict, k, d, b, c, h0=None, chunk=128, ws=None, y=None, h_l
                                _ptr(b), _ptr(c), _dtype_code(d), _ptr(h0), _ptr(y),
                                _ptr(h_last), int(chunk), _ptr(ws), ws.numel(),
                                _stream(stream)), "pdssm_scan_fwd")
+    return y, h_last, ws
+
+
+def pdssm_scan_fwd_single_pass(pi_dict, k, d, b, c, h0=None, chunk=128, ws=None, y=None,
+                               h_last=None, for_bwd=False, stream=None):
+    """The forward scan as one kernel (decoupled look-back); same results and
+    workspace as pdssm_scan_fwd.  Returns (y, h_last, ws)."""
+    B, H, L, N, K, stride = _scan_shapes(pi_dict, k, d, b, c)
+    dev = d.device
+    if ws is None:
+        ws = make_workspace(B, H, L, N, K, chunk, dev, stride != 0, for_bwd)
+    _cuda(ws, "ws", (torch.uint8,))
+    if h0 is not None:
+        _cuda(h0, "h0", (torch.float32,))
+    if y is None:
+        y = torch.empty((B, H, L), dtype=torch.float32, device=dev)
+    if h_last is None:
+        h_last = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dm = dims(B, H, L, N, K)
+    _check(_lib.pdssm_scan_fwd_single_pass(ctypes.byref(dm), _ptr(pi_dict), stride, _ptr(k),
+                                           _ptr(d), _ptr(b), _ptr(c), _dtype_code(d), _ptr(h0),
+                                           _ptr(y), _ptr(h_last), int(chunk), _ptr(ws),
+                                           ws.numel(), _stream(stream)),
+           "pdssm_scan_fwd_single_pass")
     return y, h_last, ws
 
 

@@ -242,7 +242,7 @@ pdssm_status scan_fwd_impl(const pdssm_dims *dims, const int32_t *pi_dict, int64
                            const int32_t *k, const void *d, const void *b, const void *c,
                            pdssm_dtype in_dtype, const float *h0, float *y, float *h_last,
                            int64_t chunk, void *ws, size_t ws_bytes, void *stream,
-                           pdssm_trace *trace) {
+                           pdssm_trace *trace, bool single_pass = false) {
     WsLayout w;
     pdssm_status st = fwd_common(dims, pi_dict, pi_head_stride, k, d, b, in_dtype, chunk, ws,
                                  ws_bytes, false, &w);
@@ -273,7 +273,10 @@ pdssm_status scan_fwd_impl(const pdssm_dims *dims, const int32_t *pi_dict, int64
     p.h0 = h0;
     p.y = y;
     p.h_last = h_last;
-    if (fused_path(p)) {
+    if (single_pass) {
+        if (!fused_path(p))
+            return arg_fail(PDSSM_ERR_UNSUPPORTED,
+                            "the single-pass forward needs N = 32 or 64 with 16-byte aligned rows");
         if ((e = tr.mark("single pass")) != cudaSuccess) return cuda_fail(e, "trace event");
         e = launch_scan_fused(p, in_dtype, s, false);
         if (e != cudaSuccess) return cuda_fail(e, "single-pass forward");
@@ -356,6 +359,15 @@ pdssm_status pdssm_scan_fwd(const pdssm_dims *dims, const int32_t *pi_dict,
                             void *stream) {
     return scan_fwd_impl(dims, pi_dict, pi_head_stride, k, d, b, c, in_dtype, h0, y, h_last,
                          chunk, ws, ws_bytes, stream, nullptr);
+}
+
+pdssm_status pdssm_scan_fwd_single_pass(const pdssm_dims *dims, const int32_t *pi_dict,
+                                        int64_t pi_head_stride, const int32_t *k, const void *d,
+                                        const void *b, const void *c, pdssm_dtype in_dtype,
+                                        const float *h0, float *y, float *h_last, int64_t chunk,
+                                        void *ws, size_t ws_bytes, void *stream) {
+    return scan_fwd_impl(dims, pi_dict, pi_head_stride, k, d, b, c, in_dtype, h0, y, h_last,
+                         chunk, ws, ws_bytes, stream, nullptr, true);
 }
 
 pdssm_status pdssm_scan_fwd_traced(const pdssm_dims *dims, const int32_t *pi_dict,

@@ -34,7 +34,8 @@ template <typename T, int NPL, int LV>
 __device__ __forceinline__ bool phaseA_segment(const ChunkParams &p, const SmemDict &sd,
                                                unsigned char *wbase, int64_t row0, int len,
                                                int lane, SegTransfer<NPL> &out,
-                                               const int32_t *ks = nullptr) {
+                                               const int32_t *ks = nullptr, int tbase = 0,
+                                               bool init_bars = true) {
     constexpr int N = 32 * NPL;
     constexpr int ROWB = N * (int)sizeof(T);
     constexpr int TENS = kTS * ROWB;
@@ -54,10 +55,11 @@ __device__ __forceinline__ bool phaseA_segment(const ChunkParams &p, const SmemD
     ring.src[1] = reinterpret_cast<const unsigned char *>(p.b) + row0 * ROWB;
     ring.src[2] = with_y ? reinterpret_cast<const unsigned char *>(p.c) + row0 * ROWB
                          : ring.src[1];
-    ring_init_bars(ring.bar0, kFastStages, lane);
+    if (init_bars) ring_init_bars(ring.bar0, kFastStages, lane);
+    const unsigned kAll = (1u << nt) - 1u;
 
     const int ntiles = (len + kTS - 1) / kTS;
-    for (int i = 0; i < kFastStages && i < ntiles; ++i) ring.issue(i, lane);
+    for (int i = 0; i < kFastStages && i < ntiles; ++i) ring.issue_tile(tbase + i, i, kAll, lane);
 
     const uint32_t map_s = smem_u32(sd.map);
     const uint32_t seg_lane = smem_u32(sd.seg) + lane * 8;
@@ -83,14 +85,16 @@ __device__ __forceinline__ bool phaseA_segment(const ChunkParams &p, const SmemD
     int kreg = clamp_k(kload(lane, lane < kTS && lane < len), K, p.status);
 
     for (int i = 0; i < ntiles; ++i) {
-        if (!ring.wait(i)) {
-            ring.abort(i, ntiles, p.status, lane);
+        if (!ring.wait(tbase + i)) {
+            if (lane == 0) flag_status(p.status, kStTimeout);
+            for (int j = i; j < ntiles && j < i + kFastStages; ++j) ring.wait(tbase + j);
+            __syncwarp();
             return false;
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
         const int knext = kload(t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
-        const uint32_t row0s = ring.tile(i);
+        const uint32_t row0s = ring.tile(tbase + i);
         // values of step q that do not depend on the state, loaded one step
         // ahead so their latency overlaps the previous step's work
         int kk = __shfl_sync(kFull, kreg, 0);
@@ -173,7 +177,7 @@ __device__ __forceinline__ bool phaseA_segment(const ChunkParams &p, const SmemD
             if ((lane & 3) == 0 && (lane >> 2) < n) yp[t0 + (lane >> 2)] = ys;
         }
         warp_barrier();
-        if (i + kFastStages < ntiles) ring.issue(i + kFastStages, lane);
+        if (i + kFastStages < ntiles) ring.issue_tile(tbase + i + kFastStages, i + kFastStages, kAll, lane);
         kreg = clamp_k(knext, K, p.status);
     }
 #pragma unroll
@@ -361,15 +365,16 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
 // ---------------------------------------------------------------------------
 // Single-pass forward (phases A, B and C in one kernel).
 //
-// One CTA per chunk; chunks are taken in the order of a ticket counter,
-// chunk-major (ticket t: chunk t / (B H) of sequence t % (B H)), so every
-// predecessor of a chunk in its sequence holds a smaller ticket and is
-// already running or done.  The chunk is cut into kFusedWarps sub-chunks,
-// one per warp:
+// Persistent CTAs of 8 warps in teams of W warps; a team takes one chunk at
+// a time, in the order of a ticket counter, chunk-major (ticket t: chunk
+// t / (B H) of sequence t % (B H)), so every predecessor of a chunk in its
+// sequence holds a smaller ticket and is being processed by a running team
+// or is done.  The chunk is cut into W sub-chunks of about 64 steps (W = 1,
+// 2, 4 or 8), one per warp of the team:
 //   1. each warp runs phase A on its sub-chunk (local readout into y, the
 //      sub-chunk's closed transfer);
-//   2. an inclusive Hillis-Steele scan over the warps composes the
-//      sub-chunk transfers (log2 kFusedWarps rounds in shared memory): warp
+//   2. an inclusive Hillis-Steele scan over the team composes the
+//      sub-chunk transfers (log2 W rounds in shared memory): warp
 //      w holds T_w o ... o T_0, the last warp the chunk's transfer A_c;
 //   3. the last warp publishes A_c (flag kFlagAgg); warp 0 finds the carry
 //      H_{c-1} by decoupled look-back: the nearest predecessor with a
@@ -385,7 +390,6 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC_fast(const ChunkParams 
 // up flags PDSSM_ERR_TIMEOUT, takes a zero carry and still publishes, so no
 // successor waits on it.
 // ---------------------------------------------------------------------------
-constexpr int kFusedWarps = 8;
 enum : int { kFlagAgg = 1, kFlagIncl = 2 };
 
 // Transfer of chunk `unit` (as published by another CTA of this grid) in the
@@ -413,7 +417,7 @@ __device__ __forceinline__ void load_published(const ChunkParams &p, int64_t uni
 // transfer_ops.cuh).  Each lane polls one predecessor flag; the window of 32
 // moves back while every flag in it is kFlagAgg.  Returns false if the wait
 // ran past p.wait_ns (x is then zero).
-__device__ __noinline__ bool lookback_carry(const ChunkParams &p, int64_t bh, int64_t cidx,
+__device__ __forceinline__ bool lookback_carry(const ChunkParams &p, int64_t bh, int64_t cidx,
                                             bool perm, ScatterScratch &sc, int lane,
                                             float (&x)[2]) {
     const int64_t u0 = bh * p.C;
@@ -460,10 +464,20 @@ __device__ __noinline__ bool lookback_carry(const ChunkParams &p, int64_t bh, in
         else
             x[r] = p.h0 ? p.h0[bh * p.N + e] : 0.f;
     }
+    // the aggregates after the base, oldest first; the next one's loads are
+    // in flight while the current one is applied
+    int P[2], Pn[2];
+    float D[2], V[2], Dn[2], Vn[2];
+    if (base + 1 < cidx) load_published(p, u0 + base + 1, lane, Pn, Dn, Vn);
     for (int64_t j = base + 1; j < cidx; ++j) {
-        int P[2];
-        float D[2], V[2], z[2];
-        load_published(p, u0 + j, lane, P, D, V);
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            P[r] = Pn[r];
+            D[r] = Dn[r];
+            V[r] = Vn[r];
+        }
+        if (j + 1 < cidx) load_published(p, u0 + j + 1, lane, Pn, Dn, Vn);
+        float z[2];
 #pragma unroll
         for (int r = 0; r < 2; ++r) z[r] = D[r] * x[r];
         warp_scatter(P, z, V, x, sc, lane, perm);
@@ -500,17 +514,17 @@ __device__ __forceinline__ float sq2(uint32_t w, float s) {
 }
 
 // The contract's fp32 fma chains of the candidate maps of one row (first
-// maximum in ascending k).
-__device__ __noinline__ int resolve_row(const ChunkParams &p, int64_t h, int64_t urow,
-                                        unsigned cand) {
-    const int D = p.D_in;
-    const __nv_bfloat16 *ur = reinterpret_cast<const __nv_bfloat16 *>(p.u) + urow * D;
+// maximum in ascending k).  Plain arguments: a reference to the kernel's
+// parameter block would make every thread copy it to local memory.
+__device__ __noinline__ int resolve_row(const __nv_bfloat16 *u, const float *Wsel, int D, int K,
+                                        int64_t h, int64_t urow, unsigned cand) {
+    const __nv_bfloat16 *ur = u + urow * D;
     float bv = 0.f;
     int best = -1;
     while (cand) {
         const int kk = __ffs(cand) - 1;
         cand &= cand - 1;
-        const float *wr = p.W_sel + (h * p.K + kk) * D;
+        const float *wr = Wsel + (h * K + kk) * D;
         float acc = 0.f;
         for (int q = 0; q < D; ++q) acc = __fmaf_rn(__ldg(wr + q), __bfloat162float(ur[q]), acc);
         if (best < 0 || acc > bv) {
@@ -522,8 +536,8 @@ __device__ __noinline__ int resolve_row(const ChunkParams &p, int64_t h, int64_t
 }
 
 // Selection of rows [0, n) starting at u row urow0 (b * L + t0) for head h:
-// writes k of each row into ks[row].  Whi / Wlo: [16][D/2] packed bf16
-// pairs of this head's W (rows >= K zero); Wn = max_k ||W_hk|| rounded up.
+// writes k of each row into ks[row].  Whi / Wlo: [K][D/2] packed bf16 pairs
+// of this head's W; Wn = max_k ||W_hk|| rounded up.
 __device__ void select_rows_mma(const ChunkParams &p, const uint32_t *Whi, const uint32_t *Wlo,
                                 float Wn, int64_t h, int64_t urow0, int n, int32_t *ks, int lane) {
     const int D = p.D_in, K = (int)p.K, D2 = D / 2;
@@ -548,9 +562,14 @@ __device__ void select_rows_mma(const ChunkParams &p, const uint32_t *Whi, const
 #pragma unroll
             for (int nt = 0; nt < 2; ++nt) {
                 if (nt >= ntl) break;
-                const int wrow = (nt * 8 + g) * D2 + kb + q;
-                mma_bf16_16816(acc[nt], a0, a1, a2, a3, Whi[wrow], Whi[wrow + 4]);
-                mma_bf16_16816(acc[nt], a0, a1, a2, a3, Wlo[wrow], Wlo[wrow + 4]);
+                // rows past K (staged only for k < K) contribute zero
+                const int n = nt * 8 + g;
+                const int wrow = n * D2 + kb + q;
+                const bool live = n < K;
+                mma_bf16_16816(acc[nt], a0, a1, a2, a3, live ? Whi[wrow] : 0u,
+                               live ? Whi[wrow + 4] : 0u);
+                mma_bf16_16816(acc[nt], a0, a1, a2, a3, live ? Wlo[wrow] : 0u,
+                               live ? Wlo[wrow + 4] : 0u);
             }
         }
         // row norms: the four lanes of a quad share rows g and g + 8
@@ -592,7 +611,8 @@ __device__ void select_rows_mma(const ChunkParams &p, const uint32_t *Whi, const
                 } else {
                     // near tie, or no finite logit: the exact chains decide
                     if (cand == 0) cand = (1u << K) - 1u;
-                    kv = resolve_row(p, h, urow0 + row, cand);
+                    kv = resolve_row(reinterpret_cast<const __nv_bfloat16 *>(p.u), p.W_sel, D,
+                                     K, h, urow0 + row, cand);
                 }
                 ks[row] = kv;
             }
@@ -611,110 +631,95 @@ struct FusedScratch {
     float xs[64];
 };
 
-template <typename T, int NPL, bool SEL>
-__global__ void __launch_bounds__(kFusedWarps * 32, 3) k_scan_fused(const ChunkParams p) {
-    extern __shared__ __align__(128) unsigned char sm_f_raw[];
-    unsigned char *sm = smem_base256(sm_f_raw);
-    pdl_trigger();
-    pdl_wait();   // dictionary tables and cleared flags come from the preceding work
+// Persistent CTAs of kFusedCtaWarps warps, split into teams of W warps; a
+// team takes one chunk (ticket) at a time and syncs on its own named
+// barrier, so teams never wait for one another.  The register budget is
+// sized for 24 resident warps per SM (16 for fp32 rows of 64, whose phase A
+// needs more than 80 registers).
+constexpr int kFusedCtaWarps = 8;
+
+template <typename T, int NPL>
+constexpr int fused_min_blocks() {
+    return (sizeof(T) == 4 && NPL == 2 ? 16 : 24) / kFusedCtaWarps;
+}
+
+// Shared memory of the persistent kernel: the header (tickets, chunk states,
+// carries, kFusedHeader bytes), the dictionary
+// (one slot for a shared dictionary, one per team otherwise), the warps'
+// regions, then (selection) each warp's indices and one staging area per
+// team for W_sel's hi / lo parts.
+// Header of the persistent kernel's shared memory (bytes): per team a ticket
+// and the max row norm of W_sel (16 bytes), per warp its FusedChunk, per
+// team the carry H_{c-1} (64 floats).
+constexpr int kFusedTickets = 0;
+constexpr int kFusedStates = kFusedTickets + kFusedCtaWarps * 16;
+constexpr int kFusedCarries = kFusedStates + kFusedCtaWarps * 48;
+constexpr int kFusedHeader = (kFusedCarries + kFusedCtaWarps * 256 + 255) / 256 * 256;
+
+struct FusedLayout {
+    size_t dict, regions, ks, wstage, total;
+    int slot, smax, wbytes;
+    bool wstage_own;
+};
+__host__ __device__ inline FusedLayout fused_layout(const ChunkParams &p, int W, bool sel) {
+    FusedLayout l;
+    const int teams = kFusedCtaWarps / W;
+    l.slot = dict_slot_bytes((int)p.K, (int)p.N, p.dict_content);
+    l.dict = (size_t)kFusedHeader;
+    l.regions = l.dict + (size_t)(p.dict_hs ? teams : 1) * l.slot;
+    l.ks = l.regions + (size_t)kFusedCtaWarps * p.smem_per_warp;
+    l.smax = (int)((p.chunk + W - 1) / W);
+    l.wbytes = 4 * (int)p.K * p.D_in;   // hi and lo bf16 parts of K rows
+    // (never inside the warps' regions: their ring barriers stay live from
+    // chunk to chunk)
+    l.wstage_own = sel;
+    l.wstage = l.ks + (sel ? (size_t)kFusedCtaWarps * l.smax * 4 : 0);
+    l.total = l.wstage + (l.wstage_own ? (size_t)teams * l.wbytes : 0);
+    return l;
+}
+
+__device__ __forceinline__ void team_sync(int team, int W) {
+    if (W == 1)
+        __syncwarp();
+    else
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + team), "r"(W * 32) : "memory");
+}
+
+// Per-warp state of the chunk in progress, parked in shared memory across
+// phase A so that it holds no registers there.
+struct FusedChunk {
+    int64_t unit, cidx, bh, row0;
+    int wlen, pad;
+};
+static_assert(sizeof(FusedChunk) <= 48, "chunk state slot");
+
+// Steps 2-4 of a chunk (after phase A) for one warp of a team; reloads the
+// chunk's state from shared memory and advances the ring slot count tb by
+// phase C's tiles.
+template <typename T, int NPL, bool SEL, int W, int LV>
+__device__ __forceinline__ void steps_2_to_4(const ChunkParams &p, unsigned char *sm,
+                                             const SegTransfer<NPL> &tr, bool ok, int &tb) {
     constexpr int N = 32 * NPL;
     constexpr int ROWB = N * (int)sizeof(T);
     constexpr int ES = (int)sizeof(T);
     using RingT = FastRing<3, ROWB>;
-    static_assert(kFastStages * RingT::STAGEB >= (int)sizeof(FusedScratch),
-                  "scan scratch must fit the staging ring");
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    unsigned long long *s_ticket = reinterpret_cast<unsigned long long *>(sm);
-    float *s_carry = reinterpret_cast<float *>(sm + 64);            // [64]
-    unsigned char *dict_s = sm + 512;
-    if (threadIdx.x == 0) *s_ticket = atomicAdd(p.ticket, 1ull);
-    __syncthreads();
-    const int64_t tk = (int64_t)*s_ticket;
-    const int64_t BH = p.B * p.H;
-    const int64_t cidx = tk / BH, bh = tk - cidx * BH;
-    const int64_t unit = bh * p.C + cidx;
-    copy_slot(dict_s, p, p.dict_hs ? (bh % p.H) : 0, threadIdx.x, blockDim.x, ES);
-    __syncthreads();
-    const SmemDict sd = dict_view(p, dict_s);
-    const bool perm = __ldg(p.dict_stats + 1) <= 1;   // every map a permutation
-
-    const int64_t s0 = cidx * p.chunk;
-    const int len = (int)imin64(p.chunk, p.L - s0);
-    const int S = (len + kFusedWarps - 1) / kFusedWarps;
-    const int ws0 = min(warp * S, len);
-    const int wlen = min(S, len - ws0);
-    const int64_t row0 = bh * p.L + s0 + ws0;
-    unsigned char *wregions = dict_s + dict_slot_bytes((int)p.K, (int)p.N, p.dict_content);
-    unsigned char *wbase = wregions + (size_t)warp * p.smem_per_warp;
-    const int32_t *ks = nullptr;
-
-    // 0. (SEL) the selection of this warp's sub-chunk, into shared memory
-    if constexpr (SEL) {
-        const int Smax = (int)((p.chunk + kFusedWarps - 1) / kFusedWarps);
-        int32_t *ksw = reinterpret_cast<int32_t *>(wregions + (size_t)kFusedWarps * p.smem_per_warp) +
-                       warp * Smax;
-        const int D = p.D_in, D2 = D / 2;
-        const int64_t hh = bh % p.H, bb = bh / p.H;
-        // W of this head split into bf16 hi / lo parts (rows >= K zero), in
-        // the warp regions (idle until phase A), and max_k ||W_hk|| rounded up
-        uint32_t *Whi = reinterpret_cast<uint32_t *>(wregions);
-        uint32_t *Wlo = Whi + 16 * D2;
-        int *wn_bits = reinterpret_cast<int *>(sm + 8);
-        if (threadIdx.x == 0) *wn_bits = 0;
-        __syncthreads();
-        for (int rr = warp; rr < 16; rr += kFusedWarps) {
-            float ss = 0.f;
-            for (int d2 = lane; d2 < D2; d2 += 32) {
-                float w0 = 0.f, w1 = 0.f;
-                if (rr < (int)p.K) {
-                    const float2 wv = *reinterpret_cast<const float2 *>(
-                        p.W_sel + (hh * p.K + rr) * D + 2 * d2);
-                    w0 = wv.x;
-                    w1 = wv.y;
-                }
-                const __nv_bfloat16 h0b = __float2bfloat16_rn(w0), h1b = __float2bfloat16_rn(w1);
-                const __nv_bfloat16 l0b = __float2bfloat16_rn(w0 - __bfloat162float(h0b));
-                const __nv_bfloat16 l1b = __float2bfloat16_rn(w1 - __bfloat162float(h1b));
-                Whi[rr * D2 + d2] = (uint32_t)__bfloat16_as_ushort(h0b) |
-                                    ((uint32_t)__bfloat16_as_ushort(h1b) << 16);
-                Wlo[rr * D2 + d2] = (uint32_t)__bfloat16_as_ushort(l0b) |
-                                    ((uint32_t)__bfloat16_as_ushort(l1b) << 16);
-                ss = __fmaf_ru(w0, w0, ss);
-                ss = __fmaf_ru(w1, w1, ss);
-            }
-#pragma unroll
-            for (int o = 16; o; o >>= 1) ss = __fadd_ru(ss, __shfl_xor_sync(kFull, ss, o));
-            if (lane == 0) atomicMax(wn_bits, __float_as_int(ss));   // non-negative: bits order
-        }
-        __syncthreads();
-        const float Wn = __fmul_ru(__fsqrt_ru(__int_as_float(*wn_bits)), 1.0009765625f);
-        select_rows_mma(p, Whi, Wlo, Wn, hh, bb * p.L + s0 + ws0, wlen, ksw, lane);
-        __syncwarp();
-        if (p.k_out)
-            for (int i = lane; i < wlen; i += 32) p.k_out[row0 + i] = ksw[i];
-        ks = ksw;
-        // every warp is done with W before phase A's copies land in the regions
-        fence_proxy_async_shared();
-        __syncthreads();
-    }
-
-    // 1. phase A of this warp's sub-chunk
-    SegTransfer<NPL> tr;
-    bool ok;
-    switch (step_variant(p.dict_stats)) {
-        case 0: ok = phaseA_segment<T, NPL, 0>(p, sd, wbase, row0, wlen, lane, tr, ks); break;
-        case 1: ok = phaseA_segment<T, NPL, 1>(p, sd, wbase, row0, wlen, lane, tr, ks); break;
-        case 2: ok = phaseA_segment<T, NPL, 2>(p, sd, wbase, row0, wlen, lane, tr, ks); break;
-        case 3: ok = phaseA_segment<T, NPL, 3>(p, sd, wbase, row0, wlen, lane, tr, ks); break;
-        default: ok = phaseA_segment<T, NPL, 5>(p, sd, wbase, row0, wlen, lane, tr, ks); break;
-    }
-    const int ntA = (wlen + kTS - 1) / kTS;
+    constexpr bool perm = LV == 0;
+    int tid = (int)threadIdx.x;
+    asm volatile("" : "+r"(tid));
+    const int warp = tid >> 5, lane = tid & 31;
+    const int team = warp / W, tw = warp - team * W;
+    const volatile FusedChunk *st = reinterpret_cast<const volatile FusedChunk *>(sm + kFusedStates) + warp;
+    const int64_t unit = st->unit, cidx = st->cidx, bh = st->bh, row0 = st->row0;
+    const int wlen = st->wlen;
+    const FusedLayout lay = fused_layout(p, W, SEL);
+    unsigned char *wteam = sm + lay.regions + (size_t)(team * W) * p.smem_per_warp;
+    unsigned char *wbase = wteam + (size_t)tw * p.smem_per_warp;
     FusedScratch &fs = *reinterpret_cast<FusedScratch *>(wbase);
-    FusedScratch &last = *reinterpret_cast<FusedScratch *>(
-        dict_s + dict_slot_bytes((int)p.K, (int)p.N, p.dict_content) +
-        (size_t)(kFusedWarps - 1) * p.smem_per_warp);
+    FusedScratch &last = *reinterpret_cast<FusedScratch *>(wteam + (size_t)(W - 1) * p.smem_per_warp);
+    float *t_carry = reinterpret_cast<float *>(sm + kFusedCarries) + team * 64;
+    const int ntA = (wlen + kTS - 1) / kTS;
 
-    // 2. the sub-chunk transfer into the scan layout, then the in-CTA scan
+    // 2. the sub-chunk transfer into the scan layout, then the team scan
     __syncwarp();
 #pragma unroll
     for (int r = 0; r < NPL; ++r) {
@@ -736,14 +741,14 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 3) k_scan_fused(const ChunkP
         a.D[r] = fs.D[0][lane + 32 * r];
         a.V[r] = fs.V[0][lane + 32 * r];
     }
-    __syncthreads();
+    team_sync(team, W);
     int cur = 0;
 #pragma unroll
-    for (int dd = 1; dd < kFusedWarps; dd <<= 1) {
-        if (warp >= dd) {
-            // this warp's aggregate goes after warp (warp - dd)'s
-            const FusedScratch &src = *reinterpret_cast<const FusedScratch *>(
-                wbase - (size_t)dd * p.smem_per_warp);
+    for (int dd = 1; dd < W; dd <<= 1) {
+        if (tw >= dd) {
+            // this warp's aggregate goes after warp (tw - dd)'s
+            const FusedScratch &src =
+                *reinterpret_cast<const FusedScratch *>(wbase - (size_t)dd * p.smem_per_warp);
             Agg lo;
 #pragma unroll
             for (int r = 0; r < 2; ++r) {
@@ -762,11 +767,11 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 3) k_scan_fused(const ChunkP
             fs.V[nxt][lane + 32 * r] = a.V[r];
         }
         cur = nxt;
-        __syncthreads();
+        team_sync(team, W);
     }
 
     // 3. publish the chunk's transfer; find and publish its carry
-    if (warp == kFusedWarps - 1) {
+    if (tw == W - 1) {
         const int64_t o = unit * p.N;
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
@@ -783,7 +788,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 3) k_scan_fused(const ChunkP
             if (lane == 0) st_release_gpu(p.look + unit, kFlagAgg);
         }
     }
-    if (warp == 0) {
+    if (tw == 0) {
         float x[2];
         if (cidx == 0) {
 #pragma unroll
@@ -812,19 +817,19 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 3) k_scan_fused(const ChunkP
                 p.Hc[o + e] = hc[r];
                 if (cidx == p.C - 1 && p.h_last) p.h_last[bh * p.N + e] = hc[r];
             }
-            s_carry[lane + 32 * r] = e < p.N ? x[r] : 0.f;
+            t_carry[lane + 32 * r] = e < p.N ? x[r] : 0.f;
         }
         __threadfence();
         __syncwarp();
         if (lane == 0) st_release_gpu(p.look + unit, kFlagIncl);
     }
-    __syncthreads();
+    team_sync(team, W);
 
-    // 4. this sub-chunk's carry, then its carry correction
+    // 4. this sub-chunk's carry, then its carry correction (ring slots tb ..)
     float xw[2];
 #pragma unroll
-    for (int r = 0; r < 2; ++r) xw[r] = s_carry[lane + 32 * r];
-    if (warp > 0) {
+    for (int r = 0; r < 2; ++r) xw[r] = t_carry[lane + 32 * r];
+    if (tw > 0) {
         const FusedScratch &prev = *reinterpret_cast<const FusedScratch *>(wbase - p.smem_per_warp);
         int P[2];
         float z[2], V[2];
@@ -842,13 +847,162 @@ __global__ void __launch_bounds__(kFusedWarps * 32, 3) k_scan_fused(const ChunkP
     float w[NPL];
 #pragma unroll
     for (int r = 0; r < NPL; ++r) w[r] = fs.xs[lane * NPL + r];
-    // every warp is done with the scratch before copies land in the rings
+    // the team is done with the scratch before copies land in its rings
     fence_proxy_async_shared();
-    __syncthreads();
-    if (ok && wlen > 0 && !(cidx == 0 && warp == 0 && p.h0 == nullptr)) {
+    team_sync(team, W);
+    if (ok && wlen > 0 && !(cidx == 0 && tw == 0 && p.h0 == nullptr)) {
+        const SmemDict sd = dict_view(p, sm + lay.dict + (p.dict_hs ? (size_t)team * lay.slot : 0));
+        const int32_t *ks = SEL ? reinterpret_cast<const int32_t *>(sm + lay.ks) + warp * lay.smax
+                                : nullptr;
         float *ybuf = reinterpret_cast<float *>(wbase + kFastStages * RingT::STAGEB) + 2 * kPbStride;
         phaseC_segment<T, NPL, 3, 2>(p, sd, smem_u32(wbase), smem_u32(ybuf + kYbufFloats), ybuf,
-                                     row0, wlen, w, ntA, lane, ks);
+                                     row0, wlen, w, tb, lane, ks);
+        tb += ntA;
+    }
+}
+
+// The chunk loop of one team (every warp of the CTA runs it); LV selects
+// phase A's PD step.
+template <typename T, int NPL, bool SEL, int W, int LV>
+__device__ __forceinline__ void fused_teams(const ChunkParams &p, unsigned char *sm) {
+    constexpr int N = 32 * NPL;
+    constexpr int ROWB = N * (int)sizeof(T);
+    constexpr int ES = (int)sizeof(T);
+    using RingT = FastRing<3, ROWB>;
+    constexpr bool perm = LV == 0;   // every map a permutation
+    int64_t cur_head = -1;
+    int tb = 0;
+
+    for (;;) {
+        // addresses are recomputed from an opaque thread index where they
+        // are used, so they are not held in registers across phase A
+        int tid = (int)threadIdx.x;
+        asm volatile("" : "+r"(tid));
+        const int warp = tid >> 5, lane = tid & 31;
+        const int team = warp / W, tw = warp - team * W;
+        unsigned long long *t_ticket = reinterpret_cast<unsigned long long *>(sm + kFusedTickets + team * 16);
+        FusedChunk *st = reinterpret_cast<FusedChunk *>(sm + kFusedStates) + warp;
+        team_sync(team, W);   // the previous chunk's reads of the header are done
+        if (tw == 0 && lane == 0) {
+            // after a wait gave up anywhere (status flagged), take no more
+            // chunks: waits on chunks nobody will process would each run to
+            // their cap
+            const bool stop = (*reinterpret_cast<volatile int *>(p.status) & kStTimeout) != 0;
+            *t_ticket = stop ? ~0ull : atomicAdd(p.ticket, 1ull);
+        }
+        team_sync(team, W);
+        const int64_t tk = (int64_t)*t_ticket;
+        if (tk < 0 || tk >= p.units) break;
+        const FusedLayout lay = fused_layout(p, W, SEL);
+        const int64_t BH = p.B * p.H;
+        const int64_t cidx = tk / BH, bh = tk - cidx * BH;
+        const int64_t hh = bh % p.H;
+        const int64_t s0 = cidx * p.chunk;
+        const int len = (int)imin64(p.chunk, p.L - s0);
+        const int S = (len + W - 1) / W;
+        const int ws0 = min(tw * S, len);
+        const int wlen = min(S, len - ws0);
+        const int64_t row0 = bh * p.L + s0 + ws0;
+        if (lane == 0) {
+            st->unit = bh * p.C + cidx;
+            st->cidx = cidx;
+            st->bh = bh;
+            st->row0 = row0;
+            st->wlen = wlen;
+        }
+        unsigned char *dict_s = sm + lay.dict + (p.dict_hs ? (size_t)team * lay.slot : 0);
+        if (p.dict_hs && hh != cur_head) {
+            copy_slot(dict_s, p, hh, tw * 32 + lane, W * 32, ES);
+            cur_head = hh;
+            team_sync(team, W);
+        }
+        unsigned char *wbase = sm + lay.regions + (size_t)warp * p.smem_per_warp;
+        const int32_t *ks = nullptr;
+
+        // 0. (SEL) the selection of this warp's sub-chunk, into shared memory
+        if constexpr (SEL) {
+            int *t_wn = reinterpret_cast<int *>(sm + kFusedTickets + team * 16 + 8);
+            int32_t *ksw = reinterpret_cast<int32_t *>(sm + lay.ks) + warp * lay.smax;
+            const int D = p.D_in, D2 = D / 2;
+            const int64_t bb = bh / p.H;
+            // W_sel of this head split into bf16 hi / lo parts in the team's
+            // staging area, and max_k ||W_hk|| rounded up
+            uint32_t *Whi = reinterpret_cast<uint32_t *>(sm + lay.wstage + (size_t)team * lay.wbytes);
+            uint32_t *Wlo = Whi + (int)p.K * D2;
+            if (tw == 0 && lane == 0) *t_wn = 0;
+            team_sync(team, W);
+            for (int rr = tw; rr < (int)p.K; rr += W) {
+                float ss = 0.f;
+                for (int d2 = lane; d2 < D2; d2 += 32) {
+                    const float2 wv = *reinterpret_cast<const float2 *>(
+                        p.W_sel + (hh * p.K + rr) * D + 2 * d2);
+                    const float w0 = wv.x, w1 = wv.y;
+                    const __nv_bfloat16 h0b = __float2bfloat16_rn(w0), h1b = __float2bfloat16_rn(w1);
+                    const __nv_bfloat16 l0b = __float2bfloat16_rn(w0 - __bfloat162float(h0b));
+                    const __nv_bfloat16 l1b = __float2bfloat16_rn(w1 - __bfloat162float(h1b));
+                    Whi[rr * D2 + d2] = (uint32_t)__bfloat16_as_ushort(h0b) |
+                                        ((uint32_t)__bfloat16_as_ushort(h1b) << 16);
+                    Wlo[rr * D2 + d2] = (uint32_t)__bfloat16_as_ushort(l0b) |
+                                        ((uint32_t)__bfloat16_as_ushort(l1b) << 16);
+                    ss = __fmaf_ru(w0, w0, ss);
+                    ss = __fmaf_ru(w1, w1, ss);
+                }
+#pragma unroll
+                for (int o = 16; o; o >>= 1) ss = __fadd_ru(ss, __shfl_xor_sync(kFull, ss, o));
+                if (lane == 0) atomicMax(t_wn, __float_as_int(ss));   // non-negative: bits order
+            }
+            team_sync(team, W);
+            const float Wn = __fmul_ru(__fsqrt_ru(__int_as_float(*t_wn)), 1.0009765625f);
+            select_rows_mma(p, Whi, Wlo, Wn, hh, bb * p.L + s0 + ws0, wlen, ksw, lane);
+            __syncwarp();
+            if (p.k_out)
+                for (int i = lane; i < wlen; i += 32) p.k_out[row0 + i] = ksw[i];
+            ks = ksw;
+            // the team is done with W_sel before phase A's copies land
+            fence_proxy_async_shared();
+            team_sync(team, W);
+        }
+
+        // 1. phase A of this warp's sub-chunk (ring slots tb ..)
+        SegTransfer<NPL> tr;
+        const bool ok =
+            phaseA_segment<T, NPL, LV>(p, dict_view(p, dict_s), wbase, row0, wlen, lane, tr, ks, tb, false);
+        tb += (wlen + kTS - 1) / kTS;
+        steps_2_to_4<T, NPL, SEL, W, LV>(p, sm, tr, ok, tb);
+    }
+}
+
+template <typename T, int NPL, bool SEL, int W>
+__global__ void __launch_bounds__(kFusedCtaWarps * 32, (fused_min_blocks<T, NPL>()))
+    k_scan_fused(const ChunkParams p) {
+    extern __shared__ __align__(128) unsigned char sm_f_raw[];
+    unsigned char *sm = smem_base256(sm_f_raw);
+    pdl_trigger();
+    pdl_wait();   // dictionary tables and cleared flags come from the preceding work
+    constexpr int N = 32 * NPL;
+    constexpr int ROWB = N * (int)sizeof(T);
+    constexpr int ES = (int)sizeof(T);
+    using RingT = FastRing<3, ROWB>;
+    static_assert(kFastStages * RingT::STAGEB >= (int)sizeof(FusedScratch),
+                  "scan scratch must fit the staging ring");
+    const FusedLayout lay = fused_layout(p, W, SEL);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int team = warp / W;
+    unsigned char *dict_s = sm + lay.dict + (p.dict_hs ? (size_t)team * lay.slot : 0);
+    unsigned char *wbase = sm + lay.regions + (size_t)warp * p.smem_per_warp;
+    float *ybuf = reinterpret_cast<float *>(wbase + kFastStages * RingT::STAGEB) + 2 * kPbStride;
+    const uint32_t bar0 = smem_u32(ybuf + kYbufFloats);
+    // a shared dictionary is staged once; this warp's ring barriers start
+    // here and keep their phases from chunk to chunk (slot tb)
+    if (p.dict_hs == 0) copy_slot(dict_s, p, 0, threadIdx.x, blockDim.x, ES);
+    ring_init_bars(bar0, kFastStages, lane);
+    __syncthreads();
+    switch (step_variant(p.dict_stats)) {
+        case 0: fused_teams<T, NPL, SEL, W, 0>(p, sm); break;
+        case 1: fused_teams<T, NPL, SEL, W, 1>(p, sm); break;
+        case 2: fused_teams<T, NPL, SEL, W, 2>(p, sm); break;
+        case 3: fused_teams<T, NPL, SEL, W, 3>(p, sm); break;
+        default: fused_teams<T, NPL, SEL, W, 5>(p, sm); break;
     }
 }
 
@@ -913,37 +1067,61 @@ bool fused_select_ok(const ChunkParams &p, const void *u, const float *W) {
            p.chunk <= 1024 && ((uintptr_t)u % 16) == 0 && ((uintptr_t)W % 16) == 0;
 }
 
-// The single-pass forward: one CTA of kFusedWarps warps per chunk; with
-// `select`, the CTA also takes its chunk's selection (p.u, p.W_sel).
-cudaError_t launch_scan_fused(ChunkParams p, pdssm_dtype dt, cudaStream_t st, bool select) {
-    const int es = dt == PDSSM_BF16 ? 2 : 4;
-    p.dict_content = (dt == PDSSM_BF16 ? kDictMap16 : kDictMap) | kDictSeg;
-    p.smem_per_warp = warp_smem_bytes(kFastStages, 3, (int)p.N * es);
-    p.wpc = kFusedWarps;
-    size_t smem = 512 + (size_t)dict_slot_bytes((int)p.K, (int)p.N, p.dict_content) +
-                  (size_t)kFusedWarps * p.smem_per_warp + 256;
-    if (select) {
-        // the sub-chunks' indices after the warp regions; W's hi / lo parts
-        // (64 D_in bytes) fit inside the regions
-        smem += (size_t)kFusedWarps * ((p.chunk + kFusedWarps - 1) / kFusedWarps) * 4;
-        if ((size_t)64 * p.D_in > (size_t)kFusedWarps * p.smem_per_warp) return cudaErrorInvalidValue;
-    }
+// Warps (sub-chunks) per chunk of the single-pass forward, by measurement on
+// the three benchmark workloads (chunk 128: 1 warp per chunk; chunk 256: 2).
+// More warps per chunk shorten the distance between phase A's read of a
+// sub-chunk and phase C's re-read (more L2 hits) but add team barriers and a
+// scan per chunk, which cost more than the hits save.
+static int fused_warps(int64_t chunk) { return chunk <= 128 ? 1 : 2; }
+
+// The single-pass forward: persistent CTAs (as many as fit the GPU, at most
+// one team per chunk), each of teams of fused_warps(chunk) warps; with
+// `select`, a team also takes its chunk's selection (p.u, p.W_sel).
+template <typename T, int NPL, bool SEL>
+static cudaError_t launch_fused_t(ChunkParams p, cudaStream_t st) {
+    const int W = fused_warps(p.chunk);
+    p.wpc = kFusedCtaWarps;
+    const size_t smem = fused_layout(p, W, SEL).total + 256;
     auto go = [&](auto kern) {
         cudaError_t e =
             cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
-        return launch_pdl(kern, dim3((unsigned)p.units), dim3(kFusedWarps * 32), smem, st, p);
+        int dev = 0, sms = 0, per_sm = 0;
+        if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+            return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kFusedCtaWarps * 32,
+                                                               smem)) != cudaSuccess)
+            return e;
+        if (per_sm < 1) return cudaErrorInvalidConfiguration;
+        const int64_t teams = kFusedCtaWarps / W;
+        const int64_t need = (p.units + teams - 1) / teams;
+        const int64_t grid = imin64((int64_t)sms * per_sm, need);
+        return launch_pdl(kern, dim3((unsigned)grid), dim3(kFusedCtaWarps * 32), smem, st, p);
     };
+    switch (W) {
+        case 1: return go(k_scan_fused<T, NPL, SEL, 1>);
+        case 2: return go(k_scan_fused<T, NPL, SEL, 2>);
+        case 4: return go(k_scan_fused<T, NPL, SEL, 4>);
+        default: return go(k_scan_fused<T, NPL, SEL, 8>);
+    }
+}
+
+cudaError_t launch_scan_fused(ChunkParams p, pdssm_dtype dt, cudaStream_t st, bool select) {
+    const int es = dt == PDSSM_BF16 ? 2 : 4;
+    p.dict_content = (dt == PDSSM_BF16 ? kDictMap16 : kDictMap) | kDictSeg;
+    p.smem_per_warp = warp_smem_bytes(kFastStages, 3, (int)p.N * es);
     if (select) {
         if (dt == PDSSM_BF16)
-            return p.N == 64 ? go(k_scan_fused<__nv_bfloat16, 2, true>)
-                             : go(k_scan_fused<__nv_bfloat16, 1, true>);
-        return p.N == 64 ? go(k_scan_fused<float, 2, true>) : go(k_scan_fused<float, 1, true>);
+            return p.N == 64 ? launch_fused_t<__nv_bfloat16, 2, true>(p, st)
+                             : launch_fused_t<__nv_bfloat16, 1, true>(p, st);
+        return p.N == 64 ? launch_fused_t<float, 2, true>(p, st)
+                         : launch_fused_t<float, 1, true>(p, st);
     }
     if (dt == PDSSM_BF16)
-        return p.N == 64 ? go(k_scan_fused<__nv_bfloat16, 2, false>)
-                         : go(k_scan_fused<__nv_bfloat16, 1, false>);
-    return p.N == 64 ? go(k_scan_fused<float, 2, false>) : go(k_scan_fused<float, 1, false>);
+        return p.N == 64 ? launch_fused_t<__nv_bfloat16, 2, false>(p, st)
+                         : launch_fused_t<__nv_bfloat16, 1, false>(p, st);
+    return p.N == 64 ? launch_fused_t<float, 2, false>(p, st) : launch_fused_t<float, 1, false>(p, st);
 }
 
 cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {

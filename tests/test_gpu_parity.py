@@ -30,12 +30,13 @@ def run_fwd(inp, chunk, k=None, for_bwd=False):
     return t, kk, y, hl, ws
 
 
-def check_fwd(inp, chunk, k_np=None):
+def check_fwd(inp, chunk, k_np=None, single=False):
     t = to_device(inp)
     if k_np is None:
         k_np = oracle_k(inp)
     kk = dev(k_np, torch.int32)
-    y, hl, ws = pd.pdssm_scan_fwd(t["pi"], kk, t["d"], t["b"], t["c"], t["h0"], chunk=chunk)
+    fwd = pd.pdssm_scan_fwd_single_pass if single else pd.pdssm_scan_fwd
+    y, hl, ws = fwd(t["pi"], kk, t["d"], t["b"], t["c"], t["h0"], chunk=chunk)
     torch.cuda.synchronize()
     assert pd.pdssm_ws_status(ws) == 0
     y_ref, hl_ref = oracle.scan_fwd(inp.pi, k_np, inp.d, inp.b, inp.c, inp.h0)
@@ -237,7 +238,8 @@ def test_single_pass_transfers_and_carries(N, dtype, kind):
     inp = small(N + len(kind), 2, 3, 1000, N, 6, kind=kind, dtype=dtype)
     chunk = 64
     t = to_device(inp)
-    y, hl, ws = pd.pdssm_scan_fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=chunk)
+    y, hl, ws = pd.pdssm_scan_fwd_single_pass(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"],
+                                              chunk=chunk)
     Pi, Dl, v, Hc = pd.pdssm_ws_transfers(ws, 2, 3, 1000, N, 6, chunk)
     torch.cuda.synchronize()
     assert pd.pdssm_ws_status(ws) == 0
@@ -254,7 +256,7 @@ def test_single_pass_transfers_and_carries(N, dtype, kind):
 def test_single_pass_chunk_sizes(chunk, N):
     """Chunks shorter than the CTA's eight sub-chunks leave warps with empty
     sub-chunks; ragged chunks and tails throughout."""
-    check_fwd(small(chunk + N, 1, 3, 777, N, 5), chunk=chunk)
+    check_fwd(small(chunk + N, 1, 3, 777, N, 5), chunk=chunk, single=True)
 
 
 @pytest.mark.parametrize("N,kind", [(32, "perm"), (64, "maps")])
@@ -262,7 +264,62 @@ def test_single_pass_long_look_back(N, kind):
     """One sequence of 60000 steps in chunks of 8: hundreds of chunks of the
     same sequence run at once, so look-backs walk back over whole windows of
     published aggregates."""
-    check_fwd(small(5, 1, 1, 60000, N, 8, kind=kind), chunk=8)
+    check_fwd(small(5, 1, 1, 60000, N, 8, kind=kind), chunk=8, single=True)
+
+
+@pytest.mark.parametrize("idx,over", [(2, dict(B=2, H=3, L=1000)), (3, dict(H=4, L=3000)),
+                                      (4, dict(B=1, H=3, L=2000))])
+def test_single_pass_workloads_reduced(idx, over):
+    inp = gen.generate(gen.workload(idx, **over))
+    check_fwd(inp, inp.cfg["chunk"], single=True)
+
+
+def test_single_pass_then_backward():
+    """The single-pass forward leaves the workspace the adjoint reads: the
+    backward after it matches the oracle."""
+    inp = small(9, 2, 2, 700, 64, 6)
+    t = to_device(inp)
+    y, hl, ws = pd.pdssm_scan_fwd_single_pass(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"],
+                                              chunk=64, for_bwd=True)
+    g = pd.pdssm_scan_bwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], t["g_y"], ws, chunk=64)
+    torch.cuda.synchronize()
+    assert pd.pdssm_ws_status(ws) == 0
+    ref = oracle.scan_bwd(inp.pi, inp.k, inp.d, inp.b, inp.c, inp.h0, inp.g_y)
+    for a, r in zip(g, ref):
+        assert floored_relerr(a.cpu().numpy(), r) <= TOL_F32
+
+
+def test_single_pass_rejects_unsupported_shapes():
+    inp = small(1, 1, 1, 50, 24, 3)
+    t = to_device(inp)
+    with pytest.raises(pd.PdssmError):
+        pd.pdssm_scan_fwd_single_pass(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=16)
+
+
+@pytest.mark.parametrize("idx", [2, 3])
+def test_single_pass_full_size_equals_three_kernels(idx):
+    """Full benchmark sizes: the single-pass forward and the three-kernel
+    forward agree within the workload's tolerance (and bitwise-equal
+    integer transfers), and each is deterministic."""
+    cfg = gen.workload(idx)
+    inp = gen.generate(cfg)
+    t = to_device(inp)
+    k = t["k"] if t["k"] is not None else pd.pdssm_select(t["u"], t["W"])
+    y3, h3, ws3 = pd.pdssm_scan_fwd(t["pi"], k, t["d"], t["b"], t["c"], t["h0"], chunk=cfg["chunk"])
+    y1, h1, ws1 = pd.pdssm_scan_fwd_single_pass(t["pi"], k, t["d"], t["b"], t["c"], t["h0"],
+                                                chunk=cfg["chunk"])
+    y1b, h1b, _ = pd.pdssm_scan_fwd_single_pass(t["pi"], k, t["d"], t["b"], t["c"], t["h0"],
+                                                chunk=cfg["chunk"])
+    torch.cuda.synchronize()
+    assert pd.pdssm_ws_status(ws1) == 0
+    assert torch.equal(y1, y1b) and torch.equal(h1, h1b)
+    tol = tol_for(inp)
+    assert floored_relerr(y1.cpu().numpy(), y3.cpu().numpy()) <= tol
+    assert floored_relerr(h1.cpu().numpy(), h3.cpu().numpy()) <= tol
+    B, H, L, N = inp.d.shape
+    P1 = pd.pdssm_ws_transfers(ws1, B, H, L, N, cfg["K"], cfg["chunk"])[0]
+    P3 = pd.pdssm_ws_transfers(ws3, B, H, L, N, cfg["K"], cfg["chunk"])[0]
+    assert torch.equal(P1, P3)
 
 
 @pytest.mark.parametrize("which", [0, 1])
@@ -454,11 +511,13 @@ def test_forward_empty_sequence():
     assert torch.equal(hl, t["h0"])
 
 
-def test_forward_deterministic():
+@pytest.mark.parametrize("single", [False, True])
+def test_forward_deterministic(single):
     inp = gen.generate(gen.workload(4, B=1, H=4, L=4096))
     t = to_device(inp)
-    y1, h1, _ = pd.pdssm_scan_fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=128)
-    y2, h2, _ = pd.pdssm_scan_fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=128)
+    fwd = pd.pdssm_scan_fwd_single_pass if single else pd.pdssm_scan_fwd
+    y1, h1, _ = fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=128)
+    y2, h2, _ = fwd(t["pi"], t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=128)
     assert torch.equal(y1, y2) and torch.equal(h1, h2)
 
 
