@@ -56,6 +56,9 @@ def parse():
                     help="override L (small cases for profiler captures)")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the stiff and forward+adjoint workloads of the default run")
+    ap.add_argument("--forward", default="three_kernels", choices=["three_kernels", "single_pass"],
+                    help="forward scan entry point: pdssm_scan_fwd (phases A, B, C) or "
+                         "pdssm_scan_fwd_single_pass (one kernel, decoupled look-back)")
     return ap.parse_args()
 
 
@@ -291,7 +294,8 @@ def run_ours(args, cfg):
     # the other two benchmark workloads of the method, on the default run
     # at one GPU: the long stiff forward and the forward + exact adjoint
     if rank == 0 and out is not None and world == 1 and not args.no_extra and \
-            workload_index(args.workload) == DEFAULT_WORKLOAD and not (args.batch or args.seq_len):
+            workload_index(args.workload) == DEFAULT_WORKLOAD and \
+            not (args.batch or args.seq_len) and args.forward == "three_kernels":
         out["extra"] = {}
         for idx in EXTRA_WORKLOADS:
             xcfg = gen.workload(idx)
@@ -459,6 +463,8 @@ def measure(args, cfg, torch, pd, dev, world, rank, dist, K_steps, with_e2e, wit
                  torch.empty_like(d, dtype=torch.float32),
                  torch.empty((B, H, N), dtype=torch.float32, device=dev))
     stream = torch.cuda.current_stream()
+    single = getattr(args, "forward", "three_kernels") == "single_pass"
+    fwd = pd.pdssm_scan_fwd_single_pass if single else pd.pdssm_scan_fwd
 
     # kernel-level timing on a sample of the timed steps: events recorded
     # between the kernels of those steps (the other steps run without them,
@@ -477,12 +483,20 @@ def measure(args, cfg, torch, pd, dev, world, rank, dist, K_steps, with_e2e, wit
             launches["n"] += 1
         else:
             k = k_given
-        if tr is not None:
+        if tr is not None and not single:
             tr["fwd_res"] = pd.pdssm_scan_fwd_traced(pi, k, d, b, c, h0, chunk, ws, y, h_last,
                                                      tr["fwd"], stream=stream)
+        elif tr is not None:
+            # one kernel (after the plans): time the call as a whole
+            tr["fwd"][0].record(stream)
+            pd.pdssm_scan_fwd_single_pass(pi, k, d, b, c, h0, chunk=chunk, ws=ws, y=y,
+                                          h_last=h_last, stream=stream)
+            tr["fwd"][1].record(stream)
+            evs = tr["fwd"]
+            tr["fwd_res"] = lambda evs=evs: [("prep + single pass", evs[0].elapsed_time(evs[1]))]
         else:
-            pd.pdssm_scan_fwd(pi, k, d, b, c, h0, chunk=chunk, ws=ws, y=y, h_last=h_last,
-                              for_bwd=grad, stream=stream)
+            fwd(pi, k, d, b, c, h0, chunk=chunk, ws=ws, y=y, h_last=h_last, for_bwd=grad,
+                stream=stream)
         launches["n"] += launches_fwd
         if grad:
             if tr is not None:
@@ -500,7 +514,7 @@ def measure(args, cfg, torch, pd, dev, world, rank, dist, K_steps, with_e2e, wit
     launches_fwd = launches_bwd = 0
     step(-1)
     torch.cuda.synchronize()
-    launches_fwd = len(probe["fwd_res"]())
+    launches_fwd = 2 if single else len(probe["fwd_res"]())
     launches_bwd = len(probe["bwd_res"]()) if grad else 0
     del traced[-1]
     for _ in range(args.warmup):
@@ -565,7 +579,7 @@ def measure(args, cfg, torch, pd, dev, world, rank, dist, K_steps, with_e2e, wit
     peaks, peak_kind = measured_peaks()
     fwd_bytes, bwd_bytes, sel_bytes = algorithmic_bytes(cfg)
     achieved = fwd_bytes / (scan_ms * 1e-3) / 1e9
-    fwd_kernels = [n for n, _ in probe["fwd_res"]()]
+    fwd_kernels = ["prep", "single pass"] if single else [n for n, _ in probe["fwd_res"]()]
     roofline = {"kernel": "pdssm_scan_fwd (" + " + ".join(fwd_kernels) + ")",
                 "bound": "hbm", "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "peak_kind": peak_kind, "unit": "GB/s",
@@ -584,7 +598,9 @@ def measure(args, cfg, torch, pd, dev, world, rank, dist, K_steps, with_e2e, wit
            "steps": K_steps, "warmup": args.warmup, "ms_per_step": ms_step,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
            "dtype": "bf16" if bf else "f32", "data": "synthetic (seeded PCG64)",
-           "config": config_json(cfg, world), "roofline": roofline, "phases_ms": phases_ms,
+           "config": dict(config_json(cfg, world),
+                          forward="pdssm_scan_fwd_single_pass" if single else "pdssm_scan_fwd"),
+           "roofline": roofline, "phases_ms": phases_ms,
            "gpu_launches": launches["n"], "clocks": clk.report(),
            "e2e": e2e}
     if with_cpu and world == 1:
