@@ -78,6 +78,7 @@ ChunkParams make_params(const pdssm_dims *dm, const WsLayout &w, void *ws, int64
     p.tab = reinterpret_cast<const uint8_t *>(base + w.tab);
     p.fan = reinterpret_cast<const int32_t *>(base + w.fan);
     p.seg = reinterpret_cast<const uint2 *>(base + w.seg);
+    p.segw = reinterpret_cast<const uint2 *>(base + w.segw);
     p.dict_stats = reinterpret_cast<const int *>(base + w.status) + 1;
     p.k = k;
     p.d = d;
@@ -200,7 +201,7 @@ static pdssm_status run_prep(const pdssm_dims *dims, const int32_t *pi_dict,
                              cudaStream_t st) {
     unsigned char *base = reinterpret_cast<unsigned char *>(ws);
     // status word and the dictionary statistics (largest segment lane
-    // distance, largest fan-in)
+    // distance, largest fan-in, largest window back-span)
     cudaError_t e = cudaMemsetAsync(base + w.status, 0, 16, st);
     if (e != cudaSuccess) return cuda_fail(e, "status reset");
     // the single-pass forward's ticket counter and per-chunk flags
@@ -208,6 +209,7 @@ static pdssm_status run_prep(const pdssm_dims *dims, const int32_t *pi_dict,
     if (e != cudaSuccess) return cuda_fail(e, "look-back reset");
     e = launch_prep(*dims, pi_dict, pi_head_stride, reinterpret_cast<int32_t *>(base + w.dict),
                     reinterpret_cast<uint2 *>(base + w.seg),
+                    reinterpret_cast<uint2 *>(base + w.segw),
                     reinterpret_cast<int *>(base + w.status) + 1,
                     reinterpret_cast<uint8_t *>(base + w.tab),
                     reinterpret_cast<int32_t *>(base + w.fan), w.Hd,

@@ -297,11 +297,17 @@ __global__ void __launch_bounds__(kMaxWPC * 32, 2) k_bwdC_fast(const ChunkParams
     const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
     if (unit >= p.units) return;
     unsigned char *wbase = sm_bc + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
-    switch (step_variant(p.dict_stats)) {
+    switch (step_variant(p.dict_stats, NPL)) {
         case 0: bwdC_fast_unit<T, NPL, 0>(p, sd, wbase, unit, lane); break;
         case 1: bwdC_fast_unit<T, NPL, 1>(p, sd, wbase, unit, lane); break;
         case 2: bwdC_fast_unit<T, NPL, 2>(p, sd, wbase, unit, lane); break;
         case 3: bwdC_fast_unit<T, NPL, 3>(p, sd, wbase, unit, lane); break;
+        case kStepWin:
+            if constexpr (NPL == 2) {
+                bwdC_fast_unit<T, NPL, kStepWin>(p, sd, wbase, unit, lane);
+                break;
+            }
+            [[fallthrough]];
         default: bwdC_fast_unit<T, NPL, 5>(p, sd, wbase, unit, lane); break;
     }
 }

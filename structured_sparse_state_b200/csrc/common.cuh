@@ -40,7 +40,7 @@ enum : int { kStBadIndex = 1, kStTimeout = 2 };
 // workspace layout (all offsets 256-byte aligned)
 // ---------------------------------------------------------------------------
 struct WsLayout {
-    size_t status, dict, tab, fan, seg, look, Pi, Dl, v, Hc, wc, lam, total;
+    size_t status, dict, tab, fan, seg, segw, look, Pi, Dl, v, Hc, wc, lam, total;
     int64_t C, Hd;
 };
 
@@ -65,6 +65,7 @@ inline WsLayout ws_layout(const pdssm_dims &dm, int64_t pi_hs, int64_t chunk,
     w.tab = o;    o = align256(o + (size_t)(w.Hd * dm.K * kDcap * 64));
     w.fan = o;    o = align256(o + (size_t)(w.Hd * dm.K) * 4);
     w.seg = o;    o = align256(o + (size_t)(w.Hd * dm.K) * 32 * 8);
+    w.segw = o;   o = align256(o + (size_t)(w.Hd * dm.K) * 32 * 8);
     w.look = o;   o = align256(o + kLookHeader + units * 4);
     w.Pi = o;     o = align256(o + vecs);
     w.Dl = o;     o = align256(o + vecs);
@@ -88,8 +89,10 @@ struct ChunkParams {
     const uint8_t *tab;       // slot tables [Hd][K][kDcap][64]: s-th source of each target
     const int32_t *fan;       // largest fan-in of each map [Hd][K]
     const uint2 *seg;         // segment tables [Hd][K][32 lanes] (N = 32 or 64)
+    const uint2 *segw;        // window tables [Hd][K][32 lanes] (N = 64)
     const int *dict_stats;    // over all maps: [0] largest lane distance inside a
-                              // segment, [1] largest fan-in (1: all permutations)
+                              // segment, [1] largest fan-in (1: all permutations),
+                              // [2] largest back-span of the window tables (N = 64)
     int dict_content;         // parts of the dictionary staged in shared memory
     const int32_t *k;
     const void *d, *b, *c;
@@ -697,6 +700,18 @@ __device__ __forceinline__ unsigned char *smem_base256(unsigned char *raw) {
                                              ~uintptr_t(255));
 }
 
+// Step variant for a launch: 0 when every map is a permutation; kStepWin
+// (N = 64) when every map's window table reaches back at most two lanes;
+// else the shuffle levels of the segment tables: the smallest LV in
+// {1, 2, 3, 5} with 2^LV above the largest lane distance inside a segment.
+constexpr int kStepWin = 8;
+__device__ __forceinline__ int step_variant(const int *dict_stats, int npl) {
+    if (__ldg(dict_stats + 1) <= 1) return 0;
+    if (npl == 2 && __ldg(dict_stats + 2) <= 2) return kStepWin;
+    const int md = __ldg(dict_stats);
+    return md < 2 ? 1 : md < 4 ? 2 : md < 8 ? 3 : 5;
+}
+
 struct SmemDict {
     const int *map;        // [K][N] (2-byte entries with kDictMap16)
     const uint8_t *tab;    // [K][kDcap][64]
@@ -729,7 +744,8 @@ __device__ __forceinline__ void copy_slot(unsigned char *dst, const ChunkParams 
     if (c & kDictSeg) {
         off = (off + 7) / 8 * 8;
         uint2 *g = reinterpret_cast<uint2 *>(dst + off);
-        const uint2 *gs = p.seg + dk * K * 32;
+        const bool win = N == 64 && step_variant(p.dict_stats, 2) == kStepWin;
+        const uint2 *gs = (win ? p.segw : p.seg) + dk * K * 32;
         for (int i = tid; i < K * 32; i += nthr) g[i] = __ldg(gs + i);
     }
 }
@@ -899,27 +915,75 @@ __device__ __forceinline__ void step_perm(float (&h)[NPL], const float (&dv)[NPL
     }
 }
 
-// One PD step: LV = 0 selects the permutation step, otherwise the
-// segment-table step with LV shuffle levels; both take the exchange buffer
-// of the step's parity (pb or ob).
+// The PD step through the map's window table (N = 64, two entries per
+// lane).  The map's targets are ordered by decreasing fan-in, each target's
+// sources (ascending j) forming one segment of consecutive entries, with a
+// single-source target moved in front of an even-sized segment that would
+// otherwise start at an odd entry; so a segment of up to six sources
+// reaches back at most two lanes from the lane holding its last entry.
+// Each lane forms the partial of its last segment inside the lane ("tail"),
+// and a segment that continues into the lane from the left gets the tails of
+// the D <= 2 lanes it spans, fetched by two independent shuffles (no
+// dependent scan levels).  The owners of the targets then fetch each
+// segment's sum from the lane holding its last entry.  d * h goes to
+// per-map slots of the exchange buffer chosen (a bank colouring of the
+// bipartite graph of writer and reader instructions) so that both stores
+// and both gathers of a step touch 32 distinct banks.
+//
+// Entry word e (per map and lane):
+//   e.x: byte offsets (slot * 4) of source a, source b, the slot this lane
+//        writes element 2 * lane to, and the slot of element 2 * lane + 1
+//   e.y: bit 0 a and b share a target; bit 1 a continues the previous lane's
+//        segment; bits 2-3 D, the lanes back to the start of a's segment
+//        (when bit 1 is set); bits 4, 5 this lane's own targets have sources;
+//        bits 16-20 / 21 the lane and entry (0: a, 1: b) ending the first own
+//        target's segment, bits 22-26 / 27 the same for the second.
+// The sum of each target follows a fixed order, so the step is
+// deterministic.  pb is 256-byte aligned; callers alternate two buffers.
+__device__ __forceinline__ void step_win(float (&h)[2], const float (&dv)[2], const float (&bv)[2],
+                                         uint32_t pb, uint2 e) {
+    const uint32_t w0 = e.x, w1 = e.y;
+    sts_f32(__byte_perm(w0, pb, 0x7652), dv[0] * h[0]);
+    sts_f32(__byte_perm(w0, pb, 0x7653), dv[1] * h[1]);
+    warp_barrier();
+    const float za = lds_f32(__byte_perm(w0, pb, 0x7650));
+    const float zb = lds_f32(__byte_perm(w0, pb, 0x7651));
+    const bool ab_same = w1 & 1u;
+    const float tail = ab_same ? za + zb : zb;
+    const float t1 = __shfl_up_sync(kFull, tail, 1);
+    const float t2 = __shfl_up_sync(kFull, tail, 2);
+    const uint32_t D = (w1 >> 2) & 3u;
+    float back = D >= 1u ? t1 : 0.f;
+    if (D >= 2u) back += t2;
+    // sa: the sum of a's segment up to a; v: the sum of b's segment up to b
+    const float sa = ((w1 >> 1) & 1u) ? za + back : za;
+    const float v = ab_same ? sa + zb : zb;
+    const int l0 = (int)((w1 >> 16) & 31u), l1 = (int)((w1 >> 22) & 31u);
+    const float a0 = __shfl_sync(kFull, sa, l0), b0 = __shfl_sync(kFull, v, l0);
+    const float a1 = __shfl_sync(kFull, sa, l1), b1 = __shfl_sync(kFull, v, l1);
+    const float x0 = ((w1 >> 21) & 1u) ? b0 : a0;
+    const float x1 = ((w1 >> 27) & 1u) ? b1 : a1;
+    h[0] = ((w1 >> 4) & 1u ? x0 : 0.f) + bv[0];
+    h[1] = ((w1 >> 5) & 1u ? x1 : 0.f) + bv[1];
+}
+
+// One PD step: LV = 0 selects the permutation step, kStepWin the window
+// step (N = 64), otherwise the segment-table step with LV shuffle levels;
+// each takes the exchange buffer of the step's parity (pb or ob).
 template <int NPL, int LV>
 __device__ __forceinline__ void pd_step(float (&h)[NPL], const float (&dv)[NPL],
                                         const float (&bv)[NPL], uint32_t pb, uint32_t ob,
                                         uint2 e, int lane, int parity) {
-    if constexpr (LV == 0)
+    if constexpr (LV == 0) {
         step_perm<NPL>(h, dv, bv, parity ? ob : pb, e, lane);
-    else
+    } else if constexpr (LV == kStepWin) {
+        static_assert(NPL == 2, "the window step serves N = 64");
+        step_win(h, dv, bv, parity ? ob : pb, e);
+    } else {
         step_seg<NPL, LV>(h, dv, bv, parity ? ob : pb, e, lane);
+    }
 }
 
-// Step variant for a launch: 0 when every map is a permutation, else the
-// shuffle levels of the segment tables: the smallest LV in {1, 2, 3, 5} with
-// 2^LV above the largest lane distance inside a segment.
-__device__ __forceinline__ int step_variant(const int *dict_stats) {
-    if (__ldg(dict_stats + 1) <= 1) return 0;
-    const int md = __ldg(dict_stats);
-    return md < 2 ? 1 : md < 4 ? 2 : md < 8 ? 3 : 5;
-}
 
 // Programmatic dependent launch: a kernel launched with launch_pdl may start
 // while its predecessor in the stream finishes; pdl_wait() blocks until the
@@ -1028,7 +1092,7 @@ bool select_tc_supported(const pdssm_dims &dm, pdssm_dtype ut, const void *u, co
 cudaError_t launch_select_tc(const pdssm_dims &dm, const void *u, const float *W, int32_t *k_out,
                              float *logits_out, float *scale_out, cudaStream_t st);
 cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
-                        uint2 *seg, int *dict_stats,
+                        uint2 *seg, uint2 *segw, int *dict_stats,
                         uint8_t *tab, int32_t *fan, int64_t Hd, int *status, cudaStream_t st);
 cudaError_t launch_validate(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs,
                             const int32_t *k, int *counts, cudaStream_t st);

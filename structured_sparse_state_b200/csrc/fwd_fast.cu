@@ -222,11 +222,17 @@ __global__ void __launch_bounds__(kMaxWPC * 32, (sizeof(T) == 4 && NPL == 2) ? 2
     const int64_t unit = (int64_t)blockIdx.x * p.wpc + warp;
     if (unit >= p.units) return;
     unsigned char *wbase = sm_a + dict_region_bytes(p) + (size_t)warp * p.smem_per_warp;
-    switch (step_variant(p.dict_stats)) {
+    switch (step_variant(p.dict_stats, NPL)) {
         case 0: phaseA_fast_unit<T, NPL, 0>(p, sd, wbase, unit, lane); break;
         case 1: phaseA_fast_unit<T, NPL, 1>(p, sd, wbase, unit, lane); break;
         case 2: phaseA_fast_unit<T, NPL, 2>(p, sd, wbase, unit, lane); break;
         case 3: phaseA_fast_unit<T, NPL, 3>(p, sd, wbase, unit, lane); break;
+        case kStepWin:
+            if constexpr (NPL == 2) {
+                phaseA_fast_unit<T, NPL, kStepWin>(p, sd, wbase, unit, lane);
+                break;
+            }
+            [[fallthrough]];
         default: phaseA_fast_unit<T, NPL, 5>(p, sd, wbase, unit, lane); break;
     }
 }
@@ -997,11 +1003,17 @@ __global__ void __launch_bounds__(kFusedCtaWarps * 32, (fused_min_blocks<T, NPL>
     if (p.dict_hs == 0) copy_slot(dict_s, p, 0, threadIdx.x, blockDim.x, ES);
     ring_init_bars(bar0, kFastStages, lane);
     __syncthreads();
-    switch (step_variant(p.dict_stats)) {
+    switch (step_variant(p.dict_stats, NPL)) {
         case 0: fused_teams<T, NPL, SEL, W, 0>(p, sm); break;
         case 1: fused_teams<T, NPL, SEL, W, 1>(p, sm); break;
         case 2: fused_teams<T, NPL, SEL, W, 2>(p, sm); break;
         case 3: fused_teams<T, NPL, SEL, W, 3>(p, sm); break;
+        case kStepWin:
+            if constexpr (NPL == 2) {
+                fused_teams<T, NPL, SEL, W, kStepWin>(p, sm);
+                break;
+            }
+            [[fallthrough]];
         default: fused_teams<T, NPL, SEL, W, 5>(p, sm); break;
     }
 }

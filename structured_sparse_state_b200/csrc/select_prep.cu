@@ -127,8 +127,120 @@ cudaError_t launch_select(const pdssm_dims &dm, const void *u, pdssm_dtype ut, c
 // ---------------------------------------------------------------------------
 constexpr int kPrepWarps = 4;
 
+// Window table of one map with N = 64 (read by step_win, which documents the
+// entry word).  Order of the segments: fan-in 8 down to 2, targets ascending
+// within a fan-in, and before the first segment of an even fan-in that would
+// start at an odd entry, the next single-source target (at most three such
+// moves); the remaining single-source targets follow.  A segment of fan-in f
+// <= 6 then reaches back at most two lanes.  dict_stats[2] gets the largest
+// back-span (99 when a fan-in exceeds 8).  Lane l holds sources j = l and
+// j = l + 32 (targets ta, tb, ranks rank_a, rank_b among their target's
+// sources) and the fan-ins cnt0, cnt1 of targets l and l + 32; fmax is the
+// map's largest fan-in.  Every index into the 64-entry scratch arrays is
+// masked to stay inside them.
+__device__ __forceinline__ void prep_window(int64_t m, int lane, int ta, int tb, int rank_a,
+                                            int rank_b, int cnt0, int cnt1, int fmax,
+                                            int *s_start, int *s_src, int *s_tgt,
+                                            const int *s_cnt, int *s_ent, int *s_slot,
+                                            uint2 *__restrict__ segw, int *dict_stats) {
+    __syncwarp();   // the segment table's reads of the scratch arrays are done
+    if (fmax > 8) {
+        if (lane == 0) atomicMax(dict_stats + 2, 99);
+        return;
+    }
+    const unsigned lt = (1u << lane) - 1u;
+    // group of each fan-in: counts, and ranks of this lane's two targets
+    unsigned lo[9], hi[9];
+#pragma unroll
+    for (int f = 1; f <= 8; ++f) {
+        lo[f] = __ballot_sync(kFull, cnt0 == f);
+        hi[f] = __ballot_sync(kFull, cnt1 == f);
+    }
+    int gstart[9];
+    int ins0 = -1, ins1 = -1, ins2 = -1, nins = 0;
+    const int n1 = __popc(lo[1]) + __popc(hi[1]);
+    int pos = 0;
+#pragma unroll
+    for (int f = 8; f >= 2; --f) {
+        const int nf = __popc(lo[f]) + __popc(hi[f]);
+        gstart[f] = pos;
+        if (nf > 0 && (f & 1) == 0 && (pos & 1) && nins < 3 && nins < n1) {
+            if (nins == 0) ins0 = pos;
+            else if (nins == 1) ins1 = pos;
+            else ins2 = pos;
+            ++nins;
+            ++pos;
+            gstart[f] = pos;
+        }
+        pos += nf * f;
+    }
+    const int tail = pos;
+    auto start_of = [&](int f, int rank) {
+        if (f == 0) return -1;
+        if (f >= 2) {
+            int g = 0;
+#pragma unroll
+            for (int q = 2; q <= 8; ++q)
+                if (q == f) g = gstart[q];
+            return g + rank * f;
+        }
+        return rank == 0 && nins > 0 ? ins0 : rank == 1 && nins > 1 ? ins1
+             : rank == 2 && nins > 2 ? ins2 : tail + (rank - nins);
+    };
+    int r0 = 0, r1 = 0;
+#pragma unroll
+    for (int f = 1; f <= 8; ++f) {
+        if (cnt0 == f) r0 = __popc(lo[f] & lt);
+        if (cnt1 == f) r1 = __popc(lo[f]) + __popc(hi[f] & lt);
+    }
+    s_start[lane] = start_of(cnt0, r0);
+    s_start[lane + 32] = start_of(cnt1, r1);
+    __syncwarp();
+    // entries of the sources j = lane, lane + 32
+    const int ea = (s_start[ta & 63] + rank_a) & 63, eb = (s_start[tb & 63] + rank_b) & 63;
+    s_ent[lane] = ea;
+    s_ent[lane + 32] = eb;
+    s_src[ea] = lane;
+    s_tgt[ea] = ta;
+    s_src[eb] = lane + 32;
+    s_tgt[eb] = tb;
+    __syncwarp();
+    // bank colouring: element 2l is stored by the first store of lane l,
+    // element 2l + 1 by the second; the gather of entry e is the first
+    // (e even) or the second (e odd) load.  Colours 0 .. m - 1 go to the
+    // elements stored first and gathered first and to those stored second
+    // and gathered second, m .. 31 to the two mixed classes.
+    const bool a_first = (s_ent[2 * lane] & 1) == 0, b_first = (s_ent[2 * lane + 1] & 1) == 0;
+    const unsigned ma = __ballot_sync(kFull, a_first), mb = __ballot_sync(kFull, b_first);
+    const int mcount = __popc(ma);
+    const int col_a = a_first ? __popc(ma & lt) : mcount + __popc(~ma & lt);
+    const int col_b = b_first ? mcount + __popc(mb & lt) : __popc(~mb & lt);
+    s_slot[2 * lane] = col_a & 31;
+    s_slot[2 * lane + 1] = 32 + (col_b & 31);
+    __syncwarp();
+    const int a = 2 * lane, b = 2 * lane + 1;
+    const int src_a = s_src[a], src_b = s_src[b];
+    const int tg_a = s_tgt[a], tg_b = s_tgt[b];
+    const bool ab_same = tg_a == tg_b;
+    const bool a_cont = lane > 0 && s_tgt[a - 1] == tg_a;
+    const int D = a_cont ? lane - (s_start[tg_a & 63] >> 1) : 0;
+    const int f0 = s_cnt[a], f1 = s_cnt[b];   // fan-ins of this lane's own targets
+    const int e0 = f0 > 0 ? (s_start[a] + f0 - 1) & 63 : 0;
+    const int e1 = f1 > 0 ? (s_start[b] + f1 - 1) & 63 : 0;
+    const uint32_t w0 = (uint32_t)(s_slot[src_a & 63] * 4) | (uint32_t)(s_slot[src_b & 63] * 4) << 8 |
+                        (uint32_t)(s_slot[a] * 4) << 16 | (uint32_t)(s_slot[b] * 4) << 24;
+    const uint32_t w1 = (ab_same ? 1u : 0u) | (a_cont ? 2u : 0u) | (uint32_t)(min(D, 3)) << 2 |
+                        (f0 > 0 ? 1u : 0u) << 4 | (f1 > 0 ? 1u : 0u) << 5 |
+                        (uint32_t)(e0 >> 1) << 16 | (uint32_t)(e0 & 1) << 21 |
+                        (uint32_t)(e1 >> 1) << 22 | (uint32_t)(e1 & 1) << 27;
+    segw[m * 32 + lane] = make_uint2(w0, w1);
+    const int mdw = __reduce_max_sync(kFull, D);
+    if (lane == 0) atomicMax(dict_stats + 2, mdw);
+}
+
 __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *__restrict__ dict,
-                       uint2 *__restrict__ seg, int *__restrict__ dict_stats,
+                       uint2 *__restrict__ seg, uint2 *__restrict__ segw,
+                       int *__restrict__ dict_stats,
                        uint8_t *__restrict__ tab, int32_t *__restrict__ fan, int64_t nmaps,
                        int K, int N, int *status) {
     __shared__ int s_off[kPrepWarps][65];   // first sorted entry of each target (+ total)
@@ -136,6 +248,8 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
     __shared__ int s_tgt[kPrepWarps][64];   // sorted entries: target
     __shared__ int s_cnt0[kPrepWarps][64];  // sources of each target among j < 32
     __shared__ int s_cnt[kPrepWarps][64];   // sources of each target
+    __shared__ int s_ent[kPrepWarps][64];   // window table: entry of each source
+    __shared__ int s_slot[kPrepWarps][64];  // window table: exchange slot of each element
     pdl_trigger();
     const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
     const int64_t m = (int64_t)blockIdx.x * (blockDim.x >> 5) + wib;
@@ -252,14 +366,16 @@ __global__ void k_prep(const int32_t *__restrict__ pi, int64_t pi_hs, int32_t *_
     seg[m * 32 + lane] = make_uint2(w0, w1);
     const int md = __reduce_max_sync(kFull, dist);
     if (lane == 0) atomicMax(dict_stats, md);
+    if (N == 64) prep_window(m, lane, ta, tb, rank_a, rank_b, cnt0, cnt1, D, s_off[wib], s_src[wib],
+                             s_tgt[wib], s_cnt[wib], s_ent[wib], s_slot[wib], segw, dict_stats);
 }
 
 cudaError_t launch_prep(const pdssm_dims &dm, const int32_t *pi, int64_t pi_hs, int32_t *dict,
-                        uint2 *seg, int *dict_stats,
+                        uint2 *seg, uint2 *segw, int *dict_stats,
                         uint8_t *tab, int32_t *fan, int64_t Hd, int *status, cudaStream_t st) {
     const int64_t nmaps = Hd * dm.K;
     const int64_t grid = (nmaps + kPrepWarps - 1) / kPrepWarps;
-    k_prep<<<(unsigned)grid, 32 * kPrepWarps, 0, st>>>(pi, pi_hs, dict, seg, dict_stats, tab, fan,
+    k_prep<<<(unsigned)grid, 32 * kPrepWarps, 0, st>>>(pi, pi_hs, dict, seg, segw, dict_stats, tab, fan,
                                                        nmaps, (int)dm.K, (int)dm.N, status);
     return cudaGetLastError();
 }

@@ -453,16 +453,44 @@ def _lane_distance(row, npl):
     return md
 
 
+def _window_span(row):
+    """Largest back-span in lanes of the window table of one N = 64 map
+    (None when a fan-in exceeds 8): segments in decreasing fan-in, targets
+    ascending within a fan-in, a single-source target moved in front of an
+    even-sized segment that would start at an odd entry (at most three
+    times), the remaining single-source targets last; two entries per lane."""
+    cnt = np.bincount(row, minlength=64)
+    if cnt.max() > 8:
+        return None
+    n1 = int((cnt == 1).sum())
+    pos, nins, starts = 0, 0, {}
+    for f in range(8, 1, -1):
+        tg = [t for t in range(64) if cnt[t] == f]
+        if tg and f % 2 == 0 and pos % 2 == 1 and nins < 3 and nins < n1:
+            nins += 1
+            pos += 1
+        for t in tg:
+            starts[t] = pos
+            pos += f
+    span = 0
+    for t, s0 in starts.items():
+        span = max(span, (s0 + cnt[t] - 1) // 2 - s0 // 2)
+    return span
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("N,fan,levels", [
     (32, 2, 1), (32, 3, 2), (32, 5, 3), (32, 9, 5),
-    (64, 3, 1), (64, 5, 2), (64, 9, 3), (64, 17, 5)])
+    (64, 3, 0), (64, 5, 0), (64, 6, 0), (64, 7, 2), (64, 9, 3), (64, 17, 5)])
 def test_segment_step_shuffle_levels(N, fan, levels, dtype):
     """Maps that are permutations except for one target receiving `fan`
     sources.  The run of that target's sources spans a number of lanes that
     decides how many shuffle levels the segmented sum of the state update
     takes (1, 2, 3 or 5 levels for runs spanning under 2, 4, 8 or 32
-    lanes); each case lands in the class named by `levels`."""
+    lanes); each case lands in the class named by `levels`.  With N = 64 a
+    dictionary whose window tables reach back at most two lanes takes the
+    window step instead (levels = 0); fan-ins of 7 and more fall back to the
+    segment scan."""
     inp = small(70 + N + fan, 2, 2, 400, N, 5, dtype=dtype)
     rng = np.random.default_rng(N * 100 + fan)
     pi = inp.pi.copy()
@@ -473,8 +501,43 @@ def test_segment_step_shuffle_levels(N, fan, levels, dtype):
         pi[kk] = row
     inp.pi = pi
     md = max(_lane_distance(r, N // 32) for r in pi)
-    assert {1: md < 2, 2: 2 <= md < 4, 3: 4 <= md < 8, 5: md >= 8}[levels], md
+    if N == 64:
+        spans = [_window_span(r) for r in pi]
+        window = all(sp is not None and sp <= 2 for sp in spans)
+        assert window == (levels == 0), spans
+    if levels:
+        assert {1: md < 2, 2: 2 <= md < 4, 3: 4 <= md < 8, 5: md >= 8}[levels], md
     check_fwd(inp, chunk=64)
+    check_bwd(inp, chunk=64)
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("case", ["mixed_fan_in", "no_single_source", "pairs_only",
+                                  "fan_in_seven"])
+def test_window_step_dictionaries(case, dtype):
+    """N = 64 dictionaries around the window table's limits: maps mixing
+    fan-ins 2 to 6 with single-source targets to move in front of
+    misaligned even-sized segments, maps with no single-source target at
+    all, maps whose targets all have two sources (no segment crosses a
+    lane), and maps with one target of fan-in 7 (a back-span of three
+    lanes: the segment scan takes over)."""
+    sizes = {"mixed_fan_in": [6, 5, 4, 4, 3, 2, 2],
+             "no_single_source": [6, 5, 5, 4, 4, 3, 3] + [2] * 17,
+             "pairs_only": [2] * 32,
+             "fan_in_seven": [7, 3, 2]}[case]
+    sizes = sizes + [1] * (64 - sum(sizes))
+    rng = np.random.default_rng(len(case))
+    inp = small(90 + len(case), 2, 2, 333, 64, 6, dtype=dtype)
+    rows = []
+    for _ in range(inp.pi.shape[0]):
+        targets = rng.permutation(64)[:len(sizes)]
+        row = np.concatenate([[t] * f for t, f in zip(targets, sizes)])
+        rows.append(row[rng.permutation(64)].astype(np.int32))
+    inp.pi = np.stack(rows)
+    spans = [_window_span(r) for r in inp.pi]
+    assert all(sp is not None and sp <= 2 for sp in spans) == (case != "fan_in_seven"), spans
+    check_fwd(inp, chunk=64)
+    check_fwd(inp, chunk=128)
     check_bwd(inp, chunk=64)
 
 
