@@ -588,6 +588,13 @@ def measure(args, cfg, torch, pd, dev, world, rank, dist, K_steps, with_e2e, wit
                 "algorithmic_bytes_per_launch": fwd_bytes,
                 "launch_ms": round(scan_ms, 5),
                 "launch_samples": len(sampled)}
+    if roofline["traffic"]:
+        # the DRAM bytes ncu counted per launch over the same launch time: the
+        # rate HBM actually sustained (the three-phase split re-reads d and c,
+        # so this is above the algorithmic rate)
+        dram_gbs = roofline["traffic"] / (scan_ms * 1e-3) / 1e9
+        roofline["dram_achieved"] = round(dram_gbs, 1)
+        roofline["dram_frac"] = round(dram_gbs / peaks["hbm_gbs"], 4)
     if grad:
         bwd_ms = sum(v for n, v in phases_ms.items() if n.startswith("bwd"))
         roofline["bwd"] = {"kernel": "pdssm_scan_bwd", "algorithmic_bytes_per_launch": bwd_bytes,

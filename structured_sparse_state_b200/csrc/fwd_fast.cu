@@ -279,7 +279,16 @@ __device__ __forceinline__ bool phaseC_segment(const ChunkParams &p, const SmemD
         return valid ? (ks ? kp[idx] : __ldg(kp + idx)) : 0;
     };
     float *yp = p.y + row0;
+    // the global loads of a tile (its local readout y, written by phase A,
+    // and the selection indices) are issued a tile ahead of their use: y of
+    // tile i + 1 and the indices of tile i + 2 load while tile i runs
+    auto yload = [&](int ti) {
+        const int t = ti * kTS + (lane >> 2);
+        return ((lane & 3) == 0 && t < len && (lane >> 2) < kTS) ? yp[t] : 0.f;
+    };
     int kreg = clamp_k(kload(lane, lane < kTS && lane < len), K, p.status);
+    int knext = kload(kTS + lane, lane < kTS && kTS + lane < len);
+    float ycur = yload(0);
 
     for (int i = 0; i < ntiles; ++i) {
         if (!ring.wait(tbase + i)) {
@@ -290,8 +299,8 @@ __device__ __forceinline__ bool phaseC_segment(const ChunkParams &p, const SmemD
         }
         const int t0 = i * kTS;
         const int n = min(kTS, len - t0);
-        const int knext = kload(t0 + kTS + lane, lane < kTS && t0 + kTS + lane < len);
-        const float yold = ((lane & 3) == 0 && (lane >> 2) < n) ? yp[t0 + (lane >> 2)] : 0.f;
+        const int knn = kload(t0 + 2 * kTS + lane, lane < kTS && t0 + 2 * kTS + lane < len);
+        const float ynext = yload(i + 1);
         const uint32_t row0s = ring.tile(tbase + i);
         if (n == kTS) {
             // full tile: steps unrolled, row and readout offsets immediate
@@ -328,10 +337,12 @@ __device__ __forceinline__ bool phaseC_segment(const ChunkParams &p, const SmemD
         }
         warp_barrier();
         const float ys = ybuf_quad_sum(ybuf, lane);
-        if ((lane & 3) == 0 && (lane >> 2) < n) yp[t0 + (lane >> 2)] = yold + ys;
+        if ((lane & 3) == 0 && (lane >> 2) < n) yp[t0 + (lane >> 2)] = ycur + ys;
         warp_barrier();
         if (i + kFastStages < ntiles) ring.issue_tile(tbase + i + kFastStages, i + kFastStages, kMask, lane);
         kreg = clamp_k(knext, K, p.status);
+        knext = knn;
+        ycur = ynext;
     }
     return true;
 }
