@@ -194,13 +194,19 @@ __device__ __forceinline__ void apply_gather(const int (&P)[NPL], const float (&
     __syncwarp();
 }
 
+// One CTA of nw warps per (b, h), or (G > 1) a cluster of G CTAs per
+// sequence: the chunks are split over G * nw warps; each CTA reduces its
+// warps' aggregates to a CTA total by a five-level tree, and warp 0 of CTA r
+// starts from g_hlast advanced through the totals of CTAs G - 1 .. r + 1,
+// read through distributed shared memory.
 template <int NPL>
-__global__ void k_bwdB(const ChunkParams p) {
+__global__ void k_bwdB(const ChunkParams p, int G) {
     extern __shared__ __align__(16) unsigned char sm_bb[];
     const int nw = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int N = (int)p.N;
-    const int64_t bh = blockIdx.x;
+    const int64_t bh = blockIdx.x / G;
+    const int rank = G > 1 ? (int)cluster_rank() : 0;
     const int64_t C = p.C;
     float *sXall = reinterpret_cast<float *>(sm_bb);             // [nw][64]
     int *sPall = reinterpret_cast<int *>(sXall + nw * kMaxN);     // [nw][64]
@@ -209,10 +215,16 @@ __global__ void k_bwdB(const ChunkParams p) {
     float *aggD = reinterpret_cast<float *>(aggP + nw * kMaxN);
     float *aggW = aggD + nw * kMaxN;
     float *carry = aggW + nw * kMaxN;
+    // G > 1: the reduction tree's aggregates [nw][64] (P, D, W); slot 0 ends
+    // up with the CTA total
+    int *treP = reinterpret_cast<int *>(carry + nw * kMaxN);
+    float *treD = reinterpret_cast<float *>(treP + nw * kMaxN);
+    float *treW = treD + nw * kMaxN;
     float *sX = sXall + warp * kMaxN;
     int *sP = sPall + warp * kMaxN;
     float *sD = sDall + warp * kMaxN;
-    const int64_t c0 = C * warp / nw, c1 = C * (warp + 1) / nw;
+    const int64_t gw = (int64_t)rank * nw + warp, nwt = (int64_t)G * nw;
+    const int64_t c0 = C * gw / nwt, c1 = C * (gw + 1) / nwt;
     const int64_t u0 = bh * C;
 
     if (c0 < c1) {
@@ -253,12 +265,79 @@ __global__ void k_bwdB(const ChunkParams p) {
         }
     }
     __syncthreads();
+    if (G > 1) {
+        // the CTA total R_0 o R_1 o ... o R_{nw-1} (R_0 applied last): at
+        // level d, warp w (w a multiple of 2d) composes its slot with slot
+        // w + d: w = w_a + D_a * w_b[P_a], D = D_a * D_b[P_a], P = P_b[P_a].
+        // Every warp's segment is non-empty (at least 64 chunks per CTA).
+        int tP[NPL];
+        float tD[NPL], tW[NPL];
+#pragma unroll
+        for (int r = 0; r < NPL; ++r) {
+            const int e = lane * NPL + r;
+            tP[r] = e < N ? aggP[warp * kMaxN + e] : 0;
+            tD[r] = e < N ? aggD[warp * kMaxN + e] : 0.f;
+            tW[r] = e < N ? aggW[warp * kMaxN + e] : 0.f;
+            if (e < N) {
+                treP[warp * kMaxN + e] = tP[r];
+                treD[warp * kMaxN + e] = tD[r];
+                treW[warp * kMaxN + e] = tW[r];
+            }
+        }
+        __syncthreads();
+        for (int d = 1; d < nw; d <<= 1) {
+            const bool active = (warp % (2 * d)) == 0 && warp + d < nw;
+            if (active) {
+                const int b0 = (warp + d) * kMaxN;
+#pragma unroll
+                for (int r = 0; r < NPL; ++r) {
+                    const int q = tP[r];
+                    tW[r] = tW[r] + tD[r] * treW[b0 + q];
+                    tD[r] = tD[r] * treD[b0 + q];
+                    tP[r] = treP[b0 + q];
+                }
+            }
+            __syncthreads();
+            if (active) {
+#pragma unroll
+                for (int r = 0; r < NPL; ++r) {
+                    const int e = lane * NPL + r;
+                    if (e < N) {
+                        treP[warp * kMaxN + e] = tP[r];
+                        treD[warp * kMaxN + e] = tD[r];
+                        treW[warp * kMaxN + e] = tW[r];
+                    }
+                }
+            }
+            __syncthreads();
+        }
+        cluster_sync_all();   // every CTA's total (slot 0) is in place
+    }
     if (warp == 0) {
         float x[NPL];
 #pragma unroll
         for (int r = 0; r < NPL; ++r) {
             const int e = lane * NPL + r;
             x[r] = (e < N && p.g_hlast) ? p.g_hlast[bh * p.N + e] : 0.f;
+        }
+        // the cluster's later CTAs, last first
+        for (int q = G - 1; q > rank; --q) {
+            int P[NPL];
+            float D[NPL], W[NPL];
+#pragma unroll
+            for (int r = 0; r < NPL; ++r) {
+                const int e = lane * NPL + r;
+                const int ee = e < N ? e : 0;
+                P[r] = ldc_s32(cluster_map(smem_u32(treP + ee), (uint32_t)q));
+                D[r] = ldc_f32(cluster_map(smem_u32(treD + ee), (uint32_t)q));
+                W[r] = ldc_f32(cluster_map(smem_u32(treW + ee), (uint32_t)q));
+                if (e >= N) {
+                    P[r] = 0;
+                    D[r] = 0.f;
+                    W[r] = 0.f;
+                }
+            }
+            apply_gather<NPL>(P, D, W, x, sX, N, lane);
         }
         for (int w = nw - 1; w >= 0; --w) {
 #pragma unroll
@@ -279,7 +358,7 @@ __global__ void k_bwdB(const ChunkParams p) {
                 apply_gather<NPL>(P, D, W, x, sX, N, lane);
             }
         }
-        if (p.g_h0) {
+        if (p.g_h0 && rank == 0) {
 #pragma unroll
             for (int r = 0; r < NPL; ++r) {
                 const int e = lane * NPL + r;
@@ -287,7 +366,11 @@ __global__ void k_bwdB(const ChunkParams p) {
             }
         }
     }
-    __syncthreads();
+    // every CTA is done reading the others' totals (G > 1); carries visible
+    if (G > 1)
+        cluster_sync_all();
+    else
+        __syncthreads();
     float x[NPL];
 #pragma unroll
     for (int r = 0; r < NPL; ++r) {
@@ -513,24 +596,42 @@ cudaError_t launch_bwdC(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st) {
     return dt == PDSSM_BF16 ? bwdC_t<__nv_bfloat16>(p, st) : bwdC_t<float>(p, st);
 }
 
+template <int NPL>
+static cudaError_t launch_bwdB_t(const ChunkParams &p, int nw, int G, cudaStream_t st) {
+    const size_t smem = (size_t)nw * kMaxN * 4 * (G > 1 ? 10 : 7);
+    const int64_t BH = p.B * p.H;
+    cudaError_t e =
+        cudaFuncSetAttribute(k_bwdB<NPL>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (G > 1) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3((unsigned)(BH * G));
+        cfg.blockDim = dim3(nw * 32);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = st;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = (unsigned)G;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, k_bwdB<NPL>, p, G);
+    }
+    k_bwdB<NPL><<<(unsigned)BH, nw * 32, smem, st>>>(p, G);
+    return cudaGetLastError();
+}
+
 cudaError_t launch_bwdB(const ChunkParams &p, cudaStream_t st) {
     if (p.units == 0) return cudaSuccess;
     const int nw = (int)imin64(32, p.C);
-    const size_t smem = (size_t)nw * kMaxN * 4 * 7;
-    const int64_t BH = p.B * p.H;
-    cudaError_t e;
-    if (p.N > 32) {
-        e = cudaFuncSetAttribute(k_bwdB<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-        if (e != cudaSuccess) return e;
-        k_bwdB<2><<<(unsigned)BH, nw * 32, smem, st>>>(p);
-    } else {
-        e = cudaFuncSetAttribute(k_bwdB<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
-        if (e != cudaSuccess) return e;
-        k_bwdB<1><<<(unsigned)BH, nw * 32, smem, st>>>(p);
-    }
-    return cudaGetLastError();
+    int dev = 0, sms = 148;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    const int G = carry_scan_cluster(p.B * p.H, p.C, sms);
+    return p.N > 32 ? launch_bwdB_t<2>(p, nw, G, st) : launch_bwdB_t<1>(p, nw, G, st);
 }
 
 }  // namespace pdssm

@@ -1011,6 +1011,67 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
     return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
+// Distributed shared memory of a thread-block cluster (1-D clusters): this
+// CTA's rank, the address of a shared variable of this CTA mapped to the same
+// variable of CTA `rank`, plain loads through such an address, and the
+// barrier over every thread of every CTA of the cluster (release / acquire,
+// so shared-memory writes before it are visible to the cluster after it).
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ int ldc_s32(uint32_t a) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ float ldc_f32(uint32_t a) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(a) : "memory");
+    return v;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\t"
+                 "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// launch_pdl with clusters of `cluster` CTAs along x (the grid a multiple).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_cluster_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                      int cluster, cudaStream_t st, Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = (unsigned)cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
+// CTAs per sequence of the carry scans (phase B, bwd B): with few sequences
+// a sequence's chunks are split over a cluster of G CTAs (G a power of two
+// up to 8, G x sequences within the SM count, at least 64 chunks per CTA),
+// so that more SMs share the scan.
+inline int carry_scan_cluster(int64_t BH, int64_t C, int sms) {
+    int G = 1;
+    while (G < 8 && BH * 2 * G <= sms && C >= (int64_t)64 * 2 * G) G *= 2;
+    return G;
+}
+
 // Warps per CTA for a chunk kernel with `per_warp` bytes of shared memory
 // per warp: 4 or 8, whichever keeps more warps resident per SM by the
 // runtime's occupancy calculation (registers, shared memory with the

@@ -238,38 +238,49 @@ __global__ void __launch_bounds__(kMaxWPC * 32) k_phaseC(const ChunkParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// phase B: one CTA of nw warps per (b, h).  Chunks are split into nw
-// contiguous segments: (1) each warp composes its segment's transfers into
-// one aggregate, (2) the aggregates are combined by an inclusive
-// Hillis-Steele scan (log2 nw rounds) and applied to h0, which gives every
-// segment's carry, (3) each warp re-applies its segment's transfers from its
-// carry and stores every H_c.  Transfers are held in the layout of
+// phase B: G CTAs of nw warps per (b, h) (G > 1: one thread-block cluster
+// per sequence).  Chunks are split into G * nw contiguous segments: (1) each
+// warp composes its segment's transfers into one aggregate, (2) the
+// aggregates of a CTA are combined by an inclusive Hillis-Steele scan
+// (log2 nw rounds); with G > 1 each CTA publishes its total in shared memory
+// and, after a cluster barrier, warp 0 of CTA r applies the totals of CTAs
+// 0 .. r - 1, read through distributed shared memory, to h0, which gives the
+// CTA's carry-in; the scan applied to the carry-in gives every segment's
+// carry, (3) each warp re-applies its segment's transfers from its carry
+// and stores every H_c.  Transfers are held in the layout of
 // transfer_ops.cuh (lane l: elements l and l + 32).
 // ---------------------------------------------------------------------------
 
 constexpr int kBGroup = 2;   // transfers loaded together
 
-__global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p) {
+__global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p, int G) {
     extern __shared__ __align__(16) unsigned char sm_b[];
     const int nw = blockDim.x >> 5;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_trigger();
     pdl_wait();   // the chunk transfers come from the preceding kernel
-    const int64_t bh = blockIdx.x;
+    const int64_t bh = blockIdx.x / G;
+    const int rank = G > 1 ? (int)cluster_rank() : 0;
     const int64_t C = p.C;
     const bool perm = __ldg(p.dict_stats + 1) <= 1;   // every map a permutation
-    // [2 buffers][nw][64] aggregates, [nw][64] carries, [nw] scratch
+    // [2 buffers][nw][64] aggregates, [nw][64] carries, [nw] scratch, this
+    // CTA's total (P, D, V) and its carry-in
     int *aggP = reinterpret_cast<int *>(sm_b);
     float *aggD = reinterpret_cast<float *>(aggP + 2 * nw * 64);
     float *aggV = aggD + 2 * nw * 64;
     float *carry = aggV + 2 * nw * 64;
     ScatterScratch *scr = reinterpret_cast<ScatterScratch *>(carry + nw * 64);
     ScatterScratch &sc = scr[warp];
+    int *totP = reinterpret_cast<int *>(scr + nw);
+    float *totD = reinterpret_cast<float *>(totP + 64);
+    float *totV = totD + 64;
+    float *xin = totV + 64;
     // the staged chunk transfer of the level-1 gathers reuses key / val
     int *tP = sc.key;
     float *tD = sc.val;
 
-    const int64_t c0 = C * warp / nw, c1 = C * (warp + 1) / nw;
+    const int64_t gw = (int64_t)rank * nw + warp, nwt = (int64_t)G * nw;
+    const int64_t c0 = C * gw / nwt, c1 = C * (gw + 1) / nwt;
     const int64_t u0 = bh * C;
 
     // (1) segment aggregate T_{c1-1} o ... o T_{c0}; identity for an empty segment
@@ -356,14 +367,53 @@ __global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p) {
         cur = nxt;
         __syncthreads();
     }
-    // carry at the end of this warp's segment: (prefix aggregate)(h0)
+    // the CTA's carry-in: h0, advanced (G > 1) through the totals of the
+    // cluster's earlier CTAs
+    if (G > 1) {
+        if (warp == nw - 1) {
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int e = lane + 32 * r;
+                totP[e] = a.P[r];
+                totD[e] = a.D[r];
+                totV[e] = a.V[r];
+            }
+        }
+        cluster_sync_all();
+        if (warp == 0) {
+            float x[2];
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int e = lane + 32 * r;
+                x[r] = p.h0 && e < p.N ? p.h0[bh * p.N + e] : 0.f;
+            }
+            for (int q = 0; q < rank; ++q) {
+                int P[2];
+                float D[2], V[2], z[2];
+#pragma unroll
+                for (int r = 0; r < 2; ++r) {
+                    const int e = lane + 32 * r;
+                    P[r] = ldc_s32(cluster_map(smem_u32(totP + e), (uint32_t)q));
+                    D[r] = ldc_f32(cluster_map(smem_u32(totD + e), (uint32_t)q));
+                    V[r] = ldc_f32(cluster_map(smem_u32(totV + e), (uint32_t)q));
+                    z[r] = D[r] * x[r];
+                }
+                warp_scatter(P, z, V, x, sc, lane, perm);
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r) xin[lane + 32 * r] = x[r];
+        }
+        // every CTA is done reading the others' totals, and xin is visible
+        cluster_sync_all();
+    }
+    // carry at the end of this warp's segment: (prefix aggregate)(carry-in)
     float S[2];
-    if (p.h0) {
+    if (G > 1 || p.h0) {
         float z[2];
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const int e = lane + 32 * r;
-            z[r] = a.D[r] * (e < p.N ? p.h0[bh * p.N + e] : 0.f);
+            z[r] = a.D[r] * (G > 1 ? xin[e] : (e < p.N ? p.h0[bh * p.N + e] : 0.f));
         }
         warp_scatter(a.P, z, a.V, S, sc, lane, perm);
     } else {
@@ -372,7 +422,7 @@ __global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p) {
     }
 #pragma unroll
     for (int r = 0; r < 2; ++r) carry[warp * 64 + lane + 32 * r] = S[r];
-    if (warp == nw - 1 && p.h_last) {
+    if (warp == nw - 1 && rank == G - 1 && p.h_last) {
 #pragma unroll
         for (int r = 0; r < 2; ++r) {
             const int e = lane + 32 * r;
@@ -385,7 +435,8 @@ __global__ void __launch_bounds__(1024, 1) k_phaseB(const ChunkParams p) {
 #pragma unroll
     for (int r = 0; r < 2; ++r) {
         const int e = lane + 32 * r;
-        x[r] = warp > 0 ? carry[(warp - 1) * 64 + e] : (p.h0 && e < p.N ? p.h0[bh * p.N + e] : 0.f);
+        x[r] = warp > 0 ? carry[(warp - 1) * 64 + e]
+                        : (G > 1 ? xin[e] : (p.h0 && e < p.N ? p.h0[bh * p.N + e] : 0.f));
     }
     for (int64_t g = c0; g < c1; g += kBGroup) {
         int TP[kBGroup][2];
@@ -457,12 +508,21 @@ cudaError_t launch_phaseC(const ChunkParams &p, pdssm_dtype dt, cudaStream_t st)
 cudaError_t launch_phaseB(const ChunkParams &p, cudaStream_t st) {
     if (p.units == 0) return cudaSuccess;
     const int nw = (int)imin64(32, p.C);
-    const size_t smem = (size_t)nw * 64 * 4 * 7 + (size_t)nw * sizeof(ScatterScratch);
+    const size_t smem =
+        (size_t)nw * 64 * 4 * 7 + (size_t)nw * sizeof(ScatterScratch) + (size_t)4 * 64 * 4;
     const int64_t BH = p.B * p.H;
-    cudaError_t e =
-        cudaFuncSetAttribute(k_phaseB, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    int dev = 0, sms = 148;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    return launch_pdl(k_phaseB, dim3((unsigned)BH), dim3(nw * 32), smem, st, p);
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
+        return e;
+    const int G = carry_scan_cluster(BH, p.C, sms);
+    e = cudaFuncSetAttribute(k_phaseB, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (G > 1)
+        return launch_cluster_pdl(k_phaseB, dim3((unsigned)(BH * G)), dim3(nw * 32), smem, G, st,
+                                  p, G);
+    return launch_pdl(k_phaseB, dim3((unsigned)BH), dim3(nw * 32), smem, st, p, G);
 }
 
 }  // namespace pdssm

@@ -666,3 +666,20 @@ def test_validate_and_clamped_indices_are_reported():
     assert pd.pdssm_ws_status(ws) == 0
     y, hl, ws = pd.pdssm_scan_fwd(bad_pi, t["k"], t["d"], t["b"], t["c"], t["h0"], chunk=16)
     assert pd.pdssm_ws_status(ws) == 3
+
+
+@pytest.mark.parametrize("N,kind,H,L,chunk", [
+    (64, "maps", 2, 16384, 16),     # 1024 chunks per sequence: clusters of 8 CTAs
+    (32, "perm", 4, 8192, 16),      # 512 chunks: clusters of 8
+    (24, "maps", 3, 6000, 20),      # 300 chunks: clusters of 4, ragged tail
+])
+def test_carry_scan_clusters(N, kind, H, L, chunk):
+    """Few sequences with many chunks: the carry scans (phase B and bwd B)
+    split each sequence over a cluster of CTAs that combine their totals
+    through distributed shared memory; the forward, h_last and every
+    gradient (g_hlast given, so the adjoint's carry starts non-zero) must
+    match the oracle."""
+    inp = small(100 + N, 1, H, L, N, 6, kind=kind)
+    check_fwd(inp, chunk)
+    rng = np.random.default_rng(N)
+    check_bwd(inp, chunk, g_hlast=rng.standard_normal((1, H, N)).astype(np.float32))
