@@ -150,7 +150,9 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
     const int64_t s = cidx * p.chunk;
     const int len = (int)imin64(p.chunk, p.L - s);
 
-    using RingT = FastRing<3, ROWB>;
+    // two tensors per stage: d, then b (pass 1) or c (pass 2) in the second
+    // slot, so a warp's ring is 2/3 of three slots and more warps fit an SM
+    using RingT = FastRing<2, ROWB>;
     float *pbuf = reinterpret_cast<float *>(wbase + kFastStages * RingT::STAGEB);
     float *lbuf = pbuf + 2 * kPbStride;
     float *hsm = lbuf + 2 * kPbStride;                // [kTS + 1][64]
@@ -158,19 +160,23 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
     ring.ring_s = smem_u32(wbase);
     ring.bar0 = smem_u32(hsm + (kTS + 1) * kMaxN);
     ring.len = len;
-    ring.nt = 3;
+    ring.nt = 2;
     const int64_t row0 = bh * p.L + s;
+    const unsigned char *src_b = reinterpret_cast<const unsigned char *>(p.b) + row0 * ROWB;
+    const unsigned char *src_c = reinterpret_cast<const unsigned char *>(p.c) + row0 * ROWB;
     ring.src[0] = reinterpret_cast<const unsigned char *>(p.d) + row0 * ROWB;
-    ring.src[1] = reinterpret_cast<const unsigned char *>(p.b) + row0 * ROWB;
-    ring.src[2] = reinterpret_cast<const unsigned char *>(p.c) + row0 * ROWB;
+    ring.src[1] = src_b;
     ring_init_bars(ring.bar0, kFastStages, lane);
 
     const int ntiles = (len + kTS - 1) / kTS;
     const int total = 2 * ntiles;   // pass 1 tiles, then pass 2 tiles (reverse)
     auto tile_of = [&](int m) { return m < ntiles ? m : 2 * ntiles - 1 - m; };
     // pass 1 stages d and b, pass 2 d and c
-    auto mask_of = [&](int m) { return m < ntiles ? 3u : 5u; };
-    for (int m = 0; m < kFastStages && m < total; ++m) ring.issue_tile(m, tile_of(m), mask_of(m), lane);
+    auto issue = [&](int m) {
+        ring.src[1] = m < ntiles ? src_b : src_c;
+        ring.issue_tile(m, tile_of(m), 3u, lane);
+    };
+    for (int m = 0; m < kFastStages && m < total; ++m) issue(m);
 
     const uint32_t map_s = smem_u32(sd.map);
     const uint32_t seg_lane = smem_u32(sd.seg) + lane * 8;
@@ -252,7 +258,7 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
                 float dv[NPL], cv[NPL], hq[NPL], hp[NPL], lam[NPL], gcv[NPL], gdv[NPL];
                 int t4[NPL];
                 lds_own<T, NPL>(row + own_off, dv);
-                lds_own<T, NPL>(row + own_off + 2 * TENS, cv);
+                lds_own<T, NPL>(row + own_off + TENS, cv);
                 lds_own<float, NPL>(hs_lane + (q + 1) * (kMaxN * 4), hq);
                 lds_own<float, NPL>(hs_lane + q * (kMaxN * 4), hp);
                 targets4<NPL>(map_s + kk * (N * 4) + lane * NPL * 4, t4);
@@ -278,8 +284,7 @@ __device__ __forceinline__ void bwdC_fast_unit(const ChunkParams &p, const SmemD
         }
         warp_barrier();
         if (m + kFastStages < total) {
-            const int mn = m + kFastStages;
-            ring.issue_tile(mn, tile_of(mn), mask_of(mn), lane);
+            issue(m + kFastStages);
         }
         // the next pass-2 tile's states (written by this lane in pass 1)
         if (m + 1 >= ntiles && m + 1 < total) load_states(tile_of(m + 1));
@@ -333,7 +338,7 @@ cudaError_t launch_bwdC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
     const int es = dt == PDSSM_BF16 ? 2 : 4;
     p.dict_content = kDictMap | kDictSeg;
     // ring, exchange buffers pb / ob and lbuf, the tile's states, barriers
-    p.smem_per_warp = (kFastStages * 3 * kTS * (int)p.N * es + kBwdFastExtraFloats * 4 +
+    p.smem_per_warp = (kFastStages * 2 * kTS * (int)p.N * es + kBwdFastExtraFloats * 4 +
                        2 * kPbStride * 4 + kFastStages * 8 + 255) / 256 * 256;
     const size_t smem = 0;
     if (dt == PDSSM_BF16)
