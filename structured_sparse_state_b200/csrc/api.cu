@@ -196,17 +196,22 @@ static pdssm_status fwd_common(const pdssm_dims *dims, const int32_t *pi_dict,
     return PDSSM_OK;
 }
 
+// look: also clear the single-pass forward's ticket counter and per-chunk
+// flags (only that kernel reads them).
 static pdssm_status run_prep(const pdssm_dims *dims, const int32_t *pi_dict,
                              int64_t pi_head_stride, const WsLayout &w, void *ws,
-                             cudaStream_t st) {
+                             cudaStream_t st, bool look) {
     unsigned char *base = reinterpret_cast<unsigned char *>(ws);
     // status word and the dictionary statistics (largest segment lane
     // distance, largest fan-in, largest window back-span)
     cudaError_t e = cudaMemsetAsync(base + w.status, 0, 16, st);
     if (e != cudaSuccess) return cuda_fail(e, "status reset");
     // the single-pass forward's ticket counter and per-chunk flags
-    e = cudaMemsetAsync(base + w.look, 0, kLookHeader + (size_t)(dims->B * dims->H * w.C) * 4, st);
-    if (e != cudaSuccess) return cuda_fail(e, "look-back reset");
+    if (look) {
+        e = cudaMemsetAsync(base + w.look, 0, kLookHeader + (size_t)(dims->B * dims->H * w.C) * 4,
+                            st);
+        if (e != cudaSuccess) return cuda_fail(e, "look-back reset");
+    }
     e = launch_prep(*dims, pi_dict, pi_head_stride, reinterpret_cast<int32_t *>(base + w.dict),
                     reinterpret_cast<uint2 *>(base + w.seg),
                     reinterpret_cast<uint2 *>(base + w.segw),
@@ -259,7 +264,7 @@ pdssm_status scan_fwd_impl(const pdssm_dims *dims, const int32_t *pi_dict, int64
     Tracer tr{trace, s};
     cudaError_t e = tr.mark("prep");
     if (e != cudaSuccess) return cuda_fail(e, "trace event");
-    st = run_prep(dims, pi_dict, pi_head_stride, w, ws, s);
+    st = run_prep(dims, pi_dict, pi_head_stride, w, ws, s, single_pass);
     if (st != PDSSM_OK) return st;
     if (dims->L == 0) {
         if (h_last) {
@@ -407,7 +412,7 @@ pdssm_status pdssm_select_scan_fwd(const pdssm_dims *dims, const void *u, pdssm_
                         "(<= 256), K <= 16, N = 32 or 64 with 16-byte aligned rows and chunk <= "
                         "1024; use pdssm_select and pdssm_scan_fwd otherwise");
     cudaStream_t s = (cudaStream_t)stream;
-    st = run_prep(dims, pi_dict, pi_head_stride, w, ws, s);
+    st = run_prep(dims, pi_dict, pi_head_stride, w, ws, s, true);
     if (st != PDSSM_OK) return st;
     p.h0 = h0;
     p.y = y;
@@ -450,7 +455,7 @@ pdssm_status pdssm_chunk_transfers(const pdssm_dims *dims, const int32_t *pi_dic
     if (dims->L > 0 && (!Pi_out || !Delta_out || !v_out))
         return arg_fail(PDSSM_ERR_INVALID_ARG, "NULL output pointer");
     cudaStream_t s = (cudaStream_t)stream;
-    st = run_prep(dims, pi_dict, pi_head_stride, w, ws, s);
+    st = run_prep(dims, pi_dict, pi_head_stride, w, ws, s, false);
     if (st != PDSSM_OK) return st;
     if (dims->L == 0) return PDSSM_OK;
     ChunkParams p = make_params(dims, w, ws, chunk, k, d, b, nullptr, in_dtype);
