@@ -163,7 +163,7 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 }
 
 // 1-D bulk copy global -> shared, completion counted on an mbarrier.  Plain
-// per-CTA copy of this GPU's own memory (no multicast).
+// per-CTA copy of this GPU's own memory, delivered to this CTA only.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes,
                                          uint32_t bar) {
     asm volatile(
