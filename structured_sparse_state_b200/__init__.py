@@ -440,8 +440,8 @@ def pdssm_ws_transfers(ws, B, H, L, N, K, chunk, per_head_dict=False, stream=Non
 
 def pdssm_wait_selftest(which: int, cap_ns: int, device=None, stream=None) -> int:
     """Runs a bounded wait that nothing completes (0: look-back flag, 1:
-    mbarrier) with the given cap; returns the status word's verdict
-    (PDSSM_ERR_TIMEOUT = 5 expected).  Synchronises."""
+    mbarrier) with the given cap; returns the status the workspace's status
+    word maps to (PDSSM_ERR_TIMEOUT = 5 expected).  Synchronises."""
     n = int(_lib.pdssm_wait_selftest_ws_bytes())
     ws = torch.empty(n, dtype=torch.uint8, device=device or "cuda")
     _check(_lib.pdssm_wait_selftest(int(which), int(cap_ns), _ptr(ws), n, _stream(stream)),
