@@ -1,0 +1,54 @@
+// Dispatch of the single-pass forward (fused.cuh) and the bounded-wait
+// self-test.
+#include "fused.cuh"
+
+namespace pdssm {
+
+// Self-test of the bounded waits (a failure made on purpose, without a
+// fault): which = 0 runs the look-back of chunk 1 of a sequence whose chunk 0
+// never publishes; which = 1 waits on an mbarrier that nothing completes.
+// Either gives up after p.wait_ns and flags PDSSM_ERR_TIMEOUT.  One warp.
+__global__ void k_wait_selftest(const ChunkParams p, int which) {
+    __shared__ __align__(16) ScatterScratch sc;
+    __shared__ __align__(8) uint64_t bar;
+    const int lane = threadIdx.x & 31;
+    if (which == 0) {
+        float x[2];
+        lookback_carry(p, 0, 1, true, sc, lane, x);
+    } else {
+        if (lane == 0) {
+            mbar_init(smem_u32(&bar), 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
+        const bool done = mbar_wait_bounded(smem_u32(&bar), 0, p.wait_ns);
+        if (!done && lane == 0) flag_status(p.status, kStTimeout);
+    }
+}
+
+cudaError_t launch_wait_selftest(const ChunkParams &p, int which, cudaStream_t st) {
+    k_wait_selftest<<<1, 32, 0, st>>>(p, which);
+    return cudaGetLastError();
+}
+
+// The single-pass forward serves the fast-path shapes (one CTA per chunk:
+// the grid must fit the launch limit).
+bool fused_path(const ChunkParams &p) { return fast_path(p) && p.units <= 0x7fffffff; }
+
+// The selection runs inside the single-pass forward for bf16 u with D_in a
+// multiple of 16 (at most 256), K <= 16, and chunks of at most 1024 steps
+// (their indices stay in shared memory).
+bool fused_select_ok(const ChunkParams &p, const void *u, const float *W) {
+    return fused_path(p) && p.D_in % 16 == 0 && p.D_in >= 16 && p.D_in <= 256 && p.K <= 16 &&
+           p.chunk <= 1024 && ((uintptr_t)u % 16) == 0 && ((uintptr_t)W % 16) == 0;
+}
+
+cudaError_t launch_scan_fused(ChunkParams p, pdssm_dtype dt, cudaStream_t st, bool select) {
+    const int es = dt == PDSSM_BF16 ? 2 : 4;
+    p.dict_content = (dt == PDSSM_BF16 ? kDictMap16 : kDictMap) | kDictSeg;
+    p.smem_per_warp = warp_smem_bytes(kFastStages, 3, (int)p.N * es);
+    if (dt == PDSSM_BF16) return select ? launch_fused_bf16_sel(p, st) : launch_fused_bf16(p, st);
+    return select ? launch_fused_f32_sel(p, st) : launch_fused_f32(p, st);
+}
+
+}  // namespace pdssm
