@@ -288,14 +288,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     pdl_wait();
     bool ok = true;
     if (warp == kTcEpiWarps) {
-        // ---- control: MMAs of tile j, then the copy of tile j + 1 into the
-        // stage tile j - 1 used
+        // ---- control: the copy of tile j + 1 into the stage tile j - 1 used
+        // (as soon as that stage is free: its product done and its norms
+        // read), then the MMAs of tile j
         if (lane == 0) {
             const uint32_t idesc = umma_idesc_bf16(NP);
             const uint32_t bbase = smem_u32(Bs);
             int j = 0;
             for (int tile = blockIdx.x; tile < p.ntiles; tile += gridDim.x, ++j) {
                 const int s = j & 1;
+                // tile j + 1 goes to the stage of tile j - 1 (the first two
+                // tiles were issued before the weight split)
+                const int next = tile + gridDim.x;
+                if (j >= 1 && next < p.ntiles) {
+                    const int sp = s ^ 1;
+                    ok = mbar_wait_bounded(bar(A_EMPTY + sp), (uint32_t)(((j - 1) >> 1) & 1)) && ok;
+                    issue_a(next, sp);
+                }
                 ok = mbar_wait_bounded(bar(A_FULL + s), (uint32_t)((j >> 1) & 1)) && ok;
                 if (j >= 2)
                     ok = mbar_wait_bounded(bar(T_EMPTY + s), (uint32_t)(((j - 2) >> 1) & 1)) && ok;
@@ -327,14 +336,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                 }
                 umma_commit(bar(T_FULL + s));
                 umma_commit(bar(A_EMPTY + s));
-                // tile j + 1 goes to the stage of tile j - 1 (the first two
-                // tiles were issued before the weight split)
-                const int next = tile + gridDim.x;
-                if (j >= 1 && next < p.ntiles) {
-                    const int sp = s ^ 1;
-                    ok = mbar_wait_bounded(bar(A_EMPTY + sp), (uint32_t)(((j - 1) >> 1) & 1)) && ok;
-                    issue_a(next, sp);
-                }
             }
         }
         __syncwarp();   // the warp reaches the final CTA barrier together
