@@ -1,35 +1,7 @@
-// Dispatch of the single-pass forward (fused.cuh) and the bounded-wait
-// self-test.
+// Dispatch of the single-pass forward (fused.cuh).
 #include "fused.cuh"
 
 namespace pdssm {
-
-// Self-test of the bounded waits (a failure made on purpose, without a
-// fault): which = 0 runs the look-back of chunk 1 of a sequence whose chunk 0
-// never publishes; which = 1 waits on an mbarrier that nothing completes.
-// Either gives up after p.wait_ns and flags PDSSM_ERR_TIMEOUT.  One warp.
-__global__ void k_wait_selftest(const ChunkParams p, int which) {
-    __shared__ __align__(16) ScatterScratch sc;
-    __shared__ __align__(8) uint64_t bar;
-    const int lane = threadIdx.x & 31;
-    if (which == 0) {
-        float x[2];
-        lookback_carry(p, 0, 1, true, sc, lane, x);
-    } else {
-        if (lane == 0) {
-            mbar_init(smem_u32(&bar), 1);
-            fence_mbar_init();
-        }
-        __syncwarp();
-        const bool done = mbar_wait_bounded(smem_u32(&bar), 0, p.wait_ns);
-        if (!done && lane == 0) flag_status(p.status, kStTimeout);
-    }
-}
-
-cudaError_t launch_wait_selftest(const ChunkParams &p, int which, cudaStream_t st) {
-    k_wait_selftest<<<1, 32, 0, st>>>(p, which);
-    return cudaGetLastError();
-}
 
 // The single-pass forward serves the fast-path shapes (one CTA per chunk:
 // the grid must fit the launch limit).

@@ -1,7 +1,8 @@
 // Forward phases A and C (three-phase forward) for a state that fills the
 // warp (N = 32 or 64) with 16-byte aligned rows, on the segment routines
-// of fwd_segments.cuh.  The general kernels in fwd.cu serve every other N
-// and unaligned rows.
+// of fwd_segments.cuh, and the bounded-wait self-test.  The general kernels
+// in fwd.cu serve every other N and unaligned rows.
+#include "fused.cuh"   // the look-back of the bounded-wait self-test
 #include "fwd_segments.cuh"
 
 namespace pdssm {
@@ -120,6 +121,33 @@ cudaError_t launch_phaseC_fast(ChunkParams p, pdssm_dtype dt, cudaStream_t st) {
                          : launch_fast(k_phaseC_fast<__nv_bfloat16, 1>, p, smem, st);
     return p.N == 64 ? launch_fast(k_phaseC_fast<float, 2>, p, smem, st)
                      : launch_fast(k_phaseC_fast<float, 1>, p, smem, st);
+}
+
+// Self-test of the bounded waits (a failure made on purpose, without a
+// fault): which = 0 runs the look-back of chunk 1 of a sequence whose chunk 0
+// never publishes; which = 1 waits on an mbarrier that nothing completes.
+// Either gives up after p.wait_ns and flags PDSSM_ERR_TIMEOUT.  One warp.
+__global__ void k_wait_selftest(const ChunkParams p, int which) {
+    __shared__ __align__(16) ScatterScratch sc;
+    __shared__ __align__(8) uint64_t bar;
+    const int lane = threadIdx.x & 31;
+    if (which == 0) {
+        float x[2];
+        lookback_carry(p, 0, 1, true, sc, lane, x);
+    } else {
+        if (lane == 0) {
+            mbar_init(smem_u32(&bar), 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
+        const bool done = mbar_wait_bounded(smem_u32(&bar), 0, p.wait_ns);
+        if (!done && lane == 0) flag_status(p.status, kStTimeout);
+    }
+}
+
+cudaError_t launch_wait_selftest(const ChunkParams &p, int which, cudaStream_t st) {
+    k_wait_selftest<<<1, 32, 0, st>>>(p, which);
+    return cudaGetLastError();
 }
 
 }  // namespace pdssm
