@@ -511,30 +511,32 @@ def test_segment_step_shuffle_levels(N, fan, levels, dtype):
     check_bwd(inp, chunk=64)
 
 
+@pytest.mark.parametrize("per_head", [False, True])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("case", ["mixed_fan_in", "no_single_source", "pairs_only",
                                   "fan_in_seven"])
-def test_window_step_dictionaries(case, dtype):
+def test_window_step_dictionaries(case, dtype, per_head):
     """N = 64 dictionaries around the window table's limits: maps mixing
     fan-ins 2 to 6 with single-source targets to move in front of
     misaligned even-sized segments, maps with no single-source target at
     all, maps whose targets all have two sources (no segment crosses a
     lane), and maps with one target of fan-in 7 (a back-span of three
-    lanes: the segment scan takes over)."""
+    lanes: the segment scan takes over); shared by all heads, or one
+    dictionary per head (each warp stages its head's tables)."""
     sizes = {"mixed_fan_in": [6, 5, 4, 4, 3, 2, 2],
              "no_single_source": [6, 5, 5, 4, 4, 3, 3] + [2] * 17,
              "pairs_only": [2] * 32,
              "fan_in_seven": [7, 3, 2]}[case]
     sizes = sizes + [1] * (64 - sum(sizes))
     rng = np.random.default_rng(len(case))
-    inp = small(90 + len(case), 2, 2, 333, 64, 6, dtype=dtype)
+    inp = small(90 + len(case), 2, 2, 333, 64, 6, dtype=dtype, per_head=per_head)
     rows = []
-    for _ in range(inp.pi.shape[0]):
+    for _ in range(inp.pi.size // 64):
         targets = rng.permutation(64)[:len(sizes)]
         row = np.concatenate([[t] * f for t, f in zip(targets, sizes)])
         rows.append(row[rng.permutation(64)].astype(np.int32))
-    inp.pi = np.stack(rows)
-    spans = [_window_span(r) for r in inp.pi]
+    inp.pi = np.stack(rows).reshape(inp.pi.shape)
+    spans = [_window_span(r) for r in inp.pi.reshape(-1, 64)]
     assert all(sp is not None and sp <= 2 for sp in spans) == (case != "fan_in_seven"), spans
     check_fwd(inp, chunk=64)
     check_fwd(inp, chunk=128)
